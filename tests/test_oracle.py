@@ -1,0 +1,247 @@
+"""Pins of the CPU oracle against the mathematics (closed forms, brute force, library
+routines, invariants).  No GPU needed."""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import pbsa_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def geom(fh=16, fw=24, th=8, tw=8, d=8):
+    return {"frame_h": fh, "frame_w": fw, "tile_h": th, "tile_w": tw, "scale": 1.0 / math.sqrt(d)}
+
+
+# ------------------------------------------------------------------ representatives
+@pytest.mark.parametrize("th,tw", [(8, 8), (4, 16), (16, 4)])
+def test_block_reps_closed_form(th, tw):
+    g = geom(16, 32, th, tw)
+    n_frames, H, d = 2, 3, 4
+    fh, fw = g["frame_h"], g["frame_w"]
+    x = np.zeros((n_frames * fh * fw, H, d))
+    for f in range(n_frames):
+        for y in range(fh):
+            for xx in range(fw):
+                t = f * fh * fw + y * fw + xx
+                for h in range(H):
+                    x[t, h, :] = f * 1000 + y * fw + xx + 0.5 * h + 0.25 * np.arange(d)
+    reps = O.block_reps(x, g, n_frames)
+    tpr, bpf = fw // tw, (fh // th) * (fw // tw)
+    assert reps.shape == (H, n_frames * bpf, d)
+    for b in range(n_frames * bpf):
+        f, rem = divmod(b, bpf)
+        ty, tx = divmod(rem, tpr)
+        # mean of y over the tile rows and of x over the tile columns
+        my, mx = ty * th + (th - 1) / 2, tx * tw + (tw - 1) / 2
+        for h in range(H):
+            want = f * 1000 + my * fw + mx + 0.5 * h + 0.25 * np.arange(d)
+            np.testing.assert_allclose(reps[h, b], want, rtol=0, atol=1e-9)
+
+
+def test_block_rows_cover_frame_once():
+    g = geom(32, 48)
+    seen = np.concatenate([O.block_token_rows(32, 48, 8, 8, b) for b in range(2 * 24)])
+    assert sorted(seen.tolist()) == list(range(2 * 32 * 48))
+
+
+# ------------------------------------------------------------------ selection
+def test_topk_ties_go_to_lower_id():
+    scores = np.zeros(10, np.float32)
+    gids = [17, 3, 9, 11, 4, 8, 30, 1, 2, 5]
+    got = [gids[i] for i in O.topk_select(scores, gids, 4)]
+    assert got == [1, 2, 3, 4]
+
+
+def test_topk_brute_force_and_permutation():
+    rng = np.random.default_rng(0)
+    for trial in range(50):
+        n, k = int(rng.integers(1, 9)), int(rng.integers(1, 6))
+        sc = rng.integers(-3, 3, n).astype(np.float32)  # many exact ties
+        gids = rng.permutation(100)[:n].tolist()
+        sel = {gids[i] for i in O.topk_select(sc, gids, k)}
+        # brute force: the chosen set is the lexicographically best k-subset under
+        # (score desc, gid asc) -- every chosen one beats every unchosen one
+        best = None
+        for comb in itertools.combinations(range(n), min(k, n)):
+            key = sorted(((-float(sc[i]), gids[i]) for i in comb))
+            if best is None or key < best[0]:
+                best = (key, {gids[i] for i in comb})
+        assert sel == best[1]
+        perm = rng.permutation(n)
+        sel2 = {gids[perm[i]] for i in O.topk_select(sc[perm], [gids[j] for j in perm], k)}
+        assert sel2 == sel
+
+
+# ------------------------------------------------------------------ attention
+def _sdpa64(q, k, v, scale):
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float64))[None, None]
+    return torch.nn.functional.scaled_dot_product_attention(t(q), t(k), t(v), scale=scale)[0, 0].numpy()
+
+
+def test_all_blocks_selected_is_dense_attention():
+    g = geom(16, 16, 8, 8, d=64)
+    rng = np.random.default_rng(1)
+    hist, chunk, H, d = 6, 1, 2, 64
+    q = rng.standard_normal((chunk * 256, H, d))
+    k = rng.standard_normal((hist * 256, H, d))
+    v = rng.standard_normal((hist * 256, H, d))
+    # capacity holds sinks + every middle block, top-k takes the whole window
+    plan = O.single_step_plan(q, k, g, hist, chunk, capacity=4 + 12, window=2, topk=8, gamma=0.9)
+    for h in range(H):
+        for r in range(4):
+            gids = plan["P"][h] + plan["sel"][h][r]
+            assert sorted(gids) == list(range(24))
+            out, lse = O.attend_gids(q, k, v, g, h, r, gids, q_first_frame=hist)
+            qb = O.block_tokens(q, g, hist * 4 + r, hist)[:, h]
+            ref = _sdpa64(qb, k[:, h], v[:, h], g["scale"])
+            np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+            logits = g["scale"] * qb @ k[:, h].T
+            np.testing.assert_allclose(lse, torch.logsumexp(torch.from_numpy(logits), 1).numpy(),
+                                       rtol=0, atol=1e-12)
+
+
+def test_softmax_rows_sum_to_one_and_convex_hull():
+    rng = np.random.default_rng(2)
+    n, m = 5, 12
+    q = rng.standard_normal((n, 7)) * 3
+    k = rng.standard_normal((m, 7)) * 3
+    eye = np.eye(m)
+    p, _ = O.attention(q, k, eye, 0.5)          # V = identity -> out is the softmax matrix
+    np.testing.assert_allclose(p.sum(axis=1), 1.0, atol=1e-14)
+    assert (p > 0).all()
+    v = rng.standard_normal((m, 3))
+    out, _ = O.attention(q, k, v, 0.5)
+    assert (out <= v.max(axis=0) + 1e-12).all() and (out >= v.min(axis=0) - 1e-12).all()
+    perm = rng.permutation(m)
+    out2, _ = O.attention(q, k[perm], v[perm], 0.5)
+    np.testing.assert_allclose(out, out2, atol=1e-13)
+
+
+def test_empty_key_set():
+    out, lse = O.attention(np.ones((3, 4)), np.zeros((0, 4)), np.zeros((0, 4)), 1.0)
+    assert (out == 0).all() and np.isneginf(lse).all()
+
+
+# ------------------------------------------------------------------ backward
+def test_backward_finite_differences():
+    rng = np.random.default_rng(3)
+    n, m, d = 4, 6, 5
+    q, k, v, do = (rng.standard_normal(s) for s in ((n, d), (m, d), (m, d), (n, d)))
+    scale = 0.7
+    dq, dk, dv = O.attention_bwd(q, k, v, do, scale)
+    f = lambda q_, k_, v_: float((O.attention(q_, k_, v_, scale)[0] * do).sum())
+    eps = 1e-6
+    for name, a, g_ in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        num = np.zeros_like(a)
+        for idx in np.ndindex(a.shape):
+            ap, am = a.copy(), a.copy()
+            ap[idx] += eps
+            am[idx] -= eps
+            args_p = {"q": q, "k": k, "v": v}
+            args_m = dict(args_p)
+            args_p[name], args_m[name] = ap, am
+            num[idx] = (f(args_p["q"], args_p["k"], args_p["v"])
+                        - f(args_m["q"], args_m["k"], args_m["v"])) / (2 * eps)
+        np.testing.assert_allclose(g_, num, rtol=1e-6, atol=1e-8)
+
+
+# ------------------------------------------------------------------ memory update
+def test_memory_update_closed_form():
+    fx = json.load(open(os.path.join(GOLDEN, "memory_update_closed_form.json")))
+    prev = [np.nan if p is None else p for p in fx["prev_ema"]]
+    ema, keep, a = O.memory_update(np.array(fx["q_reps"]), np.array(fx["pool_reps"]), fx["pool_gids"],
+                                   prev, fx["is_sink"], 1.0, fx["gamma"], fx["capacity"])
+    np.testing.assert_allclose(a, fx["expected_a"], atol=1e-15)
+    np.testing.assert_allclose(ema, fx["expected_ema"], atol=1e-15)
+    assert keep.tolist() == fx["expected_keep"]
+
+
+def test_memory_update_invariants():
+    rng = np.random.default_rng(4)
+    for trial in range(30):
+        nq, nb, d = int(rng.integers(1, 6)), int(rng.integers(2, 30)), 8
+        n_sink = int(rng.integers(0, min(nb, 5) + 1))
+        C = int(rng.integers(n_sink, nb + 3))
+        qr, pr = rng.standard_normal((nq, d)), rng.standard_normal((nb, d))
+        gids = rng.permutation(1000)[:nb].tolist()
+        sink = [i < n_sink for i in range(nb)]
+        prev = np.where(rng.random(nb) < 0.5, np.nan, rng.random(nb) * 0.1)
+        ema, keep, a = O.memory_update(qr, pr, gids, prev, sink, 0.3, 0.9, C)
+        assert abs(a.sum() - 1.0) < 1e-12
+        assert keep.sum() <= C and all(keep[i] for i in range(n_sink))
+        if C >= nb:
+            assert keep.all()
+        dropped = [ema[i] for i in range(nb) if not keep[i]]
+        kept_ns = [ema[i] for i in range(nb) if keep[i] and not sink[i]]
+        if dropped and kept_ns:
+            assert min(kept_ns) >= max(dropped)
+    # a constant score stream is a fixed point of the EMA
+    qr, pr = rng.standard_normal((3, 8)), rng.standard_normal((5, 8))
+    _, _, a = O.memory_update(qr, pr, list(range(5)), [np.nan] * 5, [False] * 5, 0.3, 0.9, 5)
+    ema, _, _ = O.memory_update(qr, pr, list(range(5)), a, [False] * 5, 0.3, 0.9, 5)
+    np.testing.assert_allclose(ema, a, atol=1e-15)
+
+
+def test_memory_update_equal_ema_ties_to_lower_id():
+    pr = np.zeros((4, 2))
+    ema, keep, _ = O.memory_update(np.ones((1, 2)), pr, [9, 7, 8, 6], [np.nan] * 4,
+                                   [False] * 4, 1.0, 0.9, 2)
+    assert {g for g, kp in zip([9, 7, 8, 6], keep) if kp} == {6, 7}
+
+
+# ------------------------------------------------------------------ workload plans
+def test_rollout_windows_and_capacity_5s():
+    """5 s rollout shapes: 24 blocks/frame, chunks of 3 frames, W = 6, C = 96."""
+    g = geom(32, 48, 8, 8, d=4)
+    ro = O.RolloutOracle(g, heads=1, capacity=96, window=6, topk=32, gamma=0.9)
+    rng = np.random.default_rng(5)
+    local_sizes, p_sizes, evicted = [], [], []
+    for c in range(7):
+        f0 = 3 * c
+        local_sizes.append(len(ro.local()))
+        q = rng.standard_normal((1, 72, 4))
+        sel = ro.select(q)
+        if c == 0:
+            assert sel is None
+        else:
+            assert len(sel[0][0][0]) == len(ro.P[0]) + min(32, len(ro.local()))
+        ev = ro.commit(f0, 3, rng.standard_normal((1, 72, 4)), q)
+        evicted.append(sorted({b // 24 for b in ev}))
+        p_sizes.append(len(ro.P[0]))
+        assert set(range(24)) <= set(ro.P[0]) and len(ro.P[0]) <= 96
+    assert local_sizes == [0, 48, 120, 144, 144, 144, 144]
+    assert evicted == [[], [], [1, 2], [3, 4, 5], [6, 7, 8], [9, 10, 11], [12, 13, 14]]
+    assert p_sizes[:3] == [24, 24, 72] and all(p == 96 for p in p_sizes[3:])
+
+
+def test_single_step_partition_5s():
+    """Last-chunk decode of the 5 s video: 18 history frames = 24 sinks + 264 middle + 144 local."""
+    g = geom(32, 48, 8, 8, d=4)
+    q = np.random.default_rng(6).standard_normal((3 * 1536, 1, 4))
+    k = np.random.default_rng(7).standard_normal((18 * 1536, 1, 4))
+    plan = O.single_step_plan(q, k, g, 18, 3, capacity=96, window=6, topk=32, gamma=0.9,
+                              k_chunk=np.zeros(1))
+    assert len(plan["sinks"]) == 24 and len(plan["middle"]) == 264 and len(plan["local"]) == 144
+    assert plan["local"][0] == 12 * 24 and plan["middle"][-1] == 12 * 24 - 1
+    assert len(plan["P"][0]) == 96 and set(range(24)) <= set(plan["P"][0])
+    assert all(len(s) == 32 and set(s) <= set(plan["local"]) for s in plan["sel"][0])
+    assert len(plan["P2"][0]) == 96
+
+
+def test_train_masks_shape():
+    g = geom(16, 16, 8, 8, d=4)      # 4 blocks per frame
+    rng = np.random.default_rng(8)
+    q = rng.standard_normal((1, 9 * 256, 1, 4))
+    k = rng.standard_normal((1, 9 * 256, 1, 4))
+    masks, _ = O.train_masks(q, k, g, 9, 3, topk=2)
+    m = masks[0][0]
+    assert m[0] == list(range(12))
+    assert len(m[12]) == 4 + 2 + 12 and set(m[12][:4]) == set(range(4))
+    assert set(m[12][4:6]) <= set(range(4, 12))
+    assert set(m[30][4:6]) <= set(range(4, 24))
