@@ -1,0 +1,275 @@
+"""Per-layer PBSA KV cache in HBM and its host-side bookkeeping.
+
+Sparse Forcing (gist.science English page, 2.B "Structured Memory Decomposition"): the KV
+cache of a layer is the persistent memory P_t (capacity C: the sink blocks of frame 0
+plus the best-scored older blocks, shared by all diffusion steps of a chunk) and the
+local window L_t (the last W frames, frame 0 excluded).  This module owns the device
+buffers of one layer and sequences the C-ABI calls; every number is computed by the
+library's kernels.
+
+Pool layout (slots of 64 tokens, per head): ``[0, C)`` persistent slots, then a ring of
+``W + chunk_frames`` frames (frame f -> ring position f mod (W + chunk_frames)), then an
+optional staging area used only by ``prefill``.  The ring holds the window plus the
+chunk being committed, so the blocks leaving the window are still intact while the
+memory update scores and copies them.
+"""
+from __future__ import annotations
+
+import dataclasses
+
+import torch
+
+from . import _lib as L
+
+
+@dataclasses.dataclass(frozen=True)
+class LayerConfig:
+    heads: int
+    head_dim: int
+    frame_h: int
+    frame_w: int
+    tile_h: int
+    tile_w: int
+    capacity: int
+    window_frames: int
+    chunk_frames: int
+    topk: int
+    gamma: float
+    dtype: str = "bf16"           # "bf16" or "f32"
+    staging_blocks: int = 0       # extra slots for prefill (history beyond the ring)
+    scale: float | None = None
+
+    @property
+    def bpf(self) -> int:
+        return (self.frame_h // self.tile_h) * (self.frame_w // self.tile_w)
+
+    @property
+    def tpf(self) -> int:
+        return self.frame_h * self.frame_w
+
+
+class PBSALayerCache:
+    def __init__(self, cfg: LayerConfig, device="cuda"):
+        self.cfg = cfg
+        self.device = torch.device(device)
+        self.geom = L.make_geom(cfg.heads, cfg.head_dim, cfg.frame_h, cfg.frame_w, cfg.tile_h,
+                                cfg.tile_w, cfg.scale or cfg.head_dim ** -0.5, cfg.dtype)
+        self.tdtype = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+        H, d, bpf, C = cfg.heads, cfg.head_dim, cfg.bpf, cfg.capacity
+        self.ring_frames = cfg.window_frames + cfg.chunk_frames
+        self.ring_base = C
+        self.stage_base = C + self.ring_frames * bpf
+        self.pool_slots = self.stage_base + cfg.staging_blocks
+        dev = self.device
+        self.k_pool = torch.zeros((H, self.pool_slots, 64, d), dtype=self.tdtype, device=dev)
+        self.v_pool = torch.zeros_like(self.k_pool)
+        self.k_reps = torch.zeros((H, self.pool_slots, d), dtype=torch.float32, device=dev)
+        self.slot_gid = torch.full((H, C), -1, dtype=torch.int32, device=dev)
+        self.slot_ema = torch.zeros((H, C), dtype=torch.float32, device=dev)
+        self.p_list = torch.zeros((H, C), dtype=torch.int32, device=dev)
+        self.p_cnt = torch.zeros((H,), dtype=torch.int32, device=dev)
+        nq = cfg.chunk_frames * bpf
+        self.max_pool_entries = C + max(self.ring_frames * bpf, cfg.staging_blocks)
+        self.ws = torch.zeros(L.pbsa_workspace_bytes(self.geom, nq, self.max_pool_entries),
+                              dtype=torch.uint8, device=dev)
+        self.kv_ld = C + max(cfg.topk, 0)
+        self.kv_ld_own = max(self.kv_ld, nq)
+        # flat buffers, viewed per call as [H, nq, ...] for chunks of up to chunk_frames frames
+        self._q_reps_buf = torch.zeros(H * nq * d, dtype=torch.float32, device=dev)
+        self._kv_slot_buf = torch.zeros(H * nq * self.kv_ld_own, dtype=torch.int32, device=dev)
+        self._kv_cnt_buf = torch.zeros(H * nq, dtype=torch.int32, device=dev)
+        self.q_reps = self._q_reps_buf.view(H, nq, d)
+        self.kv_slot = self._kv_slot_buf.view(H, nq, self.kv_ld_own)
+        self.kv_cnt = self._kv_cnt_buf.view(H, nq)
+        self.hist = 0
+        self._cand = None      # (cand_slot, cand_gid, n) of the current local window
+        self._dst_cache = {}
+
+    # ------------------------------------------------------------------ layout helpers
+    def ring_slot(self, frame: int, tile: int) -> int:
+        return self.ring_base + (frame % self.ring_frames) * self.cfg.bpf + tile
+
+    def window_frames(self, hist: int | None = None) -> list[int]:
+        h = self.hist if hist is None else hist
+        return list(range(max(1, h - self.cfg.window_frames), h))
+
+    def _ints(self, rows) -> torch.Tensor:
+        t = torch.tensor(rows, dtype=torch.int32).pin_memory()
+        return t.to(self.device, non_blocking=True)
+
+    def _frames_dst(self, first: int, n: int) -> torch.Tensor:
+        key = (first % self.ring_frames, n)
+        if key not in self._dst_cache:
+            bpf = self.cfg.bpf
+            self._dst_cache[key] = self._ints(
+                [self.ring_slot(first + f, t) for f in range(n) for t in range(bpf)])
+        return self._dst_cache[key]
+
+    def _refresh_window(self):
+        bpf, H = self.cfg.bpf, self.cfg.heads
+        frames = self.window_frames()
+        slots = [self.ring_slot(f, t) for f in frames for t in range(bpf)]
+        gids = [f * bpf + t for f in frames for t in range(bpf)]
+        n = len(slots)
+        if n == 0:
+            self._cand = (None, None, 0)
+            return
+        self._cand = (self._ints([slots] * H).view(H, n), self._ints([gids] * H).view(H, n), n)
+
+    @property
+    def kv_bytes(self) -> int:
+        """Bytes of K and V held for the persistent memory and the ring (prefill staging excluded)."""
+        c = self.cfg
+        slots = c.capacity + self.ring_frames * c.bpf
+        return 2 * c.heads * slots * 64 * c.head_dim * self.k_pool.element_size()
+
+    # ------------------------------------------------------------------ the hot path
+    def frames_of(self, x: torch.Tensor) -> int:
+        n, rem = divmod(x.shape[0], self.cfg.tpf)
+        if rem or not 0 < n <= self.cfg.chunk_frames:
+            raise ValueError(f"a chunk holds 1..{self.cfg.chunk_frames} whole frames, got {x.shape[0]} tokens")
+        return n
+
+    def query_reps(self, q: torch.Tensor, stream=None) -> torch.Tensor:
+        """a1: representatives of the chunk's query blocks -> self.q_reps [H, nq, d]."""
+        c = self.cfg
+        nq = self.frames_of(q) * c.bpf
+        self.q_reps = self._q_reps_buf[:c.heads * nq * c.head_dim].view(c.heads, nq, c.head_dim)
+        L.pbsa_blockify(self.geom, q, nq // c.bpf, self.q_reps, nq, ws=self.ws, stream=stream)
+        return self.q_reps
+
+    def select(self, q_reps: torch.Tensor, stream=None):
+        """a2: per query block, persistent slots + top-k local slots -> (kv_slot, kv_cnt, kv_ld)."""
+        c = self.cfg
+        nq = q_reps.shape[1]
+        self.kv_slot = self._kv_slot_buf[:c.heads * nq * self.kv_ld_own].view(c.heads, nq, self.kv_ld_own)
+        self.kv_cnt = self._kv_cnt_buf[:c.heads * nq].view(c.heads, nq)
+        cs, cg, n = self._cand
+        if n == 0:
+            # no local window yet: persistent slots only (score_select with no candidates)
+            L.pbsa_score_select(self.geom, q_reps, nq, self.k_reps, self.pool_slots, None, None, 0, 0,
+                                self.p_list, self.p_cnt, c.capacity, self.kv_slot, self.kv_cnt,
+                                self.kv_ld_own, ws=self.ws, stream=stream)
+        else:
+            L.pbsa_score_select(self.geom, q_reps, nq, self.k_reps, self.pool_slots, cs, cg, n, c.topk,
+                                self.p_list, self.p_cnt, c.capacity, self.kv_slot, self.kv_cnt,
+                                self.kv_ld_own, ws=self.ws, stream=stream)
+        return self.kv_slot, self.kv_cnt, self.kv_ld_own
+
+    def attend(self, q, kv_slot, kv_cnt, kv_ld, o=None, lse=None, stream=None):
+        """a3: fine attention over the listed slots."""
+        if o is None:
+            o = torch.empty_like(q)
+        L.pbsa_attend(self.geom, q, self.frames_of(q), self.k_pool, self.v_pool, self.pool_slots,
+                      kv_slot, kv_cnt, kv_ld, o, lse, ws=self.ws, stream=stream)
+        return o
+
+    def decode_step(self, q, k=None, v=None, o=None, lse=None, stream=None):
+        """One denoising step of the current chunk: returns O (raster, like q).
+
+        With an empty history the chunk attends its own blocks (``k``, ``v`` of this step,
+        written to the chunk's ring positions); otherwise P_t + top-k of L_t.
+        """
+        if self._cand is None:
+            self._refresh_window()
+        q_reps = self.query_reps(q, stream)
+        if self.hist == 0:
+            if k is None or v is None:
+                raise ValueError("the first chunk attends its own blocks: pass its k and v")
+            self._write_chunk(k, v, stream)
+            nq = q_reps.shape[1]
+            own = self._ints([[self.ring_slot(b // self.cfg.bpf, b % self.cfg.bpf) for b in range(nq)]] * nq)
+            kv_slot = torch.zeros((self.cfg.heads, nq, nq), dtype=torch.int32, device=self.device)
+            kv_slot[:] = own.view(nq, nq)
+            kv_cnt = torch.full((self.cfg.heads, nq), nq, dtype=torch.int32, device=self.device)
+            return self.attend(q, kv_slot, kv_cnt, nq, o, lse, stream)
+        kv_slot, kv_cnt, kv_ld = self.select(q_reps, stream)
+        return self.attend(q, kv_slot, kv_cnt, kv_ld, o, lse, stream)
+
+    def _write_chunk(self, k, v, stream=None):
+        n = self.frames_of(k)
+        dst = self._frames_dst(self.hist, n)
+        L.pbsa_blockify(self.geom, k, n, self.k_reps, self.pool_slots, dst, self.k_pool,
+                        self.pool_slots, ws=self.ws, stream=stream)
+        L.pbsa_blockify(self.geom, v, n, self._v_reps_sink(), self.pool_slots, dst,
+                        self.v_pool, self.pool_slots, ws=self.ws, stream=stream)
+
+    def _v_reps_sink(self) -> torch.Tensor:
+        # value representatives are not used by the method; blockify still writes them
+        if not hasattr(self, "_vreps"):
+            self._vreps = torch.empty_like(self.k_reps)
+        return self._vreps
+
+    def commit(self, k, v, q_reps_last=None, stream=None):
+        """a4: commit the finished chunk (its last-step K, V) and update the persistent memory.
+
+        The chunk's blocks enter the ring; the frames that leave the window, and frame 0's
+        sink blocks when frame 0 is in the chunk, are the candidates of the memory update,
+        scored by the chunk's last-step query representatives.
+        """
+        c = self.cfg
+        bpf, H = c.bpf, c.heads
+        q_reps_last = self.q_reps if q_reps_last is None else q_reps_last
+        first, n = self.hist, self.frames_of(k)
+        self._write_chunk(k, v, stream)
+        old_win = set(self.window_frames(first))
+        new_hist = first + n
+        new_win = set(self.window_frames(new_hist))
+        entering = {f for f in range(first, new_hist) if f != 0}
+        evicted = sorted((old_win | entering) - new_win)
+        cand = [(self.ring_slot(f, t), f * bpf + t) for f in evicted for t in range(bpf)]
+        if first == 0:
+            cand = [(self.ring_slot(0, t), t) for t in range(bpf)] + cand
+        self._update(q_reps_last, cand, stream)
+        self.hist = new_hist
+        self._refresh_window()
+
+    def _update(self, q_reps, cand, stream=None):
+        c, H = self.cfg, self.cfg.heads
+        ncand = len(cand)
+        if ncand:
+            cs = self._ints([[s for s, _ in cand]] * H).view(H, ncand)
+            cg = self._ints([[g for _, g in cand]] * H).view(H, ncand)
+        else:
+            cs = cg = None
+        L.pbsa_memory_update(self.geom, q_reps, q_reps.shape[1], self.k_reps, self.k_pool, self.v_pool,
+                             self.pool_slots, self.slot_gid, self.slot_ema, c.capacity, c.bpf, cs, cg,
+                             ncand, c.gamma, self.p_list, self.p_cnt, ws=self.ws, stream=stream)
+
+    def prefill(self, k_hist, v_hist, hist_frames: int, q_reps, stream=None):
+        """Load a history of ``hist_frames`` frames at once (single-step decode workloads).
+
+        The sinks and every middle frame (older than the window) go to the staging area and
+        one memory update with no prior EMA selects the persistent set among them, scored by
+        ``q_reps``; the window frames go to their ring positions.
+        """
+        c = self.cfg
+        bpf = c.bpf
+        win = self.window_frames(hist_frames)
+        middle = list(range(1, win[0] if win else hist_frames))
+        staged = [0] + middle
+        if len(staged) * bpf > c.staging_blocks:
+            raise ValueError(f"prefill needs {len(staged) * bpf} staging blocks, have {c.staging_blocks}")
+        dst = []
+        for f in range(hist_frames):
+            for t in range(bpf):
+                dst.append(self.stage_base + staged.index(f) * bpf + t if f in staged else self.ring_slot(f, t))
+        dst_t = self._ints(dst)
+        L.pbsa_blockify(self.geom, k_hist, hist_frames, self.k_reps, self.pool_slots, dst_t, self.k_pool,
+                        self.pool_slots, ws=self.ws, stream=stream)
+        L.pbsa_blockify(self.geom, v_hist, hist_frames, self._v_reps_sink(), self.pool_slots, dst_t,
+                        self.v_pool, self.pool_slots, ws=self.ws, stream=stream)
+        cand = [(self.stage_base + i * bpf + t, f * bpf + t) for i, f in enumerate(staged) for t in range(bpf)]
+        self._update(q_reps, cand, stream)
+        self.hist = hist_frames
+        self._refresh_window()
+
+    # ------------------------------------------------------------------ inspection
+    def persistent_gids(self) -> list[set[int]]:
+        g = self.slot_gid.cpu()
+        return [set(int(x) for x in row if x >= 0) for row in g]
+
+    def slot_to_gid(self) -> dict[int, int]:
+        """Map of ring/stage slots to global block ids for the current window (host bookkeeping)."""
+        bpf = self.cfg.bpf
+        return {self.ring_slot(f, t): f * bpf + t for f in self.window_frames() for t in range(bpf)}

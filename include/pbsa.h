@@ -1,0 +1,163 @@
+/*
+ * pbsa.h -- C ABI of the PBSA (Persistent Block-Sparse Attention) library, libpbsa.so.
+ *
+ * The method is the attention hot path of "Sparse Forcing: Native Trainable Sparse
+ * Attention for Real-time Autoregressive Diffusion Video Generation" (gist.science,
+ * English explainer, section 2 "Methodology": B "Structured Memory Decomposition",
+ * C "Persistent Block-Sparse Attention (PBSA)", E "System Implementation: PBSA Kernel").
+ * The KV cache of one attention layer is split into a persistent memory of capacity C
+ * (sink blocks plus the best-scored older blocks) and a sliding local window.  Every
+ * query block attends, in one softmax, to the persistent blocks plus its top-k local
+ * blocks, chosen by coarse scores between mean-pooled block representatives; after a
+ * chunk is finished the persistent memory is re-scored and updated in place.
+ *
+ * Conventions (all entry points)
+ *  - Every pointer argument is a DEVICE pointer owned by the caller, except the geometry
+ *    struct, which is host memory read during the call.  The library never allocates
+ *    device memory and keeps no pointer after a call returns.
+ *  - All calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and run on the current CUDA device.
+ *  - Shape and scalar errors are detected on the host and returned synchronously as
+ *    PBSA_ERR_INVALID_ARG (bad value) or PBSA_ERR_UNSUPPORTED (valid but not built);
+ *    nothing is launched in that case.  A failed launch returns PBSA_ERR_CUDA.
+ *  - Bad data found on the device (a slot id outside the pool) is skipped and recorded in
+ *    the workspace's error word; pbsa_get_device_error() reports it.  A wait inside a
+ *    kernel that exceeds its bound records PBSA_ERR_TIMEOUT the same way and the kernel
+ *    returns.  No call traps, asserts or exits.
+ *  - Token tensors are raster order [T][H][d] (T = frames * frame_h * frame_w, token
+ *    t = frame*frame_h*frame_w + y*frame_w + x), in the geometry's dtype.
+ *  - A block is 1 frame x (tile_h x tile_w) = 64 tokens.  Global block id of tile
+ *    (ty, tx) of frame f is f*bpf + ty*(frame_w/tile_w) + tx, bpf = blocks per frame.
+ *    Inside a block, token (ly, lx) is row ly*tile_w + lx.
+ *  - A pool is the block-major KV cache of one layer: [H][pool_slots][64][d] in the
+ *    geometry's dtype; k_reps is [H][pool_slots][d] fp32.  Slots 0..C-1 are the persistent
+ *    memory; the caller places the local window and any staging area after them.
+ */
+#ifndef PBSA_H
+#define PBSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PBSA_API __attribute__((visibility("default")))
+#else
+#define PBSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PBSA_OK = 0,
+  PBSA_ERR_INVALID_ARG = 1,
+  PBSA_ERR_UNSUPPORTED = 2,
+  PBSA_ERR_CUDA = 3,
+  PBSA_ERR_TIMEOUT = 4,
+  PBSA_ERR_DEVICE_INDEX = 5
+} pbsa_status;
+
+typedef enum { PBSA_F32 = 0, PBSA_BF16 = 1 } pbsa_dtype;
+
+/* Geometry of one attention layer.  tile_h*tile_w must be 64; frame_h, frame_w must be
+ * multiples of tile_h, tile_w; head_dim a multiple of 32 and <= 128 (bf16 needs 128). */
+typedef struct {
+  int heads;      /* H */
+  int head_dim;   /* d */
+  int frame_h;    /* latent tokens per frame, vertically */
+  int frame_w;    /* latent tokens per frame, horizontally */
+  int tile_h;     /* block tile height (tokens) */
+  int tile_w;     /* block tile width (tokens) */
+  float scale;    /* softmax and coarse-score scale, normally 1/sqrt(d) */
+  int dtype;      /* pbsa_dtype of token tensors and pools */
+} pbsa_geom;
+
+/* Bytes of device workspace needed by calls with at most `max_q_blocks` query blocks and
+ * at most `max_pool_entries` (= C + candidates) entries in a memory update.  The first
+ * 256 bytes hold the device error word; the caller zero-fills the workspace once before
+ * first use.  One workspace must not be used by two calls that overlap in time. */
+PBSA_API size_t pbsa_workspace_bytes(const pbsa_geom* g, int max_q_blocks, int max_pool_entries);
+
+/* a1 -- blockify: mean-pooled representatives, and optionally a block-major copy.
+ * (Chinese explainer 2.2 "blockified compression"; English 2.E "blockifying the latent
+ * space, enabling coalesced reads".)
+ *  x        [n_frames*frame_h*frame_w][H][d] raster, geometry dtype.
+ *  reps     out [H][rep_slots][d] fp32: reps[h][slot(b)] = mean of block b's 64 tokens.
+ *  dst_slot nullable [n_frames*bpf]: slot of local block b (b = f*bpf + tile); NULL means
+ *           slot b.  Slots must be < rep_slots (and < pool_slots when pool is given).
+ *  pool     nullable out [H][pool_slots][64][d]: block b's tokens are copied to slot(b).
+ * Fully overwrites the destination rows; reads nothing else. */
+PBSA_API pbsa_status pbsa_blockify(const pbsa_geom* g, const void* x, int n_frames,
+                          float* reps, int rep_slots, const int* dst_slot,
+                          void* pool, int pool_slots, void* ws, void* stream);
+
+/* a2 -- coarse score + top-k: for each head h and query block r,
+ *   score(r, c) = scale * <q_reps[h][r], k_reps[h][cand_slot[h][c]]>  (fp32)
+ * and the k best candidates (score descending, ties to the lower cand_gid, then the lower
+ * position c).  (English 2.C "Local Sparsity": top-K local blocks from compressed block
+ * representatives.)  The output row is the optional prefix followed by the selection:
+ *   out_slot[h][r][0..pc)      = prefix_slot[h][0..pc),  pc = prefix_cnt ? prefix_cnt[h] : 0
+ *   out_slot[h][r][pc + i]     = cand_slot of the i-th best candidate, i < min(k, ncand)
+ *   out_cnt[h][r]              = pc + min(k, ncand)
+ *   out_score[h][r][i]         = its score (nullable)
+ *  q_reps [H][nq][d]; k_reps [H][pool_slots][d]; cand_slot, cand_gid [H][ncand];
+ *  prefix_slot [H][prefix_ld]; out_slot [H][nq][out_ld] with out_ld >= prefix_ld + k.
+ *  ncand <= 2048. */
+PBSA_API pbsa_status pbsa_score_select(const pbsa_geom* g, const float* q_reps, int nq,
+                              const float* k_reps, int pool_slots,
+                              const int* cand_slot, const int* cand_gid, int ncand, int k,
+                              const int* prefix_slot, const int* prefix_cnt, int prefix_ld,
+                              int* out_slot, int* out_cnt, int out_ld, float* out_score,
+                              void* ws, void* stream);
+
+/* a3 -- fine attention over the selected blocks (the hybrid mask of the Chinese
+ * explainer 2.2 "掩码机制"; English 2.C "Global Access" + "Local Sparsity"):
+ * for every token i of query block r of head h,
+ *   o_i = sum_{j in A} softmax_j(scale * q_i . k_j) v_j,  lse_i = ln sum_{j in A} exp(scale * q_i . k_j)
+ * where A = the 64 tokens of each pool slot kv_slot[h][r][0..kv_cnt[h][r]) -- one joint
+ * softmax over the union.  Slots of one row must be distinct.  An empty row gives o = 0
+ * and lse = -inf.
+ *  q     [q_frames*frame_h*frame_w][H][d] raster; nq = q_frames*bpf query blocks.
+ *  k_pool, v_pool [H][pool_slots][64][d];  kv_slot [H][nq][kv_ld];  kv_cnt [H][nq].
+ *  o     out, same layout and dtype as q;  lse  nullable out [H][T_q] fp32 (raster t).
+ * bf16: tcgen05 tensor cores, fp32 accumulation, d = 128, kv_ld <= 512.
+ * fp32: exact fp32 SIMT path (d <= 128), kv_ld <= 4096. */
+PBSA_API pbsa_status pbsa_attend(const pbsa_geom* g, const void* q, int q_frames,
+                        const void* k_pool, const void* v_pool, int pool_slots,
+                        const int* kv_slot, const int* kv_cnt, int kv_ld,
+                        void* o, float* lse, void* ws, void* stream);
+
+/* a4 -- persistent-memory update ("Top-C retention"; English 2.C "Dynamic Update",
+ * Chinese 2.2 "粗粒度评分与更新"), per head h:
+ *   pool    = valid persistent slots (slot_gid[h][j] >= 0, j < C) + the candidates
+ *             (cand_slot/cand_gid [H][ncand]; e.g. the blocks leaving the local window)
+ *   p_r     = softmax over the pool of scale * <q_reps[h][r], k_reps[h][slot]>
+ *   a_b     = mean over the nq query blocks of p_{r,b}
+ *   ema_b   = a_b for a candidate, gamma*slot_ema + (1-gamma)*a_b for a persistent block
+ *   keep    = every sink (gid < n_sink_gid) + the top-(C - #sinks) others by ema_b
+ *             (ties to the lower gid)
+ * Kept persistent blocks stay in their slots; each kept candidate is copied (K, V blocks
+ * and k_reps row) from its cand_slot into a freed persistent slot (ascending slot order,
+ * candidates in rank order); slot_gid / slot_ema are rewritten (-1 / 0 for empty slots).
+ * p_list (nullable out [H][C]) receives the valid persistent slots ascending and p_cnt
+ * (nullable out [H]) their count -- the prefix for pbsa_score_select.
+ *  Requires C + ncand <= 4096; cand slots must be >= C (outside the persistent region).
+ *  Workspace: pbsa_workspace_bytes(g, nq, C + ncand). */
+PBSA_API pbsa_status pbsa_memory_update(const pbsa_geom* g, const float* q_reps, int nq,
+                               float* k_reps, void* k_pool, void* v_pool, int pool_slots,
+                               int* slot_gid, float* slot_ema, int capacity, int n_sink_gid,
+                               const int* cand_slot, const int* cand_gid, int ncand,
+                               float gamma, int* p_list, int* p_cnt, void* ws, void* stream);
+
+/* Synchronises `stream`, reads and clears the workspace's device error word, and returns
+ * it (PBSA_OK when clean). */
+PBSA_API pbsa_status pbsa_get_device_error(void* ws, void* stream);
+
+/* Static description of a status code. */
+PBSA_API const char* pbsa_status_string(pbsa_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PBSA_H */

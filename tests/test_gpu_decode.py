@@ -1,0 +1,170 @@
+"""End-to-end GPU parity of a chunk decode and of rollouts (through PBSALayerCache and the
+C-ABI) against the oracle's own plan computed from the same raw Q/K/V."""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_attention_pbsa_b200 as P
+from block_sparse_attention_pbsa_b200 import inputs as I
+from oracle import pbsa_oracle as O
+from tests._util import (EMA_NEAR_TIE_REL, F32_MAX_ABS, NEAR_TIE, assert_bf16_close, block_rows, f64,
+                         geom_dict)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def layer_cfg(w, staging=0):
+    return P.LayerConfig(w.heads, w.head_dim, w.frame_h, w.frame_w, w.tile_h, w.tile_w, w.capacity,
+                         w.window_frames, w.chunk_frames, w.topk, w.gamma, w.dtype, staging)
+
+
+def _decode_single_step(w, sample_units=None):
+    q, k, v = I.single_step(w)
+    kc = I.tokens(w, w.chunk_frames, I.stream_seed(w.seed, 4))
+    vc = I.tokens(w, w.chunk_frames, I.stream_seed(w.seed, 5))
+    bpf = w.blocks_per_frame
+    cache = P.PBSALayerCache(layer_cfg(w, (w.hist_frames - w.window_frames) * bpf))
+    qd = q.to(DEV)
+    q_reps = cache.query_reps(qd)
+    cache.prefill(k.to(DEV), v.to(DEV), w.hist_frames, q_reps)
+    P_gpu = cache.persistent_gids()
+    kv_slot, kv_cnt, ld = cache.select(q_reps)
+    lse = torch.zeros((w.heads, qd.shape[0]), device=DEV)
+    o = cache.attend(qd, kv_slot, kv_cnt, ld, lse=lse)
+    s2g = cache.slot_to_gid()
+    slot_gid = cache.slot_gid.cpu()
+    kv_slot, kv_cnt, o, lse = kv_slot.cpu(), kv_cnt.cpu(), o.cpu(), lse.cpu()
+    assert P.pbsa_get_device_error(cache.ws) == 0
+    cache.commit(kc.to(DEV), vc.to(DEV))
+    P2_gpu = cache.persistent_gids()
+    assert P.pbsa_get_device_error(cache.ws) == 0
+
+    q64, k64, v64 = f64(q), f64(k), f64(v)
+    gd = geom_dict(w)
+    plan = O.single_step_plan(q64, k64, gd, w.hist_frames, w.chunk_frames, w.capacity,
+                              w.window_frames, w.topk, w.gamma, k_chunk=f64(kc))
+    nq = w.chunk_frames * bpf
+    units = [(h, r) for h in range(w.heads) for r in range(nq)]
+    if sample_units is not None:
+        units = [units[i] for i in np.random.default_rng(0).choice(len(units), sample_units, replace=False)]
+    compared = 0
+    for h in range(w.heads):
+        boot_exact = plan["boot_gap"][h] > EMA_NEAR_TIE_REL
+        if boot_exact:
+            assert P_gpu[h] == set(plan["P"][h])
+        assert len(P_gpu[h]) == w.capacity and set(range(bpf)) <= P_gpu[h]
+        pers_slot_gid = {s: int(slot_gid[h, s]) for s in range(w.capacity) if slot_gid[h, s] >= 0}
+        for r in range(nq):
+            n = int(kv_cnt[h, r])
+            slots = kv_slot[h, r, :n].tolist()
+            gids = [pers_slot_gid[s] if s < w.capacity else s2g[s] for s in slots]
+            sel = set(gids[len(pers_slot_gid):])
+            if plan["sel_gap"][h][r] > NEAR_TIE:
+                assert sel == set(plan["sel"][h][r]), (h, r)
+            if (h, r) in units and boot_exact and plan["sel_gap"][h][r] > NEAR_TIE:
+                want, wlse = O.attend_gids(q64, k64, v64, gd, h, r, plan["P"][h] + plan["sel"][h][r],
+                                           q_first_frame=w.hist_frames)
+                rows = block_rows(w, r)
+                if w.dtype == "f32":
+                    np.testing.assert_allclose(f64(o[rows, h]), want, rtol=0, atol=F32_MAX_ABS)
+                else:
+                    assert_bf16_close(f64(o[rows, h]), want, f"h{h} r{r}")
+                np.testing.assert_allclose(f64(lse[h, rows]), wlse, rtol=0, atol=2e-3)
+                compared += 1
+        if plan["P2_gap"][h] > EMA_NEAR_TIE_REL and boot_exact:
+            assert P2_gpu[h] == set(plan["P2"][h])
+    assert compared >= len(units) // 2
+
+
+def test_decode_tiny_f32():
+    _decode_single_step(I.TINY)
+
+
+def test_decode_5s_last_chunk_bf16():
+    _decode_single_step(I.DECODE_5S, sample_units=24)
+
+
+def _rollout(w, n_chunks, sample_every=3):
+    """Layer-0 rollout: GPU cache vs the oracle state machine, chunk by chunk.  A head whose
+    memory-update boundary was a near tie is compared no further (both outcomes are valid)."""
+    bpf = w.blocks_per_frame
+    cache = P.PBSALayerCache(layer_cfg(w))
+    ro = O.RolloutOracle(geom_dict(w), w.heads, w.capacity, w.window_frames, w.topk, w.gamma)
+    gd = geom_dict(w)
+    alive = [True] * w.heads
+    offsets = ([I.ar1_offsets(w, w.total_frames, I.stream_seed(w.seed, 99, t)) for t in range(3)]
+               if w.ar_rho > 0 else None)
+    kv_hist = {"k": [], "v": []}
+    kv_bytes0 = cache.kv_bytes
+    chunks = I.rollout_chunks(w)[:n_chunks]
+    for c, (f0, nf) in enumerate(chunks):
+        assert nf == w.chunk_frames or c == 0
+        wc = dataclasses.replace(w, chunk_frames=nf)
+        for s in range(w.steps):
+            seeds = [I.stream_seed(w.seed, c, s, t) for t in range(3)]
+            if offsets is not None:
+                q, k, v = (I.tokens_with_offsets(w, off[f0:f0 + nf], sd) for off, sd in zip(offsets, seeds))
+            else:
+                q, k, v = (I.tokens(wc, nf, sd) for sd in seeds)
+            o = cache.decode_step(q.to(DEV), k.to(DEV), v.to(DEV))
+            q64 = f64(q)
+            q_reps = O.block_reps(q64, gd, nf)
+            sel = ro.select(q_reps)
+            if sel is None and s == w.steps - 1:
+                # empty history: the chunk attends its own blocks (this step's K, V)
+                own = list(range(f0 * bpf, (f0 + nf) * bpf))
+                r = c % q_reps.shape[1]
+                for h in range(w.heads):
+                    want, _ = O.attend_gids(q64, f64(k), f64(v), gd, h, r, own, q_first_frame=f0)
+                    assert_bf16_close(f64(o.cpu()[block_rows(wc, r), h]), want, f"own c{c} h{h}")
+            if sel is not None:
+                kv_slot, kv_cnt = cache.kv_slot.cpu(), cache.kv_cnt.cpu()
+                s2g = cache.slot_to_gid()
+                sg = cache.slot_gid.cpu()
+                for h in range(w.heads):
+                    if not alive[h]:
+                        continue
+                    pers = {int(x) for x in sg[h] if x >= 0}
+                    for r in range(q_reps.shape[1]):
+                        gids_want, gap = sel[h][r]
+                        n = int(kv_cnt[h, r])
+                        slots = kv_slot[h, r, :n].tolist()
+                        got = {int(sg[h, x]) if x < w.capacity else s2g[x] for x in slots}
+                        if gap > NEAR_TIE:
+                            assert got == set(gids_want), (c, s, h, r)
+                            if c % sample_every == 0 and r == (c * 7 + s) % q_reps.shape[1]:
+                                hist_k = np.concatenate(kv_hist["k"])
+                                hist_v = np.concatenate(kv_hist["v"])
+                                want, _ = O.attend_gids(q64, hist_k, hist_v, gd, h, r, sorted(got), q_first_frame=f0)
+                                assert_bf16_close(f64(o.cpu()[block_rows(wc, r), h]), want, f"c{c} h{h} r{r}")
+                        assert pers <= got
+        cache.commit(k.to(DEV), v.to(DEV))
+        assert P.pbsa_get_device_error(cache.ws) == 0
+        kv_hist["k"].append(f64(k))
+        kv_hist["v"].append(f64(v))
+        ro.commit(f0, nf, O.block_reps(f64(k), gd, nf), q_reps)
+        got_P = cache.persistent_gids()
+        for h in range(w.heads):
+            assert len(got_P[h]) <= w.capacity and set(range(bpf)) <= got_P[h]
+            if alive[h]:
+                if ro.last_gap[h] > EMA_NEAR_TIE_REL:
+                    assert got_P[h] == set(ro.P[h]), (c, h)
+                else:
+                    alive[h] = False
+        assert cache.kv_bytes == kv_bytes0   # KV memory stays flat
+    return alive
+
+
+def test_rollout_5s_layer0():
+    w = I.ROLLOUT_5S
+    alive = _rollout(w, n_chunks=7)
+    assert sum(alive) >= w.heads // 2
+
+
+@pytest.mark.slow
+def test_rollout_1min_layer0_first_chunks():
+    w = dataclasses.replace(I.ROLLOUT_1MIN, total_frames=1 + 3 * 12)
+    _rollout(w, n_chunks=13, sample_every=4)

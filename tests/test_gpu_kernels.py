@@ -1,0 +1,293 @@
+"""GPU parity of each C-ABI entry point against the CPU oracle, on seeded inputs.
+
+Inputs are synthetic tensors built on the host (never outputs of the CUDA path); both
+sides consume the same values (bf16 inputs are rounded once and up-converted for the
+oracle).
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_attention_pbsa_b200 as P
+from block_sparse_attention_pbsa_b200 import inputs as I
+from oracle import pbsa_oracle as O
+from tests._util import (F32_MAX_ABS, NEAR_TIE, EMA_NEAR_TIE_REL, assert_bf16_close, block_rows,
+                         f64, geom_dict)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def geom_for(w):
+    return P.make_geom(w.heads, w.head_dim, w.frame_h, w.frame_w, w.tile_h, w.tile_w, w.scale, w.dtype)
+
+
+def ws_for(g, nq=64, pool=64):
+    return torch.zeros(P.pbsa_workspace_bytes(g, nq, pool), dtype=torch.uint8, device=DEV)
+
+
+def check_no_device_error(ws):
+    assert P.pbsa_get_device_error(ws) == 0
+
+
+# ----------------------------------------------------------------------------- blockify
+@pytest.mark.parametrize("w", [I.TINY, I.DECODE_5S, dataclasses.replace(I.DECODE_5S, tile_h=4, tile_w=16)])
+def test_blockify_reps_and_pool(w):
+    g = geom_for(w)
+    n_frames = 2
+    x = I.tokens(w, n_frames, 11)
+    nb = n_frames * w.blocks_per_frame
+    slots = nb + 5
+    dst = torch.randperm(slots, generator=torch.Generator().manual_seed(3))[:nb].to(torch.int32)
+    reps = torch.zeros((w.heads, slots, w.head_dim), device=DEV)
+    pool = torch.zeros((w.heads, slots, 64, w.head_dim), dtype=x.dtype, device=DEV)
+    ws = ws_for(g)
+    P.pbsa_blockify(g, x.to(DEV), n_frames, reps, slots, dst.to(DEV), pool, slots, ws)
+    check_no_device_error(ws)
+    want = O.block_reps(f64(x), geom_dict(w), n_frames)
+    got = f64(reps)
+    for b in range(nb):
+        s = int(dst[b])
+        np.testing.assert_allclose(got[:, s], want[:, b], rtol=0, atol=2e-6)
+        rows = O.block_token_rows(w.frame_h, w.frame_w, w.tile_h, w.tile_w, b)
+        assert torch.equal(pool[:, s].cpu(), x[rows].permute(1, 0, 2))
+
+
+# ----------------------------------------------------------------------------- score + select
+def _selection_case(seed, H=3, nq=9, pool=200, ncand=144, d=128, k=32, prefix=20, dup=False):
+    gen = torch.Generator().manual_seed(seed)
+    q = torch.randn((H, nq, d), generator=gen) * 0.3 + torch.randn((H, 1, d), generator=gen) * 0.2
+    kr = torch.randn((H, pool, d), generator=gen) * 0.3
+    if dup:
+        kr[:] = kr[:, :1]
+    cs = torch.stack([torch.randperm(pool, generator=gen)[:ncand] for _ in range(H)]).to(torch.int32)
+    cg = torch.stack([torch.randperm(5000, generator=gen)[:ncand] for _ in range(H)]).to(torch.int32)
+    ps = torch.randint(0, pool, (H, prefix), generator=gen, dtype=torch.int32)
+    pc = torch.tensor([prefix - h for h in range(H)], dtype=torch.int32)
+    return q, kr, cs, cg, ps, pc
+
+
+@pytest.mark.parametrize("dup", [False, True])
+@pytest.mark.parametrize("ncand,k", [(144, 32), (48, 32), (20, 32), (300, 16), (0, 8)])
+def test_score_select(ncand, k, dup):
+    H, nq, d, pool, prefix = 3, 9, 128, 400, 20
+    w = dataclasses.replace(I.DECODE_5S, heads=H)
+    g = geom_for(w)
+    q, kr, cs, cg, ps, pc = _selection_case(7 + ncand, H, nq, pool, ncand, d, k, prefix, dup)
+    out_ld = prefix + k + 3
+    out = torch.full((H, nq, out_ld), -7, dtype=torch.int32, device=DEV)
+    cnt = torch.zeros((H, nq), dtype=torch.int32, device=DEV)
+    sc = torch.zeros((H, nq, max(k, 1)), device=DEV)
+    ws = ws_for(g)
+    P.pbsa_score_select(g, q.to(DEV), nq, kr.to(DEV), pool, cs.to(DEV) if ncand else None,
+                        cg.to(DEV) if ncand else None, ncand, k, ps.to(DEV), pc.to(DEV), prefix, out,
+                        cnt, out_ld, sc, ws)
+    check_no_device_error(ws)
+    out, cnt, sc = out.cpu(), cnt.cpu(), sc.cpu()
+    kk = min(k, ncand)
+    checked = 0
+    for h in range(H):
+        for r in range(nq):
+            p = int(pc[h])
+            assert int(cnt[h, r]) == p + kk
+            assert out[h, r, :p].tolist() == ps[h, :p].tolist()
+            if ncand == 0:
+                continue
+            s64 = O.coarse_scores(f64(q[h, r:r + 1]), f64(kr[h][cs[h].long()]), w.scale)[0]
+            s32 = s64.astype(np.float32)
+            want_pos = O.topk_select(s32, cg[h].tolist(), k)
+            got_slots = out[h, r, p:p + kk].tolist()
+            np.testing.assert_allclose(sc[h, r, :kk].numpy(), s32[want_pos], rtol=0, atol=1e-5)
+            if dup or O.kth_gap(s32, cg[h].tolist(), k) > NEAR_TIE:
+                assert set(got_slots) == {int(cs[h, i]) for i in want_pos}
+                checked += 1
+            else:
+                assert len(set(got_slots)) == kk and set(got_slots) <= set(cs[h].tolist())
+    assert ncand == 0 or checked >= H * nq // 2
+
+
+# ----------------------------------------------------------------------------- attend
+def _attend_case(w, q_frames, slots, lists, seed):
+    gen = torch.Generator().manual_seed(seed)
+    dt = w.torch_dtype
+    q = (torch.randn((q_frames * w.tokens_per_frame, w.heads, w.head_dim), generator=gen)).to(dt)
+    kp = torch.randn((w.heads, slots, 64, w.head_dim), generator=gen)
+    kp = (kp + torch.randn((w.heads, slots, 1, w.head_dim), generator=gen) * 0.5).to(dt)
+    vp = torch.randn((w.heads, slots, 64, w.head_dim), generator=gen).to(dt)
+    nq = q_frames * w.blocks_per_frame
+    ld = max(1, max(len(l) for row in lists for l in row))
+    kv = torch.zeros((w.heads, nq, ld), dtype=torch.int32)
+    cnt = torch.zeros((w.heads, nq), dtype=torch.int32)
+    for h in range(w.heads):
+        for r in range(nq):
+            kv[h, r, :len(lists[h][r])] = torch.tensor(lists[h][r], dtype=torch.int32)
+            cnt[h, r] = len(lists[h][r])
+    return q, kp, vp, kv, cnt, ld
+
+
+def _run_attend(w, q, q_frames, kp, vp, kv, cnt, ld):
+    g = geom_for(w)
+    o = torch.full(q.shape, float("nan"), dtype=q.dtype, device=DEV)
+    lse = torch.zeros((w.heads, q.shape[0]), device=DEV)
+    ws = ws_for(g)
+    P.pbsa_attend(g, q.to(DEV), q_frames, kp.to(DEV), vp.to(DEV), kp.shape[1], kv.to(DEV), cnt.to(DEV),
+                  ld, o, lse, ws)
+    check_no_device_error(ws)
+    return o.cpu(), lse.cpu()
+
+
+def _oracle_unit(w, q, kp, vp, h, r, slots):
+    rows = block_rows(w, r)
+    kk = f64(kp[h][list(slots)].reshape(-1, w.head_dim)) if slots else np.zeros((0, w.head_dim))
+    vv = f64(vp[h][list(slots)].reshape(-1, w.head_dim)) if slots else np.zeros((0, w.head_dim))
+    return rows, O.attention(f64(q[rows, h]), kk, vv, w.scale)
+
+
+def _lists(rng, H, nq, slots, shared, local, empty_every=0):
+    out = []
+    for h in range(H):
+        pers = rng.choice(slots, size=shared, replace=False).tolist()
+        rest = [s for s in range(slots) if s not in pers]
+        rows = []
+        for r in range(nq):
+            if empty_every and r % empty_every == empty_every - 1:
+                rows.append([])
+                continue
+            nl = int(rng.integers(0, local + 1))
+            rows.append(pers + rng.choice(rest, size=nl, replace=False).tolist())
+        out.append(rows)
+    return out
+
+
+def test_attend_f32_tiny():
+    w = I.TINY
+    rng = np.random.default_rng(0)
+    slots = 24
+    lists = _lists(rng, w.heads, 4, slots, 8, 4, empty_every=4)
+    lists[0][0] = list(range(24))
+    q, kp, vp, kv, cnt, ld = _attend_case(w, 1, slots, lists, 5)
+    o, lse = _run_attend(w, q, 1, kp, vp, kv, cnt, ld)
+    for r in range(4):
+        rows, (want, wlse) = _oracle_unit(w, q, kp, vp, 0, r, lists[0][r])
+        np.testing.assert_allclose(f64(o[rows, 0]), want, rtol=0, atol=F32_MAX_ABS)
+        if lists[0][r]:
+            np.testing.assert_allclose(f64(lse[0, rows]), wlse, rtol=0, atol=F32_MAX_ABS)
+        else:
+            assert np.isneginf(f64(lse[0, rows])).all()
+
+
+@pytest.mark.parametrize("fh,fw,q_frames,shared,local,empty", [
+    (8, 24, 1, 10, 6, 0),      # 3 query blocks: odd count, last CTA has one half
+    (16, 16, 2, 20, 9, 5),     # empty lists and ragged counts
+    (32, 48, 1, 96, 32, 0),    # the decode shape: 96 shared + 32 local
+    (8, 8, 1, 1, 0, 0),        # a single block
+])
+def test_attend_bf16(fh, fw, q_frames, shared, local, empty):
+    w = dataclasses.replace(I.DECODE_5S, heads=2, frame_h=fh, frame_w=fw)
+    nq = q_frames * w.blocks_per_frame
+    slots = max(shared + local + 7, 40)
+    rng = np.random.default_rng(fh * 100 + fw)
+    lists = _lists(rng, w.heads, nq, slots, shared, local, empty)
+    q, kp, vp, kv, cnt, ld = _attend_case(w, q_frames, slots, lists, fh + fw)
+    o, lse = _run_attend(w, q, q_frames, kp, vp, kv, cnt, ld)
+    for h in range(w.heads):
+        for r in range(nq):
+            rows, (want, wlse) = _oracle_unit(w, q, kp, vp, h, r, lists[h][r])
+            assert_bf16_close(f64(o[rows, h]), want, f"h{h} r{r}")
+            if lists[h][r]:
+                np.testing.assert_allclose(f64(lse[h, rows]), wlse, rtol=0, atol=2e-3)
+            else:
+                assert np.isneginf(f64(lse[h, rows])).all()
+
+
+def test_attend_bf16_bad_slot_is_reported():
+    w = dataclasses.replace(I.DECODE_5S, heads=1, frame_h=8, frame_w=16)
+    lists = [[[0, 1, 999], [2, 3]]]
+    q, kp, vp, kv, cnt, ld = _attend_case(w, 1, 8, lists, 1)
+    g = geom_for(w)
+    ws = ws_for(g)
+    o = torch.zeros(q.shape, dtype=q.dtype, device=DEV)
+    P.pbsa_attend(g, q.to(DEV), 1, kp.to(DEV), vp.to(DEV), 8, kv.to(DEV), cnt.to(DEV), ld, o, None, ws)
+    assert P.pbsa_get_device_error(ws) == 5
+    assert P.pbsa_get_device_error(ws) == 0   # cleared by the read
+    # the bad entry is skipped: the row equals attention over the two valid blocks
+    rows, (want, _) = _oracle_unit(w, q, kp, vp, 0, 0, [0, 1])
+    assert_bf16_close(f64(o.cpu()[rows, 0]), want)
+
+
+def test_invalid_arguments_are_rejected_on_host():
+    w = I.DECODE_5S
+    g = geom_for(w)
+    x = torch.zeros((w.tokens_per_frame, w.heads, w.head_dim), dtype=torch.bfloat16, device=DEV)
+    reps = torch.zeros((w.heads, 24, w.head_dim), device=DEV)
+    with pytest.raises(P.PBSAError) as e:
+        P.pbsa_blockify(g, x, 0, reps, 24)
+    assert e.value.code == 1
+    bad = P.make_geom(12, 128, 32, 48, 8, 7, w.scale, "bf16")
+    with pytest.raises(P.PBSAError):
+        P.pbsa_blockify(bad, x, 1, reps, 24)
+
+
+# ----------------------------------------------------------------------------- memory update
+@pytest.mark.parametrize("n_pers,ncand,C", [(70, 72, 96), (24, 48, 96), (96, 72, 96), (0, 264, 96), (3, 5, 8)])
+def test_memory_update(n_pers, ncand, C):
+    H, d, nq, S = 3, 128, 72, min(24, C // 2)
+    w = dataclasses.replace(I.DECODE_5S, heads=H)
+    g = geom_for(w)
+    gen = torch.Generator().manual_seed(n_pers * 1000 + ncand)
+    pool = C + ncand + 10
+    qr = torch.randn((H, nq, d), generator=gen) * 0.3 + torch.randn((H, 1, d), generator=gen) * 0.3
+    kr = torch.randn((H, pool, d), generator=gen) * 0.35
+    kp = torch.randn((H, pool, 64, d), generator=gen).to(torch.bfloat16)
+    vp = torch.randn((H, pool, 64, d), generator=gen).to(torch.bfloat16)
+    sgid = torch.full((H, C), -1, dtype=torch.int32)
+    sema = torch.zeros((H, C))
+    cs = torch.zeros((H, ncand), dtype=torch.int32)
+    cg = torch.zeros((H, ncand), dtype=torch.int32)
+    for h in range(H):
+        pslots = torch.randperm(C, generator=gen)[:n_pers]
+        gids = torch.randperm(4000, generator=gen)[:n_pers + ncand] + S
+        ns = min(S, n_pers) if n_pers else 0
+        for i, s in enumerate(pslots.tolist()):
+            sgid[h, s] = i if i < ns else int(gids[i])        # the first ns are sinks (gid < S)
+            sema[h, s] = float(torch.rand((), generator=gen)) * 0.02
+        cs[h] = torch.randperm(pool - C, generator=gen)[:ncand].to(torch.int32) + C
+        cg[h] = gids[n_pers:n_pers + ncand].to(torch.int32)
+        if n_pers == 0 and ncand >= S:
+            cg[h, :S] = torch.arange(S, dtype=torch.int32)   # sinks arriving as candidates
+    kr_d, kp_d, vp_d = kr.to(DEV), kp.to(DEV), vp.to(DEV)
+    sgid_d, sema_d = sgid.to(DEV), sema.to(DEV)
+    plist = torch.full((H, C), -5, dtype=torch.int32, device=DEV)
+    pcnt = torch.zeros((H,), dtype=torch.int32, device=DEV)
+    ws = torch.zeros(P.pbsa_workspace_bytes(g, nq, C + ncand), dtype=torch.uint8, device=DEV)
+    P.pbsa_memory_update(g, qr.to(DEV), nq, kr_d, kp_d, vp_d, pool, sgid_d, sema_d, C, S, cs.to(DEV),
+                         cg.to(DEV), ncand, 0.9, plist, pcnt, ws)
+    check_no_device_error(ws)
+    new_gid, new_ema = sgid_d.cpu(), sema_d.cpu()
+    for h in range(H):
+        ent = [(s, int(sgid[h, s]), float(sema[h, s])) for s in range(C) if sgid[h, s] >= 0]
+        ent += [(int(cs[h, i]), int(cg[h, i]), np.nan) for i in range(ncand)]
+        slots_, gids_, prev = zip(*ent)
+        sink = [gg < S for gg in gids_]
+        ema, keep, a = O.memory_update(f64(qr[h]), f64(kr[h][list(slots_)]), gids_, prev, sink, w.scale, 0.9, C)
+        want = {gg for gg, kp_ in zip(gids_, keep) if kp_}
+        got = {int(x) for x in new_gid[h] if x >= 0}
+        assert len(got) <= C and {gg for gg in gids_ if gg < S} <= got
+        if O.ema_boundary_gap(ema, gids_, sink, C) > EMA_NEAR_TIE_REL:
+            assert got == want
+        ema_of = dict(zip(gids_, ema))
+        src_of = dict(zip(gids_, slots_))
+        for s in range(C):
+            gg = int(new_gid[h, s])
+            if gg < 0:
+                continue
+            np.testing.assert_allclose(float(new_ema[h, s]), ema_of[gg], rtol=2e-5, atol=1e-9)
+            src = src_of[gg]
+            if src != s:   # promoted: K, V, k_reps copied into slot s
+                assert src >= C
+                assert torch.equal(kp_d[h, s].cpu(), kp[h, src]) and torch.equal(vp_d[h, s].cpu(), vp[h, src])
+                assert torch.equal(kr_d[h, s].cpu(), kr[h, src])
+        valid = [s for s in range(C) if new_gid[h, s] >= 0]
+        assert int(pcnt[h]) == len(valid) and plist[h, :len(valid)].cpu().tolist() == valid
