@@ -1,0 +1,340 @@
+#!/usr/bin/env python
+"""PBSA chunk-decode benchmark on B200.
+
+One step = one chunk decode of one attention layer on the 5 s-video last-chunk workload
+(12 heads, d=128, 32x48-token frames in 64-token blocks, 3-frame chunk = 72 query blocks,
+18 history frames, C=96 persistent blocks, 6-frame window, top-32 local blocks), i.e.
+every row of the hot path: blockify(Q) -> coarse score + top-k -> block-sparse attention
+(tcgen05) -> commit of the chunk's K/V (blockify into the ring) -> persistent-memory
+update.  Inputs are resident in HBM before timing; L2 is flushed between timed steps;
+each step is timed with CUDA events on its stream.  The state the step mutates is
+restored (outside the timed region) so every step does identical work.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl pbsa|reference]
+
+N > 1 (torchrun, one rank per GPU): every rank decodes its own independent layer (weak
+scaling, no collective on the data path); the step time is the max over ranks.
+``--impl reference`` times the CPU oracle on the host cores on a bounded sample of the
+same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+METRIC = "PBSA ms/chunk-decode and selected-block TFLOP/s (% of B200 bf16 peak), 1 GPU"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16": p["bf16_tflops"], "bf16_sustained": p["bf16_tflops_sustained"],
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index, self.rows, self.proc = index, [], None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            threading.Thread(target=self._read, daemon=True).start()
+        except OSError:
+            self.proc = None
+        time.sleep(0.25)
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append([x.strip() for x in line.split(",")])
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            self.proc.wait(timeout=5)
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in self.rows:
+            try:
+                sm.append(float(r[0]))
+                mx = float(r[1])
+                for n, v in zip(names, r[4:8]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+            except (ValueError, IndexError):
+                continue
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def workload_config(w):
+    return {"workload": w.name, "heads": w.heads, "head_dim": w.head_dim,
+            "frame_tokens": f"{w.frame_h}x{w.frame_w}", "block": f"1 frame x {w.tile_h}x{w.tile_w}",
+            "chunk_frames": w.chunk_frames, "query_blocks": w.chunk_frames * w.blocks_per_frame,
+            "hist_frames": w.hist_frames, "capacity": w.capacity, "window_frames": w.window_frames,
+            "topk": w.topk, "kv_blocks_per_query_block": w.capacity + w.topk,
+            "l2": "flushed (256 MiB write) before every timed step"}
+
+
+# ----------------------------------------------------------------------------- CPU oracle arm
+def oracle_sample(w, q, k, v, units: int, seed: int = 0):
+    """Time the oracle on a bounded sample of one chunk decode; returns (seconds extrapolated
+    to the full step, description, threads)."""
+    from oracle import pbsa_oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:  # pragma: no cover - informational only
+        threads = 1
+    gd = {"frame_h": w.frame_h, "frame_w": w.frame_w, "tile_h": w.tile_h, "tile_w": w.tile_w, "scale": w.scale}
+    q64, k64, v64 = (t.double().numpy() for t in (q, k, v))
+    t0 = time.perf_counter()
+    plan = O.single_step_plan(q64, k64, gd, w.hist_frames, w.chunk_frames, w.capacity, w.window_frames,
+                              w.topk, w.gamma)
+    t_plan = time.perf_counter() - t0
+    nq = w.chunk_frames * w.blocks_per_frame
+    rng = np.random.default_rng(seed)
+    pick = rng.choice(w.heads * nq, size=units, replace=False)
+    t0 = time.perf_counter()
+    for u in pick:
+        h, r = divmod(int(u), nq)
+        O.attend_gids(q64, k64, v64, gd, h, r, plan["P"][h] + plan["sel"][h][r], q_first_frame=w.hist_frames)
+    t_att = (time.perf_counter() - t0) / units
+    full = t_plan + t_att * w.heads * nq
+    desc = (f"oracle selection/update plan for all {w.heads} heads (timed whole, {t_plan:.2f}s) + "
+            f"fine attention of {units} of {w.heads * nq} (head, query block) units, extrapolated")
+    return full, desc, threads
+
+
+def run_reference(args, w, rank, world):
+    if rank != 0:
+        return
+    from block_sparse_attention_pbsa_b200 import inputs as I
+    q, k, v = I.single_step(w)
+    flops = 4.0 * 64 * 64 * w.head_dim * w.heads * w.chunk_frames * w.blocks_per_frame * (w.capacity + w.topk)
+    units = 24
+    for _ in range(args.warmup):
+        oracle_sample(w, q, k, v, 4)
+    times = []
+    desc, threads = "", 1
+    for s in range(args.steps):
+        t, desc, threads = oracle_sample(w, q, k, v, units, seed=s)
+        times.append(t)
+    t = statistics.mean(times)
+    value = flops / t / 1e12
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": workload_config(w),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- PBSA arm
+def algorithmic_bytes(w, ncopy: int):
+    """Bytes each kernel group must move at minimum (per step)."""
+    H, d, bpf = w.heads, w.head_dim, w.blocks_per_frame
+    nq = w.chunk_frames * bpf
+    tok = nq * 64 * H * d * 2                      # one chunk's raster tensor, bf16
+    reps_q = H * nq * d * 4
+    nwin = w.window_frames * bpf
+    return {
+        "blockify_q": tok + reps_q,
+        "score_select": reps_q + H * nwin * d * 4 + H * nq * (w.capacity + w.topk) * 4 + H * w.capacity * 4,
+        "commit_blockify_kv": 2 * (tok + tok) + 2 * reps_q,
+        # scores/softmax: q reps + pool reps + p matrix (write, read); copies: K+V+reps per promotion
+        "memory_update": reps_q + H * (w.capacity + w.chunk_frames * bpf) * d * 4
+        + 2 * H * nq * (w.capacity + w.chunk_frames * bpf) * 4 + ncopy * 2 * (2 * 64 * d * 2 + d * 4),
+    }
+
+
+def _check_device(P, ws, when: str):
+    """Raise with the workspace's device error word (code, info, kernel id) if one is set."""
+    torch.cuda.synchronize()
+    word = ws[:16].view(torch.int32).tolist()
+    if P.pbsa_get_device_error(ws) != 0:
+        raise RuntimeError(f"device error {when}: code={word[0]} info={word[1]} kernel={word[2]}")
+
+
+def run_pbsa(args, w, rank, world, local_rank):
+    import block_sparse_attention_pbsa_b200 as P
+    from block_sparse_attention_pbsa_b200 import inputs as I
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    wr = w if rank == 0 else __import__("dataclasses").replace(w, seed=w.seed + 1000 * rank)
+    q, k, v = I.single_step(wr)
+    kc = I.tokens(wr, wr.chunk_frames, I.stream_seed(wr.seed, 4))
+    vc = I.tokens(wr, wr.chunk_frames, I.stream_seed(wr.seed, 5))
+    bpf = w.blocks_per_frame
+    cfg = P.LayerConfig(w.heads, w.head_dim, w.frame_h, w.frame_w, w.tile_h, w.tile_w, w.capacity,
+                        w.window_frames, w.chunk_frames, w.topk, w.gamma, w.dtype,
+                        (w.hist_frames - w.window_frames) * bpf)
+    cache = P.PBSALayerCache(cfg, dev)
+    qd, kcd, vcd = q.to(dev), kc.to(dev), vc.to(dev)
+    cache.prefill(k.to(dev), v.to(dev), w.hist_frames, cache.query_reps(qd))
+    step = P.ChunkDecodeStep(cache)
+    o = torch.empty_like(qd)
+    snap = step.snapshot()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    torch.cuda.synchronize(dev)
+
+    def one(marks=None):
+        step.restore(snap)
+        flush.fill_(1)
+        step.run(qd, kcd, vcd, o, stream=stream, marks=marks)
+
+    for _ in range(max(args.warmup, 3)):
+        one()
+    torch.cuda.synchronize(dev)
+    _check_device(P, cache.ws, "during warm-up")
+    flops = step.flops()
+    ncopy_dev = torch.zeros((), dtype=torch.int32)
+
+    marks = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local_rank) as clk:
+        for s in range(args.steps):
+            one(marks[s])
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    groups = ["blockify_q", "score_select", "attend", "commit_blockify_kv", "memory_update"]
+    per = {g: statistics.mean(m[i].elapsed_time(m[i + 1]) for m in marks) for i, g in enumerate(groups)}
+    step_ms = statistics.mean(m[0].elapsed_time(m[5]) for m in marks)
+    step_t = torch.tensor([step_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(step_t, op=torch.distributed.ReduceOp.MAX)
+    step_ms_max = float(step_t.item())
+    # number of block copies the memory update made (for its algorithmic bytes)
+    step.restore(snap)
+    step.run(qd, kcd, vcd, o, stream=stream)
+    torch.cuda.synchronize(dev)
+    ncopy = int((cache.slot_gid != snap[0]).sum().item())
+    _check_device(P, cache.ws, "during the timed steps")
+
+    # ---- end to end through the public API: pinned host inputs -> HBM -> step -> host output
+    qh, kh, vh = (t.pin_memory() for t in (q, kc, vc))
+    oh = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    e2e_ms = []
+    for s in range(max(1, args.steps // 2) + 1):
+        step.restore(snap)
+        flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        qd.copy_(qh, non_blocking=True)
+        kcd.copy_(kh, non_blocking=True)
+        vcd.copy_(vh, non_blocking=True)
+        step.run(qd, kcd, vcd, o, stream=stream)
+        oh.copy_(o, non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        if s > 0:
+            e2e_ms.append(e0.elapsed_time(e1))
+    e2e_t = torch.tensor([statistics.mean(e2e_ms)], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(e2e_t, op=torch.distributed.ReduceOp.MAX)
+
+    if rank != 0:
+        return
+    ab = algorithmic_bytes(w, ncopy)
+    kernels = {g: {"ms": per[g]} for g in groups}
+    for g, b in ab.items():
+        kernels[g].update({"algorithmic_bytes": b, "achieved_gbs": b / (per[g] * 1e-3) / 1e9,
+                           "frac_hbm": b / (per[g] * 1e-3) / 1e9 / peaks["hbm_gbs"]})
+    att_tflops = flops / (per["attend"] * 1e-3) / 1e12
+    kernels["attend"].update({"flops": flops, "achieved_tflops": att_tflops})
+    value = world * flops / (step_ms_max * 1e-3) / 1e12
+    h2d = sum(t.numel() * t.element_size() for t in (q, kc, vc))
+    d2h = o.numel() * o.element_size()
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": step_ms_max, "ms_per_chunk_decode": step_ms_max,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": {**workload_config(w),
+                                        "parallelism": f"{world} independent layer decodes (one per GPU)"},
+        "roofline": {"bound": "tensor", "kernel": "pbsa_attend (attend_tc_kernel)", "achieved": att_tflops,
+                     "peak": peaks["bf16"], "unit": "TFLOP/s", "frac": att_tflops / peaks["bf16"],
+                     "peak_source": f"{peaks['source']} burst bf16 (cuBLAS)",
+                     "frac_of_sustained": att_tflops / peaks["bf16_sustained"], "traffic": None},
+        "step_frac_of_bf16_peak": value / world / peaks["bf16"],
+        "kernels": kernels,
+        "kv_cache_bytes": {"pbsa_per_layer": cache.kv_bytes,
+                           "dense_21_frames_per_layer": 2 * w.heads * 21 * w.tokens_per_frame * w.head_dim * 2},
+        "e2e": {"value": world * flops / (float(e2e_t.item()) * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "ms_per_step": float(e2e_t.item()), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": P.ChunkDecodeStep.LAUNCHES * args.steps,
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        t, desc, threads = oracle_sample(w, q, k, v, units=24)
+        line["cpu_baseline"] = {"value": flops / t / 1e12, "unit": "TFLOP/s", "cores": threads,
+                                "kind": "oracle", "sample": desc, "ms_per_step": t * 1e3}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["pbsa", "reference"], default="pbsa")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    from block_sparse_attention_pbsa_b200 import inputs as I
+    w = I.DECODE_5S
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, w, rank, world)
+        return
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        run_pbsa(args, w, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

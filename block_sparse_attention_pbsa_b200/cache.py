@@ -273,3 +273,87 @@ class PBSALayerCache:
         """Map of ring/stage slots to global block ids for the current window (host bookkeeping)."""
         bpf = self.cfg.bpf
         return {self.ring_slot(f, t): f * bpf + t for f in self.window_frames() for t in range(bpf)}
+
+
+class ChunkDecodeStep:
+    """One chunk decode plus its commit, with every device-side index array prepared up front.
+
+    ``run(q, k, v)`` issues only C-ABI launches on one stream -- blockify(Q), score+top-k,
+    attend, blockify(K), blockify(V) into the chunk's ring positions, memory update (3
+    kernels) -- with no host synchronisation or allocation, so it can be timed per kernel
+    or captured in a CUDA graph.  It does not advance the cache's host bookkeeping: the same
+    step can be replayed on a restored state (see ``snapshot``/``restore``).
+    """
+
+    LAUNCHES = 8   # kernels per run(): 1 + 1 + 1 + 2 + 3
+
+    def __init__(self, cache: PBSALayerCache, q_frames: int | None = None):
+        c = cache.cfg
+        self.cache = cache
+        self.q_frames = q_frames or c.chunk_frames
+        if cache._cand is None:
+            cache._refresh_window()
+        bpf, H = c.bpf, c.heads
+        nq = self.q_frames * bpf
+        self.nq = nq
+        dev = cache.device
+        self.q_reps = torch.zeros((H, nq, c.head_dim), dtype=torch.float32, device=dev)
+        self.kv_slot = torch.zeros((H, nq, cache.kv_ld), dtype=torch.int32, device=dev)
+        self.kv_cnt = torch.zeros((H, nq), dtype=torch.int32, device=dev)
+        first = cache.hist
+        self.dst = cache._frames_dst(first, self.q_frames)
+        old_win = set(cache.window_frames(first))
+        new_win = set(cache.window_frames(first + self.q_frames))
+        entering = {f for f in range(first, first + self.q_frames) if f != 0}
+        evicted = sorted((old_win | entering) - new_win)
+        cand = [(cache.ring_slot(f, t), f * bpf + t) for f in evicted for t in range(bpf)]
+        if first == 0:
+            cand = [(cache.ring_slot(0, t), t) for t in range(bpf)] + cand
+        self.ncand = len(cand)
+        self.cs = cache._ints([[s for s, _ in cand]] * H).view(H, -1) if cand else None
+        self.cg = cache._ints([[g for _, g in cand]] * H).view(H, -1) if cand else None
+        self.vreps = cache._v_reps_sink()
+
+    def flops(self) -> float:
+        """Selected-block attention FLOPs of one run (QK^T and PV, 2 flops per MAC)."""
+        c = self.cache.cfg
+        cnt = int(self.kv_cnt.sum().item())
+        return 4.0 * 64 * 64 * c.head_dim * cnt
+
+    def run(self, q, k, v, o, lse=None, stream=None, marks=None):
+        """``marks``: optional list of torch.cuda.Event recorded after each kernel group
+        (blockify Q, select, attend, commit blockify K+V, memory update)."""
+        ca, c = self.cache, self.cache.cfg
+        g, ws, ps = ca.geom, ca.ws, ca.pool_slots
+        mk = (lambda i: marks[i].record(stream)) if marks is not None else (lambda i: None)
+        mk(0)
+        L.pbsa_blockify(g, q, self.q_frames, self.q_reps, self.nq, ws=ws, stream=stream)
+        mk(1)
+        cs, cg, n = ca._cand
+        L.pbsa_score_select(g, self.q_reps, self.nq, ca.k_reps, ps, cs, cg, n, c.topk if n else 0,
+                            ca.p_list, ca.p_cnt, c.capacity, self.kv_slot, self.kv_cnt, ca.kv_ld,
+                            ws=ws, stream=stream)
+        mk(2)
+        L.pbsa_attend(g, q, self.q_frames, ca.k_pool, ca.v_pool, ps, self.kv_slot, self.kv_cnt, ca.kv_ld,
+                      o, lse, ws=ws, stream=stream)
+        mk(3)
+        L.pbsa_blockify(g, k, self.q_frames, ca.k_reps, ps, self.dst, ca.k_pool, ps, ws=ws, stream=stream)
+        L.pbsa_blockify(g, v, self.q_frames, self.vreps, ps, self.dst, ca.v_pool, ps, ws=ws, stream=stream)
+        mk(4)
+        L.pbsa_memory_update(g, self.q_reps, self.nq, ca.k_reps, ca.k_pool, ca.v_pool, ps, ca.slot_gid,
+                             ca.slot_ema, c.capacity, c.bpf, self.cs, self.cg, self.ncand, c.gamma,
+                             ca.p_list, ca.p_cnt, ws=ws, stream=stream)
+        mk(5)
+        return o
+
+    def snapshot(self):
+        """Copies of everything ``run`` mutates outside the chunk's own ring positions."""
+        ca, C = self.cache, self.cache.cfg.capacity
+        return [t.clone() for t in (ca.slot_gid, ca.slot_ema, ca.p_list, ca.p_cnt, ca.k_reps[:, :C],
+                                    ca.k_pool[:, :C], ca.v_pool[:, :C])]
+
+    def restore(self, snap):
+        ca, C = self.cache, self.cache.cfg.capacity
+        for dst, src in zip((ca.slot_gid, ca.slot_ema, ca.p_list, ca.p_cnt, ca.k_reps[:, :C],
+                             ca.k_pool[:, :C], ca.v_pool[:, :C]), snap):
+            dst.copy_(src, non_blocking=True)
