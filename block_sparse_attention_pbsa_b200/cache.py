@@ -325,7 +325,11 @@ class ChunkDecodeStep:
         (blockify Q, select, attend, commit blockify K+V, memory update)."""
         ca, c = self.cache, self.cache.cfg
         g, ws, ps = ca.geom, ca.ws, ca.pool_slots
-        mk = (lambda i: marks[i].record(stream)) if marks is not None else (lambda i: None)
+        if marks is not None:
+            ev_stream = stream or torch.cuda.current_stream(self.cache.device)
+            mk = lambda i: marks[i].record(ev_stream)  # noqa: E731
+        else:
+            mk = lambda i: None  # noqa: E731
         mk(0)
         L.pbsa_blockify(g, q, self.q_frames, self.q_reps, self.nq, ws=ws, stream=stream)
         mk(1)
@@ -345,6 +349,20 @@ class ChunkDecodeStep:
                              ca.p_list, ca.p_cnt, ws=ws, stream=stream)
         mk(5)
         return o
+
+    def capture(self, q, k, v, o, lse=None, marks=None) -> torch.cuda.CUDAGraph:
+        """Capture ``run`` in a CUDA graph (one launch replays all kernels of the step).
+
+        Call ``run`` once before capturing (kernel attributes are set on first use).  With
+        ``marks``, pass events created with ``external=True`` so they time inside the graph.
+        """
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(device=self.cache.device)
+        side.wait_stream(torch.cuda.current_stream(self.cache.device))
+        with torch.cuda.graph(graph, stream=side):
+            self.run(q, k, v, o, lse, stream=None, marks=marks)
+        torch.cuda.current_stream(self.cache.device).wait_stream(side)
+        return graph
 
     def snapshot(self):
         """Copies of everything ``run`` mutates outside the chunk's own ring positions."""

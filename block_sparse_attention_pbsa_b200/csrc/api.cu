@@ -3,6 +3,9 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <mutex>
+#include <vector>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -50,6 +53,22 @@ bool pool_ok(const Geo& g, int pool_slots) {
 }
 
 }  // namespace
+
+cudaError_t set_smem_once(const void* kernel, int bytes) {
+  struct Entry { const void* k; int dev; int bytes; };
+  static std::mutex mu;
+  static std::vector<Entry> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const Entry& x : done)
+    if (x.k == kernel && x.dev == dev && x.bytes >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.push_back({kernel, dev, bytes});
+  return e;
+}
+
 }  // namespace pbsa
 
 using namespace pbsa;
@@ -94,7 +113,8 @@ pbsa_status pbsa_score_select(const pbsa_geom* gin, const float* q_reps, int nq,
   if ((prefix_cnt == nullptr) != (prefix_slot == nullptr)) return PBSA_ERR_INVALID_ARG;
   if (prefix_slot == nullptr) prefix_ld = 0;
   if (out_ld < prefix_ld + k) return PBSA_ERR_INVALID_ARG;
-  if (ncand > 2048) return PBSA_ERR_UNSUPPORTED;
+  if (ncand > 1024) return PBSA_ERR_UNSUPPORTED;
+  if (!aligned16(q_reps) || !aligned16(k_reps)) return PBSA_ERR_INVALID_ARG;
   return from_cuda(launch_score_select(g, q_reps, nq, k_reps, pool_slots, cand_slot, cand_gid, ncand,
                                        k, prefix_slot, prefix_cnt, prefix_ld, out_slot, out_cnt,
                                        out_ld, out_score, ws, static_cast<cudaStream_t>(stream)));
@@ -142,8 +162,9 @@ pbsa_status pbsa_memory_update(const pbsa_geom* gin, const float* q_reps, int nq
   if (ncand > 0 && (cand_slot == nullptr || cand_gid == nullptr)) return PBSA_ERR_INVALID_ARG;
   if (!(gamma >= 0.f && gamma <= 1.f)) return PBSA_ERR_INVALID_ARG;
   if (!pool_ok(g, pool_slots) || capacity > pool_slots) return PBSA_ERR_INVALID_ARG;
-  if (!aligned16(k_pool) || !aligned16(v_pool)) return PBSA_ERR_INVALID_ARG;
-  if (capacity + ncand > 4096 || nq > 65535) return PBSA_ERR_UNSUPPORTED;
+  if (!aligned16(k_pool) || !aligned16(v_pool) || !aligned16(k_reps) || !aligned16(q_reps))
+    return PBSA_ERR_INVALID_ARG;
+  if (capacity + ncand > 2048 || nq > 65535) return PBSA_ERR_UNSUPPORTED;
   return from_cuda(launch_memory_update(g, q_reps, nq, k_reps, k_pool, v_pool, pool_slots, slot_gid,
                                         slot_ema, capacity, n_sink_gid, cand_slot, cand_gid, ncand,
                                         gamma, p_list, p_cnt, ws, static_cast<cudaStream_t>(stream)));

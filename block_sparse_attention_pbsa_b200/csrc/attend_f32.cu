@@ -131,8 +131,7 @@ cudaError_t launch_attend_f32(const Geo& g, const float* q, int q_frames, const 
 #define PBSA_AF(DD)                                                                             \
   {                                                                                             \
     const size_t smem = (size_t)(3 * BT * (DD + 1) + BT * 65) * sizeof(float);                  \
-    cudaError_t e = cudaFuncSetAttribute(attend_f32_kernel<DD>,                                 \
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
+    cudaError_t e = set_smem_once((const void*)attend_f32_kernel<DD>, (int)smem);               \
     if (e != cudaSuccess) return e;                                                             \
     attend_f32_kernel<DD><<<dim3(nq, g.H), 256, smem, st>>>(q, g, k_pool, v_pool, pool_slots,   \
                                                             kv_slot, kv_cnt, kv_ld, nq, o, lse, ws); \

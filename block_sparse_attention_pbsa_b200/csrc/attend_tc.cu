@@ -504,8 +504,7 @@ cudaError_t launch_attend_tc(const Geo& g, const void* q, int q_frames, const vo
   prm.o = static_cast<__nv_bfloat16*>(o);
   prm.lse = lse;
   prm.ws = ws;
-  cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)SMEM_BYTES);
+  cudaError_t e = set_smem_once((const void*)attend_tc_kernel, (int)SMEM_BYTES);
   if (e != cudaSuccess) return e;
   dim3 grid((nq + 1) / 2, g.H);
   attend_tc_kernel<<<grid, NTHREADS, SMEM_BYTES, st>>>(qmap, kmap, vmap, prm);

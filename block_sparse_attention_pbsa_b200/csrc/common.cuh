@@ -218,6 +218,45 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// Order-preserving map of a float to uint32 (a > b  <=>  key(a) > key(b); -inf lowest).
+__device__ __forceinline__ uint32_t float_order_key(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+// Ranking key "larger value first, then lower id": compare as unsigned 64-bit, larger wins.
+__device__ __forceinline__ uint64_t rank_key(float value, int id) {
+  return ((uint64_t)float_order_key(value) << 32) | (uint64_t)(0x7FFFFFFFu - (uint32_t)max(id, 0));
+}
+
+// Copy `n` rows of D floats (row i from src_row(i), a 16-byte aligned pointer or nullptr
+// for zeros) into shared memory rows of stride DP floats.  Every thread first issues all of
+// its 16-byte loads (up to 8 at a time), then stores them: the loads overlap in flight.
+template <int D, int DP, int NT, typename RowFn>
+__device__ __forceinline__ void stage_rows(float* dst, int n, RowFn src_row) {
+  constexpr int V = D / 4;  // float4 per row
+  const int total = n * V;
+  for (int base = threadIdx.x; base < total; base += NT * 8) {
+    float4 buf[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = base + u * NT;
+      buf[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (i < total) {
+        const float* row = src_row(i / V);
+        if (row != nullptr) buf[u] = __ldg(reinterpret_cast<const float4*>(row) + (i % V));
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = base + u * NT;
+      if (i < total) {
+        float* d = dst + (i / V) * DP + (i % V) * 4;
+        d[0] = buf[u].x; d[1] = buf[u].y; d[2] = buf[u].z; d[3] = buf[u].w;
+      }
+    }
+  }
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

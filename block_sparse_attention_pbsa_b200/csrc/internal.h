@@ -64,4 +64,8 @@ cudaError_t launch_attend_bwd(const Geo& g, const void* q, int q_frames, const v
 // cuTensorMapEncodeTiled, fetched from the driver at first use (no -lcuda link needed).
 void* tensor_map_encoder();
 
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (kernel, device, size): later
+// calls, including calls made while a stream is being captured, skip the driver call.
+cudaError_t set_smem_once(const void* kernel, int bytes);
+
 }  // namespace pbsa

@@ -103,7 +103,7 @@ PBSA_API pbsa_status pbsa_blockify(const pbsa_geom* g, const void* x, int n_fram
  *   out_score[h][r][i]         = its score (nullable)
  *  q_reps [H][nq][d]; k_reps [H][pool_slots][d]; cand_slot, cand_gid [H][ncand];
  *  prefix_slot [H][prefix_ld]; out_slot [H][nq][out_ld] with out_ld >= prefix_ld + k.
- *  ncand <= 2048. */
+ *  ncand <= 1024. */
 PBSA_API pbsa_status pbsa_score_select(const pbsa_geom* g, const float* q_reps, int nq,
                               const float* k_reps, int pool_slots,
                               const int* cand_slot, const int* cand_gid, int ncand, int k,
@@ -142,7 +142,7 @@ PBSA_API pbsa_status pbsa_attend(const pbsa_geom* g, const void* q, int q_frames
  * candidates in rank order); slot_gid / slot_ema are rewritten (-1 / 0 for empty slots).
  * p_list (nullable out [H][C]) receives the valid persistent slots ascending and p_cnt
  * (nullable out [H]) their count -- the prefix for pbsa_score_select.
- *  Requires C + ncand <= 4096; cand slots must be >= C (outside the persistent region).
+ *  Requires C + ncand <= 2048; cand slots must be >= C (outside the persistent region).
  *  Workspace: pbsa_workspace_bytes(g, nq, C + ncand). */
 PBSA_API pbsa_status pbsa_memory_update(const pbsa_geom* g, const float* q_reps, int nq,
                                float* k_reps, void* k_pool, void* v_pool, int pool_slots,
