@@ -57,6 +57,8 @@ _SIGS = {
     "pbsa_attend": (_I, [ctypes.POINTER(Geom), _P, _I, _P, _P, _I, _P, _P, _I, _P, _P, _P, _P]),
     "pbsa_memory_update": (_I, [ctypes.POINTER(Geom), _P, _I, _P, _P, _P, _I, _P, _P, _I, _I, _P,
                                 _P, _I, ctypes.c_float, _P, _P, _P, _P]),
+    "pbsa_memory_update_noalloc": (_I, [ctypes.POINTER(Geom), _P, _I, _P, _P, _P, _I, _P, _P, _I, _I,
+                                        _P, _P, _I, ctypes.c_float, _P, _P, _P]),
     "pbsa_get_device_error": (_I, [_P, _P]),
     "pbsa_status_string": (ctypes.c_char_p, [_I]),
 }
@@ -159,6 +161,20 @@ def pbsa_memory_update(g: Geom, q_reps, nq, k_reps, k_pool, v_pool, pool_slots, 
         n_sink_gid, _ptr(cand_slot, torch.int32, "cand_slot"), _ptr(cand_gid, torch.int32, "cand_gid"),
         ncand, float(gamma), _ptr(p_list, torch.int32, "p_list"), _ptr(p_cnt, torch.int32, "p_cnt"),
         _ptr(ws, None, "ws"), _stream(stream)))
+
+
+def pbsa_memory_update_noalloc(g: Geom, q_reps, nq, k_reps, k_pool, v_pool, pool_slots, slot_gid,
+                               slot_ema, capacity, n_sink_gid, cand_slot, cand_gid, ncand, gamma,
+                               p_list=None, p_cnt=None, stream=None):
+    """pbsa_memory_update with the library's built-in scratch instead of a workspace."""
+    dt = _tok_dtype(g)
+    _check("pbsa_memory_update_noalloc", load().pbsa_memory_update_noalloc(
+        ctypes.byref(g), _ptr(q_reps, torch.float32, "q_reps"), nq, _ptr(k_reps, torch.float32, "k_reps"),
+        _ptr(k_pool, dt, "k_pool"), _ptr(v_pool, dt, "v_pool"), pool_slots,
+        _ptr(slot_gid, torch.int32, "slot_gid"), _ptr(slot_ema, torch.float32, "slot_ema"), capacity,
+        n_sink_gid, _ptr(cand_slot, torch.int32, "cand_slot"), _ptr(cand_gid, torch.int32, "cand_gid"),
+        ncand, float(gamma), _ptr(p_list, torch.int32, "p_list"), _ptr(p_cnt, torch.int32, "p_cnt"),
+        _stream(stream)))
 
 
 def pbsa_bwd_workspace_bytes(g: Geom, q_frames: int, pool_slots: int, kv_ld: int) -> int:

@@ -150,6 +150,28 @@ PBSA_API pbsa_status pbsa_memory_update(const pbsa_geom* g, const float* q_reps,
                                const int* cand_slot, const int* cand_gid, int ncand,
                                float gamma, int* p_list, int* p_cnt, void* ws, void* stream);
 
+/* pbsa_memory_update without a caller-provided workspace.  The paper has no counterpart;
+ * this is a library convenience for callers that cannot allocate device memory (for
+ * example a plug-in whose host application owns every device allocation, or a runtime
+ * whose memory pools are frozen).  Arguments and results are those of
+ * pbsa_memory_update, minus `ws`: the scratch is a fixed 4 MiB array inside the library,
+ * one per GPU, held from the first call until the process exits.
+ *  - Sizes: requires pbsa_workspace_bytes(g, nq, capacity + ncand) <= 4 MiB (about
+ *    4*H*nq*(capacity + ncand) bytes); larger calls return PBSA_ERR_UNSUPPORTED and
+ *    launch nothing.
+ *  - Set-up: the first call on a device looks up that device's scratch address
+ *    (cudaGetSymbolAddress); make that first call before any stream capture.
+ *  - Sharing: every call uses the same scratch, which keeps the last call's contents;
+ *    calls whose work overlaps on the GPU race.  Device-side index errors are recorded in
+ *    the scratch and not reported.
+ *  - Allocates nothing (no cudaMalloc or allocating library call). */
+PBSA_API pbsa_status pbsa_memory_update_noalloc(const pbsa_geom* g, const float* q_reps, int nq,
+                                                float* k_reps, void* k_pool, void* v_pool,
+                                                int pool_slots, int* slot_gid, float* slot_ema,
+                                                int capacity, int n_sink_gid, const int* cand_slot,
+                                                const int* cand_gid, int ncand, float gamma,
+                                                int* p_list, int* p_cnt, void* stream);
+
 /* Synchronises `stream`, reads and clears the workspace's device error word, and returns
  * it (PBSA_OK when clean). */
 PBSA_API pbsa_status pbsa_get_device_error(void* ws, void* stream);
