@@ -61,12 +61,11 @@ _SIGS = {
                                         _P, _P, _I, ctypes.c_float, _P, _P, _P]),
     "pbsa_get_device_error": (_I, [_P, _P]),
     "pbsa_status_string": (ctypes.c_char_p, [_I]),
-}
-OPTIONAL = {
     "pbsa_bwd_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(Geom), _I, _I, _I]),
     "pbsa_attend_bwd": (_I, [ctypes.POINTER(Geom), _P, _I, _P, _P, _I, _P, _P, _I, _P, _P, _P,
                              _P, _P, _P, _P, _P]),
 }
+OPTIONAL = {}
 
 
 def load(path: str = LIB_PATH) -> ctypes.CDLL:

@@ -21,7 +21,7 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libpbsa.so")
 
 SOURCES = ["api.cu", "blockify.cu", "score_select.cu", "attend_f32.cu", "attend_tc.cu",
-           "memory_update.cu", "noalloc.cu"]
+           "memory_update.cu", "noalloc.cu", "attend_bwd.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          f"-I{os.path.join(ROOT, 'include')}"]

@@ -170,6 +170,34 @@ pbsa_status pbsa_memory_update(const pbsa_geom* gin, const float* q_reps, int nq
                                         gamma, p_list, p_cnt, ws, static_cast<cudaStream_t>(stream)));
 }
 
+size_t pbsa_bwd_workspace_bytes(const pbsa_geom* gin, int q_frames, int pool_slots, int kv_ld) {
+  Geo g;
+  if (make_geo(gin, &g) != PBSA_OK || q_frames <= 0 || pool_slots <= 0 || kv_ld <= 0) return 0;
+  return attend_bwd_ws_bytes(g, q_frames, pool_slots, kv_ld);
+}
+
+pbsa_status pbsa_attend_bwd(const pbsa_geom* gin, const void* q, int q_frames, const void* k_pool,
+                            const void* v_pool, int pool_slots, const int* kv_slot, const int* kv_cnt,
+                            int kv_ld, const void* o, const void* d_o, const float* lse, void* dq,
+                            void* dk_pool, void* dv_pool, void* ws, void* stream) {
+  Geo g;
+  pbsa_status s = make_geo(gin, &g);
+  if (s != PBSA_OK) return s;
+  if (q == nullptr || k_pool == nullptr || v_pool == nullptr || kv_slot == nullptr || kv_cnt == nullptr ||
+      o == nullptr || d_o == nullptr || lse == nullptr || dq == nullptr || dk_pool == nullptr ||
+      dv_pool == nullptr || ws == nullptr)
+    return PBSA_ERR_INVALID_ARG;
+  if (q_frames <= 0 || kv_ld <= 0 || !pool_ok(g, pool_slots)) return PBSA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k_pool, v_pool, o, d_o, dq, dk_pool, dv_pool, ws};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return PBSA_ERR_INVALID_ARG;
+  if (g.dtype != PBSA_BF16 || g.d != 128 || kv_ld > 512) return PBSA_ERR_UNSUPPORTED;
+  const int64_t nq = (int64_t)q_frames * g.bpf;
+  if (nq > 512 || (int64_t)q_frames * g.tpf * g.H > ((int64_t)1 << 31)) return PBSA_ERR_UNSUPPORTED;
+  return from_cuda(launch_attend_bwd(g, q, q_frames, k_pool, v_pool, pool_slots, kv_slot, kv_cnt, kv_ld,
+                                     o, d_o, lse, dq, dk_pool, dv_pool, ws, static_cast<cudaStream_t>(stream)));
+}
+
 pbsa_status pbsa_get_device_error(void* ws, void* stream) {
   if (ws == nullptr) return PBSA_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -1,0 +1,849 @@
+// a5 -- backward of the block-sparse fine attention under the same block lists.
+//
+// Sparse Forcing (gist.science, English 2.D "Training Strategy"; Chinese 2.3): the model is
+// trained with the same dynamic sparse cache as at inference, so the sparse attention
+// needs its gradients.  With P recomputed from the forward's log-sum-exp:
+//   P = exp(scale*Q K^T - LSE),  D_i = dO_i . O_i,  dP = dO V^T,  dS = P * (dP - D),
+//   dV = P^T dO,  dQ = scale * dS K,  dK = scale * dS^T Q.
+//
+// Deterministic design (no floating-point atomics), five launches:
+//   1. bwd_prep_kernel  -- per query block: D and log2-domain LSE in block order, and the
+//      number of query blocks attending each KV slot (integer atomics);
+//   2. bwd_scan_kernel  -- per head: exclusive scan of those counts;
+//   3. bwd_fill_kernel  -- per query block: the inverse lists (KV slot -> query blocks);
+//   4. bwd_dq_kernel    -- one CTA per (head, pair of query blocks), like the forward:
+//      S = Q K^T and dP = dO V^T on tcgen05, dS into TMEM, dQ += dS K with A from TMEM;
+//   5. bwd_dkdv_kernel  -- one CTA per (head, pair of KV slots) over the query blocks that
+//      attend them (sorted, merged with a per-half mask): S^T = K Q^T, dP^T = V dO^T,
+//      dV += P^T dO and dK += dS^T Q with P^T, dS^T read from TMEM.
+#include <math.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace pbsa {
+namespace {
+
+constexpr int D = 128;
+constexpr float LOG2E = 1.4426950408889634f;
+
+__host__ __device__ inline size_t a256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct BwdLayout {
+  size_t dvec, lvec, cnt, off, cur, inv, end;
+};
+__host__ __device__ inline BwdLayout bwd_layout(int H, int nq, int ps, int kv_ld) {
+  BwdLayout L;
+  L.dvec = WS_HEADER_BYTES;
+  L.lvec = L.dvec + a256((size_t)H * nq * BT * 4);
+  L.cnt = L.lvec + a256((size_t)H * nq * BT * 4);
+  L.off = L.cnt + a256((size_t)H * ps * 4);
+  L.cur = L.off + a256((size_t)H * ps * 4);
+  L.inv = L.cur + a256((size_t)H * ps * 4);
+  L.end = L.inv + a256((size_t)H * nq * kv_ld * 4);
+  return L;
+}
+
+struct BwdGeo {
+  int H, nq, kv_ld, pool_slots;
+  int bpf, tpr, tpf, fw, th, tw;
+};
+
+__device__ __forceinline__ size_t token_of(const BwdGeo& g, int r, int row) {
+  const int f = r / g.bpf, rem = r - f * g.bpf;
+  const int ty = rem / g.tpr, tx = rem - ty * g.tpr;
+  const int ly = row / g.tw, lx = row - ly * g.tw;
+  return (size_t)f * g.tpf + (size_t)(ty * g.th + ly) * g.fw + tx * g.tw + lx;
+}
+
+// ---------------------------------------------------------------------------- 1. prep
+// D_i = sum_d dO_i * O_i (fp32 from the bf16 tensors), LSE in log2 units, both in block
+// order; counts of query blocks per KV slot.
+__global__ void __launch_bounds__(64) bwd_prep_kernel(
+    BwdGeo g, const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ d_o,
+    const float* __restrict__ lse, const int* __restrict__ kv_slot, const int* __restrict__ kv_cnt,
+    float* __restrict__ dvec, float* __restrict__ lvec, int* __restrict__ cnt, void* ws) {
+  const int r = blockIdx.x, h = blockIdx.y, row = threadIdx.x;
+  const size_t t = token_of(g, r, row);
+  const uint4* op = reinterpret_cast<const uint4*>(o + (t * g.H + h) * D);
+  const uint4* gp = reinterpret_cast<const uint4*>(d_o + (t * g.H + h) * D);
+  uint4 a[16], b[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    a[i] = __ldg(op + i);
+    b[i] = __ldg(gp + i);
+  }
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint32_t x[4] = {a[i].x, a[i].y, a[i].z, a[i].w};
+    const uint32_t y[4] = {b[i].x, b[i].y, b[i].z, b[i].w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      acc[j] = fmaf(__uint_as_float(x[j] << 16), __uint_as_float(y[j] << 16), acc[j]);
+      acc[j] = fmaf(__uint_as_float(x[j] & 0xFFFF0000u), __uint_as_float(y[j] & 0xFFFF0000u), acc[j]);
+    }
+  }
+  const size_t Tq = (size_t)g.nq / g.bpf * g.tpf;
+  const size_t bi = ((size_t)h * g.nq + r) * BT + row;
+  dvec[bi] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+  lvec[bi] = lse[(size_t)h * Tq + t] * LOG2E;
+  int c = kv_cnt[(size_t)h * g.nq + r];
+  c = min(max(c, 0), g.kv_ld);
+  const int* list = kv_slot + ((size_t)h * g.nq + r) * g.kv_ld;
+  for (int e = row; e < c; e += 64) {
+    const int s = list[e];
+    if (s < 0 || s >= g.pool_slots) {
+      record_error(ws, PBSA_ERR_DEVICE_INDEX, s, K_BWD_PREP);
+      continue;
+    }
+    atomicAdd(cnt + (size_t)h * g.pool_slots + s, 1);
+  }
+}
+
+// ---------------------------------------------------------------------------- 2. scan
+__global__ void __launch_bounds__(1024) bwd_scan_kernel(int ps, const int* __restrict__ cnt,
+                                                       int* __restrict__ off, int* __restrict__ cur) {
+  __shared__ int wsum[32];
+  const int h = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int per = (ps + 1023) / 1024;
+  const int b0 = min(tid * per, ps), b1 = min(b0 + per, ps);
+  const int* c = cnt + (size_t)h * ps;
+  int local = 0;
+  for (int i = b0; i < b1; ++i) local += c[i];
+  int x = local;   // inclusive warp scan
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) wsum[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int v = wsum[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += y;
+    }
+    wsum[lane] = v;
+  }
+  __syncthreads();
+  int run = x - local + (warp > 0 ? wsum[warp - 1] : 0);   // exclusive prefix of this thread
+  for (int i = b0; i < b1; ++i) {
+    off[(size_t)h * ps + i] = run;
+    cur[(size_t)h * ps + i] = 0;
+    run += c[i];
+  }
+}
+
+// ---------------------------------------------------------------------------- 3. fill
+__global__ void __launch_bounds__(64) bwd_fill_kernel(BwdGeo g, const int* __restrict__ kv_slot,
+                                                     const int* __restrict__ kv_cnt,
+                                                     const int* __restrict__ off, int* __restrict__ cur,
+                                                     int* __restrict__ inv) {
+  const int r = blockIdx.x, h = blockIdx.y;
+  int c = kv_cnt[(size_t)h * g.nq + r];
+  c = min(max(c, 0), g.kv_ld);
+  const int* list = kv_slot + ((size_t)h * g.nq + r) * g.kv_ld;
+  for (int e = threadIdx.x; e < c; e += 64) {
+    const int s = list[e];
+    if (s < 0 || s >= g.pool_slots) continue;
+    const size_t hs = (size_t)h * g.pool_slots + s;
+    const int pos = off[hs] + atomicAdd(cur + hs, 1);
+    inv[(size_t)h * g.nq * g.kv_ld + pos] = r;
+  }
+}
+
+__device__ __forceinline__ void wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                              void* ws, int where, int kid) {
+  if (*abort_flag) return;
+  if (!mbar_wait(bar, parity, kWaitLimitNs)) {
+    record_error(ws, PBSA_ERR_TIMEOUT, where, kid);
+    *abort_flag = 1;
+  }
+}
+
+
+// ---------------------------------------------------------------------------- shared pieces
+constexpr int NT = 384;                                 // 12 warps
+constexpr uint32_t REG_CTRL = 56, REG_WORK = 224;       // 128*56 + 256*224 = 384*168
+constexpr uint32_t IDESC_KMAJ = idesc_bf16_f32(128, 128, 0, 0);   // A, B K-major
+constexpr uint32_t IDESC_BMN = idesc_bf16_f32(128, 128, 0, 1);    // B MN-major
+
+// Merge two lists (la[0..cA), lb[0..cB)) into mslot/mflag: A's entries (bit 0, plus bit 1
+// when also in B), then the B-only entries (bit 1), in order.  Returns the merged count.
+// All threads of the CTA call it; it ends with __syncthreads().
+__device__ int merge_pair(const int* la, int cA, const int* lb, int cB, int* mslot, uint8_t* mflag,
+                          uint8_t* onlyb, int* n_out) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int i = tid; i < cA; i += NT) {
+    const int s = la[i];
+    uint8_t f = 1;
+    for (int j = 0; j < cB; ++j) f |= (lb[j] == s) ? 2 : 0;
+    mslot[i] = s;
+    mflag[i] = f;
+  }
+  for (int j = tid; j < cB; j += NT) {
+    const int s = lb[j];
+    bool in_a = false;
+    for (int i = 0; i < cA; ++i) in_a |= (la[i] == s);
+    onlyb[j] = in_a ? 0 : 1;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int pos = cA;
+    for (int base = 0; base < cB; base += 32) {
+      const int j = base + lane;
+      const bool take = j < cB && onlyb[j];
+      const unsigned bal = __ballot_sync(0xffffffffu, take);
+      if (take) {
+        const int at = pos + __popc(bal & ((1u << lane) - 1u));
+        mslot[at] = lb[j];
+        mflag[at] = 2;
+      }
+      pos += __popc(bal);
+    }
+    if (lane == 0) *n_out = pos;
+  }
+  __syncthreads();
+  return *n_out;
+}
+
+// ---------------------------------------------------------------------------- 4. dQ
+// smem: Q | dO (2 panels x [128 rows][128 B] each) | K ring (2) | V ring (2) | barriers | lists
+constexpr uint32_t Q_SM_Q = 0, Q_SM_DO = 32768, Q_SM_K = 65536, Q_SM_V = Q_SM_K + 2 * 32768;
+constexpr uint32_t Q_SM_BAR = Q_SM_V + 2 * 32768;
+constexpr uint32_t Q_SM_MISC = Q_SM_BAR + 256;
+constexpr uint32_t Q_SM_SLOT = Q_SM_MISC + 64;
+constexpr uint32_t Q_SM_FLAG = Q_SM_SLOT + 4 * 1024;
+constexpr uint32_t Q_SM_LA = Q_SM_FLAG + 1024;
+constexpr uint32_t Q_SM_LB = Q_SM_LA + 4 * 512;
+constexpr uint32_t Q_SM_ONLYB = Q_SM_LB + 4 * 512;
+constexpr uint32_t Q_SMEM_BYTES = Q_SM_ONLYB + 512 + 1024;
+enum { QB_QFULL = 0, QB_KFULL = 1, QB_KEMPTY = 3, QB_VFULL = 5, QB_VEMPTY = 7, QB_SFULL = 9,
+       QB_PFULL = 11 /* [w][i&1] */, QB_MMADONE = 15, QB_NUM = 16 };
+
+struct DqParams {
+  BwdGeo g;
+  int kv_rows;
+  float scale, scale_log2;
+  const int* kv_slot;
+  const int* kv_cnt;
+  const float* dvec;
+  const float* lvec;
+  __nv_bfloat16* dq;
+  void* ws;
+};
+
+__global__ void __launch_bounds__(NT, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap domap,
+                  const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+                  const DqParams prm) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Q_SM_BAR);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + Q_SM_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + Q_SM_MISC + 4);
+  int* n_merged_s = reinterpret_cast<int*>(sm + Q_SM_MISC + 8);
+  int* mslot = reinterpret_cast<int*>(sm + Q_SM_SLOT);
+  uint8_t* mflag = sm + Q_SM_FLAG;
+  int* la = reinterpret_cast<int*>(sm + Q_SM_LA);
+  int* lb = reinterpret_cast<int*>(sm + Q_SM_LB);
+  const BwdGeo& g = prm.g;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int h = blockIdx.y, rA = 2 * blockIdx.x, rB = rA + 1;
+  const bool hasB = rB < g.nq;
+
+  if (tid == 0) {
+    for (int i = 0; i < QB_NUM; ++i) mbar_init(&bars[i], 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&bars[QB_PFULL + i], 128);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+  int cA = prm.kv_cnt[(size_t)h * g.nq + rA];
+  int cB = hasB ? prm.kv_cnt[(size_t)h * g.nq + rB] : 0;
+  cA = min(max(cA, 0), g.kv_ld);
+  cB = min(max(cB, 0), g.kv_ld);
+  const int* listA = prm.kv_slot + ((size_t)h * g.nq + rA) * g.kv_ld;
+  const int* listB = prm.kv_slot + ((size_t)h * g.nq + (hasB ? rB : rA)) * g.kv_ld;
+  for (int i = tid; i < cA; i += NT) la[i] = listA[i];
+  for (int i = tid; i < cB; i += NT) lb[i] = listB[i];
+  __syncthreads();
+  const int n = merge_pair(la, cA, lb, cB, mslot, mflag, sm + Q_SM_ONLYB, n_merged_s);
+  for (int i = tid; i < n; i += NT) {
+    const int s = mslot[i];
+    if (s < 0 || s >= g.pool_slots) {
+      record_error(prm.ws, PBSA_ERR_DEVICE_INDEX, s, K_BWD_Q);
+      mslot[i] = -1;
+      mflag[i] = 0;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const int nsteps = (n + 1) >> 1;
+
+  if (warp < 4) {
+    setmaxnreg_dec<REG_CTRL>();
+    if (warp == 0 && lane == 0 && nsteps > 0) {
+      // ---- producer: Q and dO once, then K, V of each step
+      tma_prefetch_desc(&qmap);
+      tma_prefetch_desc(&domap);
+      tma_prefetch_desc(&kmap);
+      tma_prefetch_desc(&vmap);
+      mbar_arrive_expect_tx(&bars[QB_QFULL], 65536);
+      for (int half = 0; half < 2; ++half) {
+        const int r = (half == 1 && hasB) ? rB : rA;
+        const int f = r / g.bpf, rem = r - f * g.bpf;
+        const int ty = rem / g.tpr, tx = rem - ty * g.tpr;
+        for (int p = 0; p < 2; ++p) {
+          tma_load_5d(sm + Q_SM_Q + p * 16384 + half * 8192, &qmap, &bars[QB_QFULL], p * 64, h, tx * g.tw, ty * g.th, f);
+          tma_load_5d(sm + Q_SM_DO + p * 16384 + half * 8192, &domap, &bars[QB_QFULL], p * 64, h, tx * g.tw, ty * g.th, f);
+        }
+      }
+      auto load_pair = [&](const CUtensorMap* map, uint8_t* dst, uint64_t* bar, int i) {
+        for (int b = 0; b < 2; ++b) {
+          const int e = 2 * i + b;
+          const int slot = e < n ? mslot[e] : -1;
+          const int row0 = slot >= 0 ? (h * g.pool_slots + slot) * 64 : prm.kv_rows;
+          for (int p = 0; p < 2; ++p) tma_load_2d(dst + p * 16384 + b * 8192, map, bar, p * 64, row0);
+        }
+      };
+      int kiss = 0, viss = 0;
+      for (int i = 0; i < nsteps; ++i) {
+        const int s = i & 1;
+        wait_or_abort(&bars[QB_KEMPTY + s], ((i >> 1) & 1) ^ 1, abort_flag, prm.ws, 1, K_BWD_Q);
+        if (*abort_flag) break;
+        mbar_arrive_expect_tx(&bars[QB_KFULL + s], 32768);
+        load_pair(&kmap, sm + Q_SM_K + s * 32768, &bars[QB_KFULL + s], i);
+        kiss = i + 1;
+        wait_or_abort(&bars[QB_VEMPTY + s], ((i >> 1) & 1) ^ 1, abort_flag, prm.ws, 2, K_BWD_Q);
+        if (*abort_flag) break;
+        mbar_arrive_expect_tx(&bars[QB_VFULL + s], 32768);
+        load_pair(&vmap, sm + Q_SM_V + s * 32768, &bars[QB_VFULL + s], i);
+        viss = i + 1;
+      }
+      if (*abort_flag) {
+        mbar_wait(&bars[QB_QFULL], 0, kWaitLimitNs);
+        for (int i = (kiss > 2 ? kiss - 2 : 0); i < kiss; ++i) mbar_wait(&bars[QB_KFULL + (i & 1)], (i >> 1) & 1, kWaitLimitNs);
+        for (int i = (viss > 2 ? viss - 2 : 0); i < viss; ++i) mbar_wait(&bars[QB_VFULL + (i & 1)], (i >> 1) & 1, kWaitLimitNs);
+      }
+    }
+    if (warp == 1 && lane == 0 && nsteps > 0) {
+      // ---- MMA issuer.  TMEM: S[i&1] at 128*(i&1), dP at 256, dQ at 384.
+      const uint32_t q_base = smem_u32(sm + Q_SM_Q), do_base = smem_u32(sm + Q_SM_DO);
+      const uint32_t k_base = smem_u32(sm + Q_SM_K), v_base = smem_u32(sm + Q_SM_V);
+      auto issue_dq = [&](int j) {
+        const int s = j & 1;
+        for (int w = 0; w < 2; ++w) {
+          wait_or_abort(&bars[QB_PFULL + 2 * w + (j & 1)], (j >> 1) & 1, abort_flag, prm.ws, 3, K_BWD_Q);
+          if (*abort_flag) return;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t b = sw128_desc(k_base + s * 32768 + w * 8192 + kk * 2048, 16384, 1024);
+            mma_bf16_ts(tmem + 384, tmem + (j & 1) * 128 + w * 64 + kk * 8, b, IDESC_BMN,
+                        (j > 0 || w > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        mma_commit(&bars[QB_KEMPTY + s]);
+      };
+      wait_or_abort(&bars[QB_QFULL], 0, abort_flag, prm.ws, 4, K_BWD_Q);
+      for (int i = 0; i < nsteps && !*abort_flag; ++i) {
+        const int s = i & 1;
+        wait_or_abort(&bars[QB_KFULL + s], (i >> 1) & 1, abort_flag, prm.ws, 5, K_BWD_Q);
+        if (*abort_flag) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t a = sw128_desc(q_base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+          const uint64_t b = sw128_desc(k_base + s * 32768 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+          mma_bf16_ss(tmem + (i & 1) * 128, a, b, IDESC_KMAJ, kk > 0 ? 1u : 0u);
+        }
+        // dS(i-1) has been consumed by the softmax side once its P-full arrives; that also
+        // frees the single dP buffer for dP(i)
+        if (i >= 1) issue_dq(i - 1);
+        if (*abort_flag) break;
+        wait_or_abort(&bars[QB_VFULL + s], (i >> 1) & 1, abort_flag, prm.ws, 6, K_BWD_Q);
+        if (*abort_flag) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t a = sw128_desc(do_base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+          const uint64_t b = sw128_desc(v_base + s * 32768 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+          mma_bf16_ss(tmem + 256, a, b, IDESC_KMAJ, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&bars[QB_SFULL + (i & 1)]);
+        mma_commit(&bars[QB_VEMPTY + s]);
+      }
+      if (!*abort_flag) issue_dq(nsteps - 1);
+      mma_commit(&bars[QB_MMADONE]);
+      mbar_wait(&bars[QB_MMADONE], 0, kWaitLimitNs);
+    }
+    __syncwarp();
+  } else {
+    setmaxnreg_inc<REG_WORK>();
+    // ---- dS = P * (dP - D) for the block of the step this warpgroup owns
+    const int wg = (warp - 4) >> 2, wq = warp & 3;
+    const int row = wq * 32 + lane, half = row >> 6;
+    const bool row_valid = half == 0 || hasB;
+    const int r = half ? rB : rA;
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const size_t bi = ((size_t)h * g.nq + (row_valid ? r : rA)) * BT + (row & 63);
+    const float lse2 = prm.lvec[bi], dd = prm.dvec[bi];
+    const float c = prm.scale_log2;
+    for (int i = 0; i < nsteps; ++i) {
+      const int e = 2 * i + wg;
+      const bool v = row_valid && e < n && ((mflag[e] >> half) & 1);
+      const uint32_t tS = tmem + lane_off + (i & 1) * 128 + wg * 64;
+      const uint32_t tP = tmem + lane_off + 256 + wg * 64;
+      wait_or_abort(&bars[QB_SFULL + (i & 1)], (i >> 1) & 1, abort_flag, prm.ws, 7, K_BWD_Q);
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+      tc_fence_after();
+      uint32_t xs[2][32], xp[2][32];
+      if (__any_sync(0xffffffffu, v)) {
+        tmem_ld32(tS, xs[0]);
+        tmem_ld32(tS + 32, xs[1]);
+        tmem_ld32(tP, xp[0]);
+        tmem_ld32(tP + 32, xp[1]);
+        tmem_wait_ld();
+      }
+      uint32_t pk[32];
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+#pragma unroll
+        for (int e2 = 0; e2 < 16; ++e2) {
+          float d0 = 0.f, d1 = 0.f;
+          if (v) {
+            const float p0 = ex2_approx(fmaf(__uint_as_float(xs[q][2 * e2]), c, -lse2));
+            const float p1 = ex2_approx(fmaf(__uint_as_float(xs[q][2 * e2 + 1]), c, -lse2));
+            d0 = p0 * (__uint_as_float(xp[q][2 * e2]) - dd);
+            d1 = p1 * (__uint_as_float(xp[q][2 * e2 + 1]) - dd);
+          }
+          pk[q * 16 + e2] = pack_bf16(d0, d1);
+        }
+      }
+      tmem_st32(tS, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars[QB_PFULL + 2 * wg + (i & 1)]);
+    }
+    // ---- epilogue: dQ = scale * (dS K) -> bf16 raster rows; warpgroup w writes columns [64w, +64)
+    if (nsteps > 0) wait_or_abort(&bars[QB_MMADONE], 0, abort_flag, prm.ws, 8, K_BWD_Q);
+    if (row_valid && !__any_sync(0xffffffffu, *abort_flag != 0)) {
+      const size_t t = token_of(g, r, row & 63);
+      uint4* dst = reinterpret_cast<uint4*>(prm.dq + (t * g.H + h) * D) + wg * 8;
+      tc_fence_after();
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        uint32_t ov[32];
+        if (nsteps > 0) {
+          tmem_ld32(tmem + lane_off + 384 + wg * 64 + q * 32, ov);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e2 = 0; e2 < 32; ++e2) ov[e2] = 0u;
+        }
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t wv[4];
+#pragma unroll
+          for (int e2 = 0; e2 < 4; ++e2)
+            wv[e2] = pack_bf16(__uint_as_float(ov[cc * 8 + 2 * e2]) * prm.scale,
+                               __uint_as_float(ov[cc * 8 + 2 * e2 + 1]) * prm.scale);
+          dst[q * 4 + cc] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+
+// ---------------------------------------------------------------------------- 5. dK, dV
+// smem: K pair | V pair (2 panels x [128 keys][128 B] each) | 2 stages x (Q, dO tiles of two
+// query blocks, their log2-LSE and D rows) | barriers | lists
+constexpr uint32_t KV_SM_K = 0, KV_SM_V = 32768, KV_SM_Q = 65536;    // Q stage s at +65536*s
+constexpr uint32_t KV_STAGE = 65536;                                 // Q (32 KB) + dO (32 KB)
+constexpr uint32_t KV_SM_VEC = KV_SM_Q + 2 * KV_STAGE;               // 2 stages x [lse2 | D] x 2 blocks x 64 f32
+constexpr uint32_t KV_SM_BAR = KV_SM_VEC + 2 * 1024;
+constexpr uint32_t KV_SM_MISC = KV_SM_BAR + 256;
+constexpr uint32_t KV_SM_SLOT = KV_SM_MISC + 64;
+constexpr uint32_t KV_SM_FLAG = KV_SM_SLOT + 4 * 1024;
+constexpr uint32_t KV_SM_LA = KV_SM_FLAG + 1024;
+constexpr uint32_t KV_SM_LB = KV_SM_LA + 4 * 512;
+constexpr uint32_t KV_SM_ONLYB = KV_SM_LB + 4 * 512;
+constexpr uint32_t KV_SM_TMP = KV_SM_ONLYB + 512;                    // int[512] sort scratch
+constexpr uint32_t KV_SMEM_BYTES = KV_SM_TMP + 4 * 512 + 1024;
+enum { KB_KVFULL = 0, KB_QFULL = 1, KB_QEMPTY = 3, KB_SFULL = 5, KB_PFULL = 6 /* [w] */,
+       KB_MMADONE = 8, KB_NUM = 9 };
+
+struct DkvParams {
+  BwdGeo g;
+  int kv_rows;
+  int q_frames;
+  float scale, scale_log2;
+  const int* cnt;
+  const int* off;
+  const int* inv;
+  const float* dvec;
+  const float* lvec;
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  void* ws;
+};
+
+// Sort src[0..n) ascending into dst by rank counting (n <= 512; entries distinct or not).
+__device__ void sort_small(const int* src, int n, int* dst) {
+  for (int i = threadIdx.x; i < n; i += NT) {
+    const int x = src[i];
+    int rk = 0;
+    for (int j = 0; j < n; ++j) {
+      const int y = src[j];
+      rk += (y < x) | ((y == x) & (j < i));
+    }
+    dst[rk] = x;
+  }
+}
+
+__global__ void __launch_bounds__(NT, 1)
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap domap,
+                    const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+                    const DkvParams prm) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + KV_SM_BAR);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + KV_SM_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + KV_SM_MISC + 4);
+  int* n_merged_s = reinterpret_cast<int*>(sm + KV_SM_MISC + 8);
+  int* mslot = reinterpret_cast<int*>(sm + KV_SM_SLOT);     // merged query blocks
+  uint8_t* mflag = sm + KV_SM_FLAG;                         // bit k: attends KV slot 2p + k
+  int* la = reinterpret_cast<int*>(sm + KV_SM_LA);
+  int* lb = reinterpret_cast<int*>(sm + KV_SM_LB);
+  int* tmp = reinterpret_cast<int*>(sm + KV_SM_TMP);
+  const BwdGeo& g = prm.g;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int h = blockIdx.y, sA = 2 * blockIdx.x, sB = sA + 1;
+  const bool hasB = sB < g.pool_slots;
+
+  if (tid == 0) {
+    for (int i = 0; i < KB_NUM; ++i) mbar_init(&bars[i], 1);
+    mbar_init(&bars[KB_PFULL + 0], 128);
+    mbar_init(&bars[KB_PFULL + 1], 128);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+  // the query blocks attending each of the two slots, sorted (the inverse lists are filled
+  // with atomics, so their order is not reproducible until sorted)
+  const size_t hb = (size_t)h * g.pool_slots;
+  const int* invh = prm.inv + (size_t)h * g.nq * g.kv_ld;
+  int cA = prm.cnt[hb + sA], cB = hasB ? prm.cnt[hb + sB] : 0;
+  if (cA > 512 || cB > 512) {
+    if (tid == 0) record_error(prm.ws, PBSA_ERR_UNSUPPORTED, max(cA, cB), K_BWD_KV);
+    cA = min(cA, 512);
+    cB = min(cB, 512);
+  }
+  for (int i = tid; i < cA; i += NT) tmp[i] = invh[prm.off[hb + sA] + i];
+  __syncthreads();
+  sort_small(tmp, cA, la);
+  __syncthreads();
+  if (hasB)
+    for (int i = tid; i < cB; i += NT) tmp[i] = invh[prm.off[hb + sB] + i];
+  __syncthreads();
+  sort_small(tmp, cB, lb);
+  __syncthreads();
+  const int n = merge_pair(la, cA, lb, cB, mslot, mflag, sm + KV_SM_ONLYB, n_merged_s);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const int nsteps = (n + 1) >> 1;
+  float* vecs = reinterpret_cast<float*>(sm + KV_SM_VEC);  // [stage][lse2 blk0, lse2 blk1, D blk0, D blk1][64]
+
+  if (warp < 4) {
+    setmaxnreg_dec<REG_CTRL>();
+    if (warp == 0 && lane == 0 && nsteps > 0) {
+      // ---- producer: the K, V pair once; then Q, dO, log2-LSE, D of two query blocks per step
+      tma_prefetch_desc(&qmap);
+      tma_prefetch_desc(&domap);
+      tma_prefetch_desc(&kmap);
+      tma_prefetch_desc(&vmap);
+      mbar_arrive_expect_tx(&bars[KB_KVFULL], 65536);
+      for (int b = 0; b < 2; ++b) {
+        const int row0 = (b == 0 || hasB) ? (h * g.pool_slots + sA + b) * 64 : prm.kv_rows;
+        for (int p = 0; p < 2; ++p) {
+          tma_load_2d(sm + KV_SM_K + p * 16384 + b * 8192, &kmap, &bars[KB_KVFULL], p * 64, row0);
+          tma_load_2d(sm + KV_SM_V + p * 16384 + b * 8192, &vmap, &bars[KB_KVFULL], p * 64, row0);
+        }
+      }
+      int iss = 0;
+      for (int i = 0; i < nsteps; ++i) {
+        const int s = i & 1;
+        wait_or_abort(&bars[KB_QEMPTY + s], ((i >> 1) & 1) ^ 1, abort_flag, prm.ws, 1, K_BWD_KV);
+        if (*abort_flag) break;
+        mbar_arrive_expect_tx(&bars[KB_QFULL + s], KV_STAGE + 4 * 256);
+        uint8_t* qdst = sm + KV_SM_Q + s * KV_STAGE;
+        float* vdst = vecs + s * 256;
+        for (int b = 0; b < 2; ++b) {
+          const int e = 2 * i + b;
+          const bool real = e < n;
+          const int r = real ? mslot[e] : mslot[2 * i];
+          const int f = real ? r / g.bpf : prm.q_frames;   // a missing block is loaded out of bounds
+          const int rem = r - (r / g.bpf) * g.bpf;
+          const int ty = rem / g.tpr, tx = rem - ty * g.tpr;
+          for (int p = 0; p < 2; ++p) {
+            tma_load_5d(qdst + p * 16384 + b * 8192, &qmap, &bars[KB_QFULL + s], p * 64, h, tx * g.tw, ty * g.th, f);
+            tma_load_5d(qdst + 32768 + p * 16384 + b * 8192, &domap, &bars[KB_QFULL + s], p * 64, h, tx * g.tw,
+                        ty * g.th, f);
+          }
+          const size_t bi = ((size_t)h * g.nq + r) * BT;
+          bulk_load(vdst + b * 64, prm.lvec + bi, 256, &bars[KB_QFULL + s]);
+          bulk_load(vdst + 128 + b * 64, prm.dvec + bi, 256, &bars[KB_QFULL + s]);
+        }
+        iss = i + 1;
+      }
+      if (*abort_flag) {
+        mbar_wait(&bars[KB_KVFULL], 0, kWaitLimitNs);
+        for (int i = (iss > 2 ? iss - 2 : 0); i < iss; ++i) mbar_wait(&bars[KB_QFULL + (i & 1)], (i >> 1) & 1, kWaitLimitNs);
+      }
+    }
+    if (warp == 1 && lane == 0 && nsteps > 0) {
+      // ---- MMA issuer.  TMEM: S^T at 0, dP^T at 128, dV at 256, dK at 384 (keys on lanes).
+      const uint32_t k_base = smem_u32(sm + KV_SM_K), v_base = smem_u32(sm + KV_SM_V);
+      wait_or_abort(&bars[KB_KVFULL], 0, abort_flag, prm.ws, 2, K_BWD_KV);
+      for (int i = 0; i < nsteps && !*abort_flag; ++i) {
+        const int s = i & 1;
+        const uint32_t q_base = smem_u32(sm + KV_SM_Q + s * KV_STAGE), do_base = q_base + 32768;
+        wait_or_abort(&bars[KB_QFULL + s], (i >> 1) & 1, abort_flag, prm.ws, 3, K_BWD_KV);
+        if (*abort_flag) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {   // S^T = K Q^T and dP^T = V dO^T (M = 128 keys, N = 128 queries)
+          const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_bf16_ss(tmem + 0, sw128_desc(k_base + ko, 16, 1024), sw128_desc(q_base + ko, 16, 1024),
+                      IDESC_KMAJ, kk > 0 ? 1u : 0u);
+          mma_bf16_ss(tmem + 128, sw128_desc(v_base + ko, 16, 1024), sw128_desc(do_base + ko, 16, 1024),
+                      IDESC_KMAJ, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&bars[KB_SFULL]);
+        for (int w = 0; w < 2; ++w) {
+          wait_or_abort(&bars[KB_PFULL + w], i & 1, abort_flag, prm.ws, 4, K_BWD_KV);
+          if (*abort_flag) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {   // dV += P^T dO_w, dK += dS^T Q_w (queries of block w)
+            const uint32_t bo = w * 8192 + kk * 2048;
+            const uint32_t acc = (i > 0 || w > 0 || kk > 0) ? 1u : 0u;
+            mma_bf16_ts(tmem + 256, tmem + 0 + w * 64 + kk * 8, sw128_desc(do_base + bo, 16384, 1024), IDESC_BMN, acc);
+            mma_bf16_ts(tmem + 384, tmem + 128 + w * 64 + kk * 8, sw128_desc(q_base + bo, 16384, 1024), IDESC_BMN, acc);
+          }
+        }
+        mma_commit(&bars[KB_QEMPTY + s]);
+      }
+      mma_commit(&bars[KB_MMADONE]);
+      mbar_wait(&bars[KB_MMADONE], 0, kWaitLimitNs);
+    }
+    __syncwarp();
+  } else {
+    setmaxnreg_inc<REG_WORK>();
+    // ---- P^T and dS^T for the query block of the step this warpgroup owns; lanes are keys
+    const int wg = (warp - 4) >> 2, wq = warp & 3;
+    const int row = wq * 32 + lane, kh = row >> 6;   // key row, which slot of the pair
+    const bool row_valid = kh == 0 || hasB;
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const float c = prm.scale_log2;
+    for (int i = 0; i < nsteps; ++i) {
+      const int e = 2 * i + wg;
+      const bool v = row_valid && e < n && ((mflag[e] >> kh) & 1);
+      const uint32_t tS = tmem + lane_off + wg * 64, tD = tmem + lane_off + 128 + wg * 64;
+      const float* lse2 = vecs + (i & 1) * 256 + wg * 64;
+      const float* dd = vecs + (i & 1) * 256 + 128 + wg * 64;
+      // the step's log2-LSE / D rows arrived with its Q-full barrier (TMA bulk copies)
+      wait_or_abort(&bars[KB_QFULL + (i & 1)], (i >> 1) & 1, abort_flag, prm.ws, 7, K_BWD_KV);
+      wait_or_abort(&bars[KB_SFULL], i & 1, abort_flag, prm.ws, 5, K_BWD_KV);
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+      tc_fence_after();
+      uint32_t xs[2][32], xp[2][32];
+      if (__any_sync(0xffffffffu, v)) {
+        tmem_ld32(tS, xs[0]);
+        tmem_ld32(tS + 32, xs[1]);
+        tmem_ld32(tD, xp[0]);
+        tmem_ld32(tD + 32, xp[1]);
+        tmem_wait_ld();
+      }
+      uint32_t pp[32], pd[32];
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+#pragma unroll
+        for (int e2 = 0; e2 < 16; ++e2) {
+          const int c0 = q * 32 + 2 * e2;
+          float p0 = 0.f, p1 = 0.f, d0 = 0.f, d1 = 0.f;
+          if (v) {
+            p0 = ex2_approx(fmaf(__uint_as_float(xs[q][2 * e2]), c, -lse2[c0]));
+            p1 = ex2_approx(fmaf(__uint_as_float(xs[q][2 * e2 + 1]), c, -lse2[c0 + 1]));
+            d0 = p0 * (__uint_as_float(xp[q][2 * e2]) - dd[c0]);
+            d1 = p1 * (__uint_as_float(xp[q][2 * e2 + 1]) - dd[c0 + 1]);
+          }
+          pp[q * 16 + e2] = pack_bf16(p0, p1);
+          pd[q * 16 + e2] = pack_bf16(d0, d1);
+        }
+      }
+      tmem_st32(tS, pp);
+      tmem_st32(tD, pd);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars[KB_PFULL + wg]);
+    }
+    // ---- epilogue: dV and dK = scale * (dS^T Q) rows of the pair's slots, warpgroup w
+    // writes columns [64w, +64) of both
+    if (nsteps > 0) wait_or_abort(&bars[KB_MMADONE], 0, abort_flag, prm.ws, 6, K_BWD_KV);
+    if (row_valid && !__any_sync(0xffffffffu, *abort_flag != 0)) {
+      const size_t base = (((size_t)h * g.pool_slots + sA + kh) * BT + (row & 63)) * D;
+      uint4* dvd = reinterpret_cast<uint4*>(prm.dv + base) + wg * 8;
+      uint4* dkd = reinterpret_cast<uint4*>(prm.dk + base) + wg * 8;
+      tc_fence_after();
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        uint32_t a[32], b[32];
+        if (nsteps > 0) {
+          tmem_ld32(tmem + lane_off + 256 + wg * 64 + q * 32, a);
+          tmem_ld32(tmem + lane_off + 384 + wg * 64 + q * 32, b);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e2 = 0; e2 < 32; ++e2) a[e2] = b[e2] = 0u;
+        }
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t wa[4], wb[4];
+#pragma unroll
+          for (int e2 = 0; e2 < 4; ++e2) {
+            const int k0 = cc * 8 + 2 * e2;
+            wa[e2] = pack_bf16(__uint_as_float(a[k0]), __uint_as_float(a[k0 + 1]));
+            wb[e2] = pack_bf16(__uint_as_float(b[k0]) * prm.scale, __uint_as_float(b[k0 + 1]) * prm.scale);
+          }
+          dvd[q * 4 + cc] = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+          dkd[q * 4 + cc] = make_uint4(wb[0], wb[1], wb[2], wb[3]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+size_t attend_bwd_ws_bytes(const Geo& g, int q_frames, int pool_slots, int kv_ld) {
+  return bwd_layout(g.H, q_frames * g.bpf, pool_slots, kv_ld).end;
+}
+
+cudaError_t launch_attend_bwd(const Geo& gg, const void* q, int q_frames, const void* k_pool,
+                              const void* v_pool, int pool_slots, const int* kv_slot,
+                              const int* kv_cnt, int kv_ld, const void* o, const void* d_o,
+                              const float* lse, void* dq, void* dk_pool, void* dv_pool, void* ws,
+                              cudaStream_t st) {
+  if (gg.d != D || gg.dtype != PBSA_BF16) return cudaErrorNotSupported;
+  BwdGeo g;
+  g.H = gg.H;
+  g.nq = q_frames * gg.bpf;
+  g.kv_ld = kv_ld;
+  g.pool_slots = pool_slots;
+  g.bpf = gg.bpf;
+  g.tpr = gg.tpr;
+  g.tpf = gg.tpf;
+  g.fw = gg.fw;
+  g.th = gg.th;
+  g.tw = gg.tw;
+  const BwdLayout L = bwd_layout(g.H, g.nq, pool_slots, kv_ld);
+  char* base = static_cast<char*>(ws);
+  float* dvec = reinterpret_cast<float*>(base + L.dvec);
+  float* lvec = reinterpret_cast<float*>(base + L.lvec);
+  int* cnt = reinterpret_cast<int*>(base + L.cnt);
+  int* off = reinterpret_cast<int*>(base + L.off);
+  int* cur = reinterpret_cast<int*>(base + L.cur);
+  int* inv = reinterpret_cast<int*>(base + L.inv);
+  cudaError_t e;
+  if ((e = cudaMemsetAsync(cnt, 0, (size_t)g.H * pool_slots * 4, st)) != cudaSuccess) return e;
+
+  CUtensorMap qmap, domap, kmap, vmap;
+  {
+    const cuuint64_t dims[5] = {(cuuint64_t)D, (cuuint64_t)g.H, (cuuint64_t)gg.fw, (cuuint64_t)gg.fh,
+                                (cuuint64_t)q_frames};
+    const cuuint64_t row = (cuuint64_t)D * 2;
+    const cuuint64_t strides[4] = {row, row * g.H, row * g.H * gg.fw, row * g.H * gg.fw * gg.fh};
+    const cuuint32_t box[5] = {64, 1, (cuuint32_t)gg.tw, (cuuint32_t)gg.th, 1};
+    if (!encode_bf16(&qmap, q, 5, dims, strides, box)) return cudaErrorNotSupported;
+    if (!encode_bf16(&domap, d_o, 5, dims, strides, box)) return cudaErrorNotSupported;
+  }
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)g.H * pool_slots * BT};
+    const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t box[2] = {64, 64};
+    if (!encode_bf16(&kmap, k_pool, 2, dims, strides, box)) return cudaErrorNotSupported;
+    if (!encode_bf16(&vmap, v_pool, 2, dims, strides, box)) return cudaErrorNotSupported;
+  }
+  const float scale = gg.scale;
+  bwd_prep_kernel<<<dim3(g.nq, g.H), 64, 0, st>>>(g, static_cast<const __nv_bfloat16*>(o),
+                                                   static_cast<const __nv_bfloat16*>(d_o), lse, kv_slot,
+                                                   kv_cnt, dvec, lvec, cnt, ws);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  bwd_scan_kernel<<<g.H, 1024, 0, st>>>(pool_slots, cnt, off, cur);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  bwd_fill_kernel<<<dim3(g.nq, g.H), 64, 0, st>>>(g, kv_slot, kv_cnt, off, cur, inv);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+  DqParams dp;
+  dp.g = g;
+  dp.kv_rows = g.H * pool_slots * BT;
+  dp.scale = scale;
+  dp.scale_log2 = scale * LOG2E;
+  dp.kv_slot = kv_slot;
+  dp.kv_cnt = kv_cnt;
+  dp.dvec = dvec;
+  dp.lvec = lvec;
+  dp.dq = static_cast<__nv_bfloat16*>(dq);
+  dp.ws = ws;
+  if ((e = set_smem_once((const void*)bwd_dq_kernel, (int)Q_SMEM_BYTES)) != cudaSuccess) return e;
+  bwd_dq_kernel<<<dim3((g.nq + 1) / 2, g.H), NT, Q_SMEM_BYTES, st>>>(qmap, domap, kmap, vmap, dp);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+  DkvParams kp;
+  kp.g = g;
+  kp.kv_rows = g.H * pool_slots * BT;
+  kp.q_frames = q_frames;
+  kp.scale = scale;
+  kp.scale_log2 = scale * LOG2E;
+  kp.cnt = cnt;
+  kp.off = off;
+  kp.inv = inv;
+  kp.dvec = dvec;
+  kp.lvec = lvec;
+  kp.dk = static_cast<__nv_bfloat16*>(dk_pool);
+  kp.dv = static_cast<__nv_bfloat16*>(dv_pool);
+  kp.ws = ws;
+  if ((e = set_smem_once((const void*)bwd_dkdv_kernel, (int)KV_SMEM_BYTES)) != cudaSuccess) return e;
+  bwd_dkdv_kernel<<<dim3((pool_slots + 1) / 2, g.H), NT, KV_SMEM_BYTES, st>>>(qmap, domap, kmap, vmap, kp);
+  return cudaGetLastError();
+}
+
+}  // namespace pbsa

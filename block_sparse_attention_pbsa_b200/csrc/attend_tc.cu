@@ -451,7 +451,6 @@ void* tensor_map_encoder() {
   return fn;
 }
 
-namespace {
 // bf16 tensor map with 128-byte swizzle; dims/strides fastest first (strides in bytes, rank-1).
 bool encode_bf16(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
                  const cuuint64_t* strides, const cuuint32_t* box) {
@@ -462,7 +461,6 @@ bool encode_bf16(CUtensorMap* m, const void* base, int rank, const cuuint64_t* d
              strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
-}  // namespace
 
 cudaError_t launch_attend_tc(const Geo& g, const void* q, int q_frames, const void* k_pool,
                              const void* v_pool, int pool_slots, const int* kv_slot,

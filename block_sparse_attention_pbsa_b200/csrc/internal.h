@@ -1,5 +1,6 @@
 // Host-side declarations shared by the translation units of libpbsa.
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -63,6 +64,9 @@ cudaError_t launch_attend_bwd(const Geo& g, const void* q, int q_frames, const v
 
 // cuTensorMapEncodeTiled, fetched from the driver at first use (no -lcuda link needed).
 void* tensor_map_encoder();
+// Encode a bf16 tensor map with 128-byte swizzle (dims/strides fastest first, strides in bytes).
+bool encode_bf16(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
+                 const cuuint64_t* strides, const cuuint32_t* box);
 
 // cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (kernel, device, size): later
 // calls, including calls made while a stream is being captured, skip the driver call.

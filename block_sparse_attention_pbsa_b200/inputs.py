@@ -201,3 +201,36 @@ def train_inputs(w: Workload, *, device="cpu"):
         outs.append(torch.randn((w.batch, T, w.heads, w.head_dim), generator=g, device=device)
                     .to(w.torch_dtype))
     return tuple(outs)
+
+
+def train_lists(w: Workload, seed: int, n_frames: int | None = None, batch: int | None = None):
+    """Block lists of the trainable-path workload, with the batch folded into the frame axis.
+
+    Query block r of batch b (global block id b*F*bpf + r, F = frames per sequence) attends:
+    its own chunk's blocks; and, for chunks after the first, the sink blocks (frame 0 of its
+    sequence) plus ``topk`` blocks drawn uniformly (seeded) from the earlier non-sink blocks
+    of its sequence -- a fixed mask with the structure the trainable path uses, standing in
+    for a learned selection.  Pool slot = global block id.  Returns a list over heads of
+    lists over query blocks of slot lists.
+    """
+    F = n_frames or w.total_frames
+    B = batch or w.batch
+    bpf, cf = w.blocks_per_frame, w.chunk_frames
+    g = _gen("cpu", seed)
+    out = []
+    for h in range(w.heads):
+        rows = []
+        for b in range(B):
+            base = b * F * bpf
+            for r in range(F * bpf):
+                c = (r // bpf) // cf
+                own = list(range(base + c * cf * bpf, base + min((c + 1) * cf, F) * bpf))
+                if c == 0:
+                    rows.append(own)
+                    continue
+                earlier = list(range(base + bpf, base + c * cf * bpf))
+                k = min(w.topk, len(earlier))
+                pick = torch.randperm(len(earlier), generator=g)[:k].tolist()
+                rows.append(list(range(base, base + bpf)) + sorted(earlier[i] for i in pick) + own)
+        out.append(rows)
+    return out

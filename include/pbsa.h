@@ -128,6 +128,27 @@ PBSA_API pbsa_status pbsa_attend(const pbsa_geom* g, const void* q, int q_frames
                         const int* kv_slot, const int* kv_cnt, int kv_ld,
                         void* o, float* lse, void* ws, void* stream);
 
+/* a5 -- backward of pbsa_attend under the same lists (English 2.D "Training Strategy": the
+ * model is trained with the same dynamic sparse cache, so the sparse attention needs its
+ * gradients):
+ *   P = exp(scale * q_i . k_j - lse_i) over each row's listed blocks; D_i = dO_i . O_i;
+ *   dV = P^T dO;  dP = dO V^T;  dS = P * (dP - D);  dQ = scale * dS K;  dK = scale * dS^T Q.
+ *  q, o, d_o  [q_frames*frame_h*frame_w][H][d] raster bf16; lse [H][T_q] fp32 from pbsa_attend.
+ *  k_pool, v_pool, kv_slot, kv_cnt, kv_ld as for pbsa_attend (slots of one row distinct).
+ *  dq      out [T_q][H][d] raster bf16.
+ *  dk_pool, dv_pool out [H][pool_slots][64][d] bf16: every slot is written (slots that no
+ *          query block attends get zeros).
+ *  bf16, d = 128, kv_ld <= 512, q_frames*bpf <= 512 query blocks.  Deterministic (no
+ *  floating-point atomics).
+ *  ws: pbsa_bwd_workspace_bytes(g, q_frames, pool_slots, kv_ld) bytes of device memory whose
+ *  first 256 bytes (the error word) are zero before first use. */
+PBSA_API size_t pbsa_bwd_workspace_bytes(const pbsa_geom* g, int q_frames, int pool_slots, int kv_ld);
+PBSA_API pbsa_status pbsa_attend_bwd(const pbsa_geom* g, const void* q, int q_frames,
+                                     const void* k_pool, const void* v_pool, int pool_slots,
+                                     const int* kv_slot, const int* kv_cnt, int kv_ld,
+                                     const void* o, const void* d_o, const float* lse,
+                                     void* dq, void* dk_pool, void* dv_pool, void* ws, void* stream);
+
 /* a4 -- persistent-memory update ("Top-C retention"; English 2.C "Dynamic Update",
  * Chinese 2.2 "粗粒度评分与更新"), per head h:
  *   pool    = valid persistent slots (slot_gid[h][j] >= 0, j < C) + the candidates
