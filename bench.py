@@ -96,6 +96,23 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def profiled_traffic(profile: str, source: str):
+    """DRAM bytes per launch from a committed ncu summary, or None when the kernel source has
+    changed since the counters were taken (the summary records the source's sha256 prefix)."""
+    import hashlib
+    import re
+    try:
+        text = open(os.path.join(ROOT, "profiles", profile)).read()
+        sha = hashlib.sha256(open(os.path.join(ROOT, source), "rb").read()).hexdigest()[:16]
+    except OSError:
+        return None
+    m_sha = re.search(r"kernel_source_sha256:\s*([0-9a-f]+)", text)
+    m_tr = re.search(r"traffic_bytes_per_launch:\s*(\d+)", text)
+    if not m_sha or not m_tr or m_sha.group(1) != sha:
+        return None
+    return int(m_tr.group(1))
+
+
 def workload_config(w):
     return {"workload": w.name, "heads": w.heads, "head_dim": w.head_dim,
             "frame_tokens": f"{w.frame_h}x{w.frame_w}", "block": f"1 frame x {w.tile_h}x{w.tile_w}",
@@ -177,6 +194,68 @@ def algorithmic_bytes(w, ncopy: int):
         "memory_update": reps_q + H * (w.capacity + w.chunk_frames * bpf) * d * 4
         + 2 * H * nq * (w.capacity + w.chunk_frames * bpf) * 4 + ncopy * 2 * (2 * 64 * d * 2 + d * 4),
     }
+
+
+def run_train(P, I, dev, steps: int, peaks):
+    """Trainable-path workload (batch 2 x 9 frames, 12 heads, 3-frame chunks, sinks + top-16
+    + own chunk): forward (pbsa_attend) and backward (pbsa_attend_bwd), timed separately with
+    CUDA events, L2 flushed before each; inputs resident in HBM."""
+    w = I.TRAIN_FWD_BWD
+    frames, batch = w.total_frames, w.batch
+    qf = batch * frames
+    shape = (qf * w.tokens_per_frame, w.heads, w.head_dim)
+    gens = [torch.Generator(device=dev).manual_seed(I.stream_seed(w.seed, 20 + i)) for i in range(4)]
+    q, k, v, do = (torch.randn(shape, generator=g_, device=dev).to(torch.bfloat16) for g_ in gens)
+    lists = I.train_lists(w, I.stream_seed(w.seed, 30))
+    nq = qf * w.blocks_per_frame
+    ld = max(len(l) for row in lists for l in row)
+    kv = torch.zeros((w.heads, nq, ld), dtype=torch.int32)
+    cnt = torch.zeros((w.heads, nq), dtype=torch.int32)
+    for h in range(w.heads):
+        for r in range(nq):
+            kv[h, r, :len(lists[h][r])] = torch.tensor(lists[h][r], dtype=torch.int32)
+            cnt[h, r] = len(lists[h][r])
+    kv, cnt = kv.to(dev), cnt.to(dev)
+    g = P.make_geom(w.heads, w.head_dim, w.frame_h, w.frame_w, w.tile_h, w.tile_w, w.scale, "bf16")
+    slots = nq
+    kp = torch.empty((w.heads, slots, 64, w.head_dim), dtype=torch.bfloat16, device=dev)
+    vp = torch.empty_like(kp)
+    reps = torch.empty((w.heads, slots, w.head_dim), device=dev)
+    ws = torch.zeros(max(P.pbsa_workspace_bytes(g, 64, 64), P.pbsa_bwd_workspace_bytes(g, qf, slots, ld)),
+                     dtype=torch.uint8, device=dev)
+    P.pbsa_blockify(g, k, qf, reps, slots, None, kp, slots, ws)
+    P.pbsa_blockify(g, v, qf, reps, slots, None, vp, slots, ws)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.heads, q.shape[0]), device=dev)
+    dq = torch.empty_like(q)
+    dk, dv = torch.empty_like(kp), torch.empty_like(vp)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    fwd_ms, bwd_ms = [], []
+    for it in range(steps + 2):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        flush.fill_(1)
+        e[0].record()
+        P.pbsa_attend(g, q, qf, kp, vp, slots, kv, cnt, ld, o, lse, ws)
+        e[1].record()
+        flush.fill_(2)
+        e[2].record()
+        P.pbsa_attend_bwd(g, q, qf, kp, vp, slots, kv, cnt, ld, o, do, lse, dq, dk, dv, ws)
+        e[3].record()
+        torch.cuda.synchronize(dev)
+        if it >= 2:
+            fwd_ms.append(e[0].elapsed_time(e[1]))
+            bwd_ms.append(e[2].elapsed_time(e[3]))
+    _check_device(P, ws, "in the training workload")
+    fwd_flops = 4.0 * 64 * 64 * w.head_dim * float(cnt.sum().item())
+    bwd_flops = 2.5 * fwd_flops
+    fm, bm = statistics.mean(fwd_ms), statistics.mean(bwd_ms)
+    return {"workload": w.name, "query_blocks": nq, "heads": w.heads, "steps": steps,
+            "fwd_ms": fm, "bwd_ms": bm, "fwd_flops": fwd_flops, "bwd_flops": bwd_flops,
+            "fwd_tflops": fwd_flops / (fm * 1e-3) / 1e12, "bwd_tflops": bwd_flops / (bm * 1e-3) / 1e12,
+            "bwd_frac_of_bf16_peak": bwd_flops / (bm * 1e-3) / 1e12 / peaks["bf16"],
+            "launches_per_iteration": 6,
+            "note": "bwd FLOPs counted as 2.5x the forward's (5 GEMM-sized contractions vs 2); "
+                    "the deterministic kernels recompute S and dP in both the dQ and the dK/dV passes"}
 
 
 def _check_device(P, ws, when: str):
@@ -302,7 +381,10 @@ def run_pbsa(args, w, rank, world, local_rank):
         "roofline": {"bound": "tensor", "kernel": "pbsa_attend (attend_tc_kernel)", "achieved": att_tflops,
                      "peak": peaks["bf16"], "unit": "TFLOP/s", "frac": att_tflops / peaks["bf16"],
                      "peak_source": f"{peaks['source']} burst bf16 (cuBLAS)",
-                     "frac_of_sustained": att_tflops / peaks["bf16_sustained"], "traffic": None},
+                     "frac_of_sustained": att_tflops / peaks["bf16_sustained"],
+                     "traffic": profiled_traffic("attend_tc_decode_5s.md",
+                                                 "block_sparse_attention_pbsa_b200/csrc/attend_tc.cu"),
+                     "traffic_unit": "bytes per launch (ncu dram read + write)"},
         "step_frac_of_bf16_peak": value / world / peaks["bf16"],
         "kernels": kernels,
         "kv_cache_bytes": {"pbsa_per_layer": cache.kv_bytes,
@@ -312,6 +394,8 @@ def run_pbsa(args, w, rank, world, local_rank):
         "gpu_launches": P.ChunkDecodeStep.LAUNCHES * args.steps,
         "clocks": clk.summary(),
     }
+    if not args.no_train:
+        line["train"] = run_train(P, I, dev, 5, peaks)
     if world == 1 and not args.no_cpu_baseline:
         t, desc, threads = oracle_sample(w, q, k, v, units=24)
         line["cpu_baseline"] = {"value": flops / t / 1e12, "unit": "TFLOP/s", "cores": threads,
@@ -326,6 +410,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["pbsa", "reference"], default="pbsa")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-train", action="store_true", help="skip the forward+backward training workload")
+    ap.add_argument("--train-only", action="store_true", help="only the training workload (for profiling)")
     args = ap.parse_args()
     from block_sparse_attention_pbsa_b200 import inputs as I
     w = I.DECODE_5S
@@ -334,6 +420,12 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, w, rank, world)
+        return
+    if args.train_only:
+        import block_sparse_attention_pbsa_b200 as P
+        dev = torch.device("cuda", local_rank)
+        torch.cuda.set_device(dev)
+        print(json.dumps(run_train(P, I, dev, args.steps, load_peaks())), flush=True)
         return
     if world > 1:
         import datetime
