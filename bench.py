@@ -258,6 +258,20 @@ def run_train(P, I, dev, steps: int, peaks):
                     "the deterministic kernels recompute S and dP in both the dQ and the dK/dV passes"}
 
 
+def rank_workload(w, rank: int):
+    """Weak scaling: every rank decodes its own independent layer (same shapes, its own seed)."""
+    import dataclasses
+    return w if rank == 0 else dataclasses.replace(w, seed=w.seed + 1000 * rank)
+
+
+def max_over_ranks(x: float, device, world: int) -> float:
+    """The slowest rank's value (time-like numbers are reported as the max over ranks)."""
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
 def _check_device(P, ws, when: str):
     """Raise with the workspace's device error word (code, info, kernel id) if one is set."""
     torch.cuda.synchronize()
@@ -273,7 +287,7 @@ def run_pbsa(args, w, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     peaks = load_peaks()
-    wr = w if rank == 0 else __import__("dataclasses").replace(w, seed=w.seed + 1000 * rank)
+    wr = rank_workload(w, rank)
     q, k, v = I.single_step(wr)
     kc = I.tokens(wr, wr.chunk_frames, I.stream_seed(wr.seed, 4))
     vc = I.tokens(wr, wr.chunk_frames, I.stream_seed(wr.seed, 5))
@@ -327,10 +341,7 @@ def run_pbsa(args, w, rank, world, local_rank):
         torch.distributed.barrier()
     per = {g: statistics.mean(v) for g, v in per_runs.items()}
     step_ms = statistics.mean(step_runs)
-    step_t = torch.tensor([step_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(step_t, op=torch.distributed.ReduceOp.MAX)
-    step_ms_max = float(step_t.item())
+    step_ms_max = max_over_ranks(step_ms, dev, world)
     # number of block copies the memory update made (for its algorithmic bytes)
     step.restore(snap)
     graph.replay()
@@ -356,9 +367,7 @@ def run_pbsa(args, w, rank, world, local_rank):
         e1.synchronize()
         if s > 0:
             e2e_ms.append(e0.elapsed_time(e1))
-    e2e_t = torch.tensor([statistics.mean(e2e_ms)], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(e2e_t, op=torch.distributed.ReduceOp.MAX)
+    e2e_ms_max = max_over_ranks(statistics.mean(e2e_ms), dev, world)
 
     if rank != 0:
         return
@@ -389,8 +398,8 @@ def run_pbsa(args, w, rank, world, local_rank):
         "kernels": kernels,
         "kv_cache_bytes": {"pbsa_per_layer": cache.kv_bytes,
                            "dense_21_frames_per_layer": 2 * w.heads * 21 * w.tokens_per_frame * w.head_dim * 2},
-        "e2e": {"value": world * flops / (float(e2e_t.item()) * 1e-3) / 1e12, "unit": "TFLOP/s",
-                "ms_per_step": float(e2e_t.item()), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "e2e": {"value": world * flops / (e2e_ms_max * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "ms_per_step": e2e_ms_max, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": P.ChunkDecodeStep.LAUNCHES * args.steps,
         "clocks": clk.summary(),
     }
