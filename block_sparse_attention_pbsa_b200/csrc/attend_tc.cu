@@ -7,22 +7,26 @@
 //
 // Design (sm_100a):
 //  * One CTA per (head, pair of query blocks): the pair fills the 128 rows of one
-//    M=128 tcgen05 MMA.  The two lists are merged in shared memory; each merged entry
-//    carries a 2-bit mask (which query block of the pair attends it).  Persistent blocks
-//    are shared by both halves, so most MMA rows are useful; rows of a half that does not
-//    attend a block are masked in the softmax (p = 0) and cost no exponentials.
-//  * Each step covers two KV blocks (N = 128 keys).  A producer warp gathers the blocks
-//    with TMA (128-byte swizzle) into a 3-stage K ring and a 2-stage V ring; a block that
-//    does not exist (odd count) is loaded out of bounds, i.e. zero-filled.
-//  * An MMA warp (one thread) issues S = Q K^T into one of two TMEM S buffers.  Two
-//    softmax warpgroups each own one of the step's two blocks and run an independent
-//    online softmax (exp2 domain) over "their" half of the list, one TMEM lane = one
-//    query row per thread.  Each writes its P (bf16) back into TMEM over the S columns it
-//    consumed, and the MMA warp accumulates O_w += P_w V_w with the A operand read from
-//    TMEM, into a per-warpgroup O accumulator (TMEM = S0 | S1 | O0 | O1 = 512 columns).
-//    O_w is rescaled only when its running max grows by more than 2^8; the epilogue
+//    M=128 tcgen05 MMA.  The two lists are merged in shared memory (bitmaps of the pool
+//    slots); each merged entry carries a 2-bit mask (which query block of the pair attends
+//    it).  Persistent blocks are shared by both halves, so most MMA rows are useful; rows of
+//    a half that does not attend a block are masked in the softmax (p = 0).
+//  * Each step covers two KV blocks (N = 128 keys).  Warp 0 gathers the K blocks, warp 2
+//    the V blocks, with TMA (128-byte swizzle) into a 3-stage K ring and a 2-stage V ring;
+//    a block that does not exist (odd count) is loaded out of bounds, i.e. zero-filled.
+//    Q is loaded first, before the lists are read.
+//  * Two softmax warpgroups take alternate steps; each has its own TMEM S/P buffer and O
+//    accumulator (TMEM = S0 | S1 | O0 | O1 = 512 columns) and its own MMA issuer warp
+//    (warps 1 and 3, one thread each), so the two chains S -> softmax -> P -> PV -> next S
+//    run independently.  One TMEM lane = one query row per thread; the online softmax
+//    works in the exp2 domain with packed f32x2 arithmetic, writes P (bf16) back over the
+//    S columns it consumed, and the issuer accumulates O_w += P V with the A operand read
+//    from TMEM, then issues the next S = Q K^T of that warpgroup right behind it.
+//  * The warpgroups take turns on the exponentials (the MUFU pipe is as busy as the tensor
+//    pipe), so one warpgroup's exponentials overlap the other's MMAs.
+//  * O_w is rescaled only when its running max grows by more than 2^8; the epilogue
 //    merges the two streams exactly.
-//  * Register split: the producer/MMA warpgroup runs on 56 registers, the softmax
+//  * Register split: the producer/issuer warpgroup runs on 56 registers, the softmax
 //    warpgroups on 224 (setmaxnreg), so the softmax holds its row in registers.
 //  * Every wait is bounded; on expiry the kernel records PBSA_ERR_TIMEOUT in the
 //    workspace, drains its own copies and MMAs, frees TMEM and returns.
@@ -55,14 +59,17 @@ constexpr uint32_t SM_LA = SM_FLAG + MAXL;            // int[512]
 constexpr uint32_t SM_LB = SM_LA + 4 * 512;           // int[512]
 constexpr uint32_t SM_ONLYB = SM_LB + 4 * 512;        // uint8[512]
 constexpr uint32_t SM_STAT = SM_ONLYB + 512;          // float2[2][128] epilogue (m, l) exchange
-constexpr uint32_t SM_TOTAL = SM_STAT + 2 * 128 * 8;
+constexpr uint32_t SM_BITS = SM_STAT + 2 * 128 * 8;   // uint32[2][BITMAP_SLOTS / 32] list membership
+constexpr int BITMAP_SLOTS = 8192;                    // pools up to this many slots merge in O(n)
+constexpr uint32_t SM_TOTAL = SM_BITS + 2 * BITMAP_SLOTS / 8;
 constexpr uint32_t SMEM_BYTES = SM_TOTAL + 1024;      // + alignment slack
 
 enum { B_QFULL = 0, B_KFULL = 1, B_KEMPTY = B_KFULL + KSTAGES, B_VFULL = B_KEMPTY + KSTAGES,
        B_VEMPTY = B_VFULL + VSTAGES, B_SFULL = B_VEMPTY + VSTAGES,
-       B_PFULL = B_SFULL + 2,      // [warpgroup][step & 1]: a softmax warpgroup may run up to
-                                   // two steps ahead of the MMA warp's wait, so P-full is a ring
-       B_PVDONE = B_PFULL + 4, B_MMADONE = B_PVDONE + 2, NUM_BARS = B_MMADONE + 1 };
+       B_PFULL = B_SFULL + 2,      // [warpgroup], 128 arrivals (one per row)
+       B_MMADONE = B_PFULL + 2,
+       B_XDONE = B_MMADONE + 1,    // [warpgroup], 128 arrivals: its exponentials of a step are done
+       NUM_BARS = B_XDONE + 2 };
 static_assert(NUM_BARS * 8 <= 256, "barrier area");
 
 constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, 0, 0);
@@ -80,6 +87,26 @@ struct Params {
   void* ws;
 };
 
+// ---------------------------------------------------------------- softmax arithmetic
+// Two fp32 lanes per instruction (sm_100 packed f32x2): a = x * c + m.
+__device__ __forceinline__ void ffma2(float x0, float x1, float c, float m, float& a0, float& a1) {
+  asm("{\n\t.reg .b64 x, c, m, a;\n\t"
+      "mov.b64 x, {%2, %3};\n\tmov.b64 c, {%4, %4};\n\tmov.b64 m, {%5, %5};\n\t"
+      "fma.rn.f32x2 a, x, c, m;\n\tmov.b64 {%0, %1}, a;\n\t}"
+      : "=f"(a0), "=f"(a1) : "f"(x0), "f"(x1), "f"(c), "f"(m));
+}
+// (s0, s1) += (y0, y1)
+__device__ __forceinline__ void fadd2(float& s0, float& s1, float y0, float y1) {
+  asm("{\n\t.reg .b64 s, y;\n\t"
+      "mov.b64 s, {%0, %1};\n\tmov.b64 y, {%2, %3};\n\t"
+      "add.rn.f32x2 s, s, y;\n\tmov.b64 {%0, %1}, s;\n\t}"
+      : "+f"(s0), "+f"(s1) : "f"(y0), "f"(y1));
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
 __device__ __forceinline__ void wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                               void* ws, int where) {
   if (*abort_flag) return;
@@ -112,39 +139,79 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   // ---------------------------------------------------------------- setup
   if (tid == 0) {
     for (int i = 0; i < NUM_BARS; ++i) mbar_init(&bars[i], 1);
-    for (int i = 0; i < 4; ++i) mbar_init(&bars[B_PFULL + i], 128);
+    for (int i = 0; i < 2; ++i) mbar_init(&bars[B_PFULL + i], 128);
+    for (int i = 0; i < 2; ++i) mbar_init(&bars[B_XDONE + i], 128);
+    mbar_init(&bars[B_MMADONE], 2);
     *abort_flag = 0;
     fence_barrier_init();
+    // Q (two 64-row blocks, strided raster rows): one 5-D box per 64 columns and block
+    tma_prefetch_desc(&qmap);
+    mbar_arrive_expect_tx(&bars[B_QFULL], 32768);
+    for (int half = 0; half < 2; ++half) {
+      const int r = (half == 1 && hasB) ? rB : rA;
+      const int f = r / prm.bpf, rem = r - f * prm.bpf;
+      const int ty = rem / prm.tpr, tx = rem - ty * prm.tpr;
+      for (int p = 0; p < 2; ++p)
+        tma_load_5d(sm + SM_Q + p * 16384 + half * 8192, &qmap, &bars[B_QFULL], p * 64, h,
+                    tx * prm.tw, ty * prm.th, f);
+    }
   }
   if (warp == 1) {
     tmem_alloc(tmem_holder, 512);
     tmem_relinquish();
   }
-  // merge the two query blocks' lists; mask bit 0 = block A attends, bit 1 = block B
+  // Merge the two query blocks' lists; mask bit 0 = block A attends, bit 1 = block B.  The
+  // counts and the whole list rows are fetched together (one round trip); the Q load was
+  // issued above, as it depends on nothing here.
+  uint32_t* bitsA = reinterpret_cast<uint32_t*>(sm + SM_BITS);
+  uint32_t* bitsB = bitsA + BITMAP_SLOTS / 32;
+  const bool use_bits = prm.pool_slots <= BITMAP_SLOTS;
+  if (use_bits)
+    for (int i = tid; i < 2 * BITMAP_SLOTS / 32; i += NTHREADS) bitsA[i] = 0u;
+  const int* listA = prm.kv_slot + ((size_t)h * prm.nq + rA) * prm.kv_ld;
+  const int* listB = prm.kv_slot + ((size_t)h * prm.nq + (hasB ? rB : rA)) * prm.kv_ld;
   int cA = prm.kv_cnt[(size_t)h * prm.nq + rA];
   int cB = hasB ? prm.kv_cnt[(size_t)h * prm.nq + rB] : 0;
+  for (int i = tid; i < prm.kv_ld; i += NTHREADS) {
+    la[i] = listA[i];
+    lb[i] = listB[i];
+  }
   if (cA < 0 || cA > prm.kv_ld || cB < 0 || cB > prm.kv_ld) {
     if (tid == 0) record_error(prm.ws, PBSA_ERR_DEVICE_INDEX, cA < 0 || cA > prm.kv_ld ? cA : cB, K_ATTEND_TC);
     cA = min(max(cA, 0), prm.kv_ld);
     cB = min(max(cB, 0), prm.kv_ld);
   }
-  const int* listA = prm.kv_slot + ((size_t)h * prm.nq + rA) * prm.kv_ld;
-  const int* listB = prm.kv_slot + ((size_t)h * prm.nq + (hasB ? rB : rA)) * prm.kv_ld;
-  for (int i = tid; i < cA; i += NTHREADS) la[i] = listA[i];
-  for (int i = tid; i < cB; i += NTHREADS) lb[i] = listB[i];
   __syncthreads();
-  for (int i = tid; i < cA; i += NTHREADS) {
-    const int s = la[i];
-    uint8_t f = 1;
-    for (int j = 0; j < cB; ++j) f |= (lb[j] == s) ? 2 : 0;
-    mslot[i] = s;
-    mflag[i] = f;
-  }
-  for (int j = tid; j < cB; j += NTHREADS) {
-    const int s = lb[j];
-    bool in_a = false;
-    for (int i = 0; i < cA; ++i) in_a |= (la[i] == s);
-    onlyb[j] = in_a ? 0 : 1;
+  auto in_range = [&](int s) { return s >= 0 && s < prm.pool_slots; };
+  if (use_bits) {
+    for (int i = tid; i < cA; i += NTHREADS)
+      if (in_range(la[i])) atomicOr(&bitsA[la[i] >> 5], 1u << (la[i] & 31));
+    for (int j = tid; j < cB; j += NTHREADS)
+      if (in_range(lb[j])) atomicOr(&bitsB[lb[j] >> 5], 1u << (lb[j] & 31));
+    __syncthreads();
+    for (int i = tid; i < cA; i += NTHREADS) {
+      const int s = la[i];
+      mslot[i] = s;
+      mflag[i] = (in_range(s) && ((bitsB[s >> 5] >> (s & 31)) & 1u)) ? 3 : 1;
+    }
+    for (int j = tid; j < cB; j += NTHREADS) {
+      const int s = lb[j];
+      onlyb[j] = (in_range(s) && ((bitsA[s >> 5] >> (s & 31)) & 1u)) ? 0 : 1;
+    }
+  } else {
+    for (int i = tid; i < cA; i += NTHREADS) {
+      const int s = la[i];
+      uint8_t f = 1;
+      for (int j = 0; j < cB; ++j) f |= (lb[j] == s) ? 2 : 0;
+      mslot[i] = s;
+      mflag[i] = f;
+    }
+    for (int j = tid; j < cB; j += NTHREADS) {
+      const int s = lb[j];
+      bool in_a = false;
+      for (int i = 0; i < cA; ++i) in_a |= (la[i] == s);
+      onlyb[j] = in_a ? 0 : 1;
+    }
   }
   __syncthreads();
   if (warp == 0) {
@@ -182,104 +249,114 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   // Each role's whole body sits inside the branch that sets its register budget.
   if (warp < 4) {
   setmaxnreg_dec<REG_CTRL>();
-  // ---------------------------------------------------------------- producer warp
-  // K of step i is issued one step ahead of V of step i-1, so K runs ahead of the PV MMAs.
+  // ---------------------------------------------------------------- producer warps
+  // Warp 0 loads Q and the K ring, warp 2 the V ring, so a V stage that is still in use
+  // never holds back the prefetch of K.
+  auto load_pair = [&](const CUtensorMap* map, uint8_t* dst, uint64_t* bar, int i) {
+    for (int b = 0; b < 2; ++b) {
+      const int e = 2 * i + b;
+      const int slot = e < n ? mslot[e] : -1;
+      const int row0 = slot >= 0 ? (h * prm.pool_slots + slot) * 64 : prm.kv_rows;
+      for (int p = 0; p < 2; ++p) tma_load_2d(dst + p * 16384 + b * 8192, map, bar, p * 64, row0);
+    }
+  };
   if (warp == 0) {
     if (lane == 0 && nsteps > 0) {
-      tma_prefetch_desc(&qmap);
       tma_prefetch_desc(&kmap);
-      tma_prefetch_desc(&vmap);
-      mbar_arrive_expect_tx(&bars[B_QFULL], 32768);
-      for (int half = 0; half < 2; ++half) {
-        const int r = (half == 1 && hasB) ? rB : rA;
-        const int f = r / prm.bpf, rem = r - f * prm.bpf;
-        const int ty = rem / prm.tpr, tx = rem - ty * prm.tpr;
-        for (int p = 0; p < 2; ++p)
-          tma_load_5d(sm + SM_Q + p * 16384 + half * 8192, &qmap, &bars[B_QFULL], p * 64, h,
-                      tx * prm.tw, ty * prm.th, f);
-      }
-      int kiss = 0, viss = 0;  // steps whose K / V loads were issued
-      auto load_pair = [&](const CUtensorMap* map, uint8_t* dst, uint64_t* bar, int i) {
-        for (int b = 0; b < 2; ++b) {
-          const int e = 2 * i + b;
-          const int slot = e < n ? mslot[e] : -1;
-          const int row0 = slot >= 0 ? (h * prm.pool_slots + slot) * 64 : prm.kv_rows;
-          for (int p = 0; p < 2; ++p) tma_load_2d(dst + p * 16384 + b * 8192, map, bar, p * 64, row0);
-        }
-      };
-      for (int i = 0; i <= nsteps; ++i) {
-        if (i < nsteps) {
-          const int s = i % KSTAGES;
-          wait_or_abort(&bars[B_KEMPTY + s], ((i / KSTAGES) & 1) ^ 1, abort_flag, prm.ws, 1);
-          if (*abort_flag) break;
-          mbar_arrive_expect_tx(&bars[B_KFULL + s], 32768);
-          load_pair(&kmap, sm + SM_K + s * 32768, &bars[B_KFULL + s], i);
-          kiss = i + 1;
-        }
-        if (i >= 1) {
-          const int j = i - 1, s = j % VSTAGES;
-          wait_or_abort(&bars[B_VEMPTY + s], ((j / VSTAGES) & 1) ^ 1, abort_flag, prm.ws, 2);
-          if (*abort_flag) break;
-          mbar_arrive_expect_tx(&bars[B_VFULL + s], 32768);
-          load_pair(&vmap, sm + SM_V + s * 32768, &bars[B_VFULL + s], j);
-          viss = j + 1;
-        }
+      int kiss = 0;  // steps whose K loads were issued
+      for (int i = 0; i < nsteps; ++i) {
+        const int s = i % KSTAGES;
+        wait_or_abort(&bars[B_KEMPTY + s], ((i / KSTAGES) & 1) ^ 1, abort_flag, prm.ws, 1);
+        if (*abort_flag) break;
+        mbar_arrive_expect_tx(&bars[B_KFULL + s], 32768);
+        load_pair(&kmap, sm + SM_K + s * 32768, &bars[B_KFULL + s], i);
+        kiss = i + 1;
       }
       if (*abort_flag) {
         // drain: wait (bounded) for the last copy issued into every stage before leaving
-        mbar_wait(&bars[B_QFULL], 0, kWaitLimitNs);
         for (int i = (kiss > KSTAGES ? kiss - KSTAGES : 0); i < kiss; ++i)
           mbar_wait(&bars[B_KFULL + i % KSTAGES], (i / KSTAGES) & 1, kWaitLimitNs);
-        for (int i = (viss > VSTAGES ? viss - VSTAGES : 0); i < viss; ++i)
-          mbar_wait(&bars[B_VFULL + i % VSTAGES], (i / VSTAGES) & 1, kWaitLimitNs);
+      }
+    }
+    // Q was loaded at set-up; it must have landed before the CTA may exit, whether or not an
+    // MMA consumed it (no steps, or an abort)
+    if (lane == 0) mbar_wait(&bars[B_QFULL], 0, kWaitLimitNs);
+    __syncwarp();
+  }
+  if (warp == 2) {
+    if (lane == 0 && nsteps > 0) {
+      tma_prefetch_desc(&vmap);
+      int viss = 0;  // steps whose V loads were issued
+      for (int j = 0; j < nsteps; ++j) {
+        const int s = j % VSTAGES;
+        wait_or_abort(&bars[B_VEMPTY + s], ((j / VSTAGES) & 1) ^ 1, abort_flag, prm.ws, 2);
+        if (*abort_flag) break;
+        mbar_arrive_expect_tx(&bars[B_VFULL + s], 32768);
+        load_pair(&vmap, sm + SM_V + s * 32768, &bars[B_VFULL + s], j);
+        viss = j + 1;
+      }
+      if (*abort_flag) {
+        for (int j = (viss > VSTAGES ? viss - VSTAGES : 0); j < viss; ++j)
+          mbar_wait(&bars[B_VFULL + j % VSTAGES], (j / VSTAGES) & 1, kWaitLimitNs);
       }
     }
     __syncwarp();
   }
 
-  // ---------------------------------------------------------------- MMA warp
-  // S_i -> TMEM columns [128 (i%2), +128); P_w(i) is written by softmax warpgroup w over the
-  // first 32 columns of its block's S half; O_w accumulates in columns [256 + 128 w, +128).
-  if (warp == 1) {
+  // ---------------------------------------------------------------- MMA issuers
+  // Warp 1 issues the tensor-core work of softmax warpgroup 0 (steps 0, 2, 4, ...), warp 3
+  // that of warpgroup 1 (steps 1, 3, ...), each from one thread, so the two chains
+  // S -> softmax -> P -> PV -> next S never wait on each other's issue.  Warpgroup w owns
+  // TMEM columns [128 w, +128) for S and P and [256 + 128 w, +128) for its O accumulator.
+  // QK(i) into S_w is issued after PV(i-2), which read P(i-2) from the same columns, by
+  // the same thread, so the tensor pipe orders them; and the commit that signals S(i)
+  // also covers PV(i-2), so O_w is never rescaled under a running MMA.
+  if (warp == 1 || warp == 3) {
+    const int wg = warp >> 1;
     if (lane == 0 && nsteps > 0) {
-      const uint32_t q_base = smem_u32(sm + SM_Q), k_base = smem_u32(sm + SM_K);
-      const uint32_t v_base = smem_u32(sm + SM_V);
-      const uint32_t tO = tmem + 256;
-      auto issue_pv = [&](int j) {
-        const int sv = j % VSTAGES;
-        wait_or_abort(&bars[B_VFULL + sv], (j / VSTAGES) & 1, abort_flag, prm.ws, 4);
-        for (int w = 0; w < 2; ++w) {
-          wait_or_abort(&bars[B_PFULL + 2 * w + (j & 1)], (j >> 1) & 1, abort_flag, prm.ws, 3);
-          if (*abort_flag) return;
-          tc_fence_after();
-          const uint32_t a_tmem = tmem + (j & 1) * 128 + w * 64;
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t b = sw128_desc(v_base + sv * 32768 + w * 8192 + kk * 2048, 16384, 1024);
-            mma_bf16_ts(tO + w * 128, a_tmem + kk * 8, b, IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
-          }
-          mma_commit(&bars[B_PVDONE + w]);
-        }
-        mma_commit(&bars[B_VEMPTY + sv]);
-      };
-      wait_or_abort(&bars[B_QFULL], 0, abort_flag, prm.ws, 5);
-      for (int i = 0; i < nsteps && !*abort_flag; ++i) {
+      const uint32_t tS = tmem + wg * 128, tO = tmem + 256 + wg * 128;
+      // descriptors of the first 16-element K slice of each operand; a slice further on is
+      // the same descriptor plus its byte offset / 16 (the start-address field)
+      const uint64_t dq = sw128_desc(smem_u32(sm + SM_Q), 16, 1024);
+      const uint64_t dk = sw128_desc(smem_u32(sm + SM_K), 16, 1024);
+      const uint64_t dv = sw128_desc(smem_u32(sm + SM_V), 16384, 1024);
+      auto issue_qk = [&](int i) {   // S_w = Q K_i^T, then free the K stage
         const int sk = i % KSTAGES;
-        wait_or_abort(&bars[B_KFULL + sk], (i / KSTAGES) & 1, abort_flag, prm.ws, 6);
-        if (*abort_flag) break;
-        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t a = sw128_desc(q_base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-          const uint64_t b = sw128_desc(k_base + sk * 32768 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-          mma_bf16_ss(tmem + (i & 1) * 128, a, b, IDESC_QK, kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+          mma_bf16_ss(tS, dq + off, dk + ((sk * 32768) >> 4) + off, IDESC_QK, kk > 0 ? 1u : 0u);
         }
-        mma_commit(&bars[B_SFULL + (i & 1)]);
+        mma_commit(&bars[B_SFULL + wg]);
         mma_commit(&bars[B_KEMPTY + sk]);
-        if (i >= 1) issue_pv(i - 1);
+      };
+      wait_or_abort(&bars[B_QFULL], 0, abort_flag, prm.ws, 5);
+      if (wg < nsteps) {
+        wait_or_abort(&bars[B_KFULL + wg % KSTAGES], (wg / KSTAGES) & 1, abort_flag, prm.ws, 6);
+        if (!*abort_flag) {
+          tc_fence_after();
+          issue_qk(wg);
+        }
       }
-      if (!*abort_flag) issue_pv(nsteps - 1);
-      // every MMA this thread issued has completed once this barrier flips
+      // Steady state: everything but P(i) is awaited first, so PV(i) and QK(i+2) go to the
+      // tensor pipe back to back once the warpgroup hands over P(i).
+      for (int i = wg; i < nsteps && !*abort_flag; i += 2) {
+        const int sv = i % VSTAGES;
+        const bool more = i + 2 < nsteps;
+        wait_or_abort(&bars[B_VFULL + sv], (i / VSTAGES) & 1, abort_flag, prm.ws, 4);
+        if (more) wait_or_abort(&bars[B_KFULL + (i + 2) % KSTAGES], ((i + 2) / KSTAGES) & 1, abort_flag, prm.ws, 6);
+        wait_or_abort(&bars[B_PFULL + wg], (i >> 1) & 1, abort_flag, prm.ws, 3);
+        if (*abort_flag) break;
+        tc_fence_after();
+        // O_w += P_i V_i: P_i (128 rows x 128 keys, bf16 pairs) sits over S_w in TMEM
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ts(tO, tS + kk * 8, dv + ((sv * 32768 + kk * 2048) >> 4), IDESC_PV,
+                      (i > wg || kk > 0) ? 1u : 0u);
+        mma_commit(&bars[B_VEMPTY + sv]);
+        if (more) issue_qk(i + 2);
+      }
+      // every MMA of both issuers has completed once this barrier (count 2) flips
       mma_commit(&bars[B_MMADONE]);
       mbar_wait(&bars[B_MMADONE], 0, kWaitLimitNs);
     }
@@ -290,71 +367,85 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   setmaxnreg_inc<REG_SOFTMAX>();
   // ---------------------------------------------------------------- softmax warpgroups
   {
-    const int wg = (warp - 4) >> 2;          // 0: first block of each step, 1: second
+    const int wg = (warp - 4) >> 2;          // this warpgroup takes the steps i = wg (mod 2)
     const int wq = warp & 3;                 // TMEM lane quadrant this warp may access
     const int row = wq * 32 + lane;          // query row of the 128-row tile
     const int half = row >> 6;
     const bool row_valid = half == 0 || hasB;
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_off + wg * 128;          // S_i / P_i of this warpgroup's steps
     const uint32_t tO = tmem + lane_off + 256 + wg * 128;
     const float c = prm.scale_log2;
     float m = -INFINITY, l = 0.f;
-    for (int i = 0; i < nsteps; ++i) {
-      const int e = 2 * i + wg;
-      const bool v = row_valid && e < n && ((mflag[e] >> half) & 1);
-      const uint32_t tS = tmem + lane_off + (i & 1) * 128 + wg * 64;
-      wait_or_abort(&bars[B_SFULL + (i & 1)], (i >> 1) & 1, abort_flag, prm.ws, 7);
+    for (int i = wg; i < nsteps; i += 2) {
+      const bool va = row_valid && ((mflag[2 * i] >> half) & 1);
+      const bool vb = row_valid && 2 * i + 1 < n && ((mflag[2 * i + 1] >> half) & 1);
+      wait_or_abort(&bars[B_SFULL + wg], (i >> 1) & 1, abort_flag, prm.ws, 7);
       if (__any_sync(0xffffffffu, *abort_flag != 0)) break;  // warp-uniform exit
       tc_fence_after();
-      uint32_t x[2][32];
-      if (__any_sync(0xffffffffu, v)) {   // tcgen05.ld is warp-collective
-        tmem_ld32(tS, x[0]);
-        tmem_ld32(tS + 32, x[1]);
-        tmem_wait_ld();
-      }
-      float mb = -INFINITY;
-      if (v) {
-        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      uint32_t x[4][32];
+      // tcgen05.ld is warp-collective.  Every S column is finite (a block that does not exist
+      // was loaded as zeros), so all four are read and masking is arithmetic.  The second
+      // half is in flight while the first half's maximum is taken.
+      tmem_ld32(tS + 0, x[0]);
+      tmem_ld32(tS + 32, x[1]);
+      tmem_wait_ld();
+      tmem_ld32(tS + 64, x[2]);
+      tmem_ld32(tS + 96, x[3]);
+      float mx[2][2];
+#pragma unroll
+      for (int bb = 0; bb < 2; ++bb) {
+        if (bb == 1) tmem_wait_ld();
+        mx[bb][0] = mx[bb][1] = -INFINITY;
 #pragma unroll
         for (int q = 0; q < 2; ++q)
 #pragma unroll
-          for (int e2 = 0; e2 < 32; ++e2) mx[e2 & 3] = fmaxf(mx[e2 & 3], __uint_as_float(x[q][e2]));
-        mb = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * c;
+          for (int e2 = 0; e2 < 16; ++e2)
+            mx[bb][e2 & 1] = fmax3(mx[bb][e2 & 1], __uint_as_float(x[2 * bb + q][2 * e2]),
+                                   __uint_as_float(x[2 * bb + q][2 * e2 + 1]));
       }
+      const float mba = va ? fmaxf(mx[0][0], mx[0][1]) : -INFINITY;
+      const float mbb = vb ? fmaxf(mx[1][0], mx[1][1]) : -INFINITY;
+      const float mb = fmaxf(mba, mbb) * c;
       float alpha = 1.f;
       bool rescale_o = false;
       if (mb > m + 8.0f) {  // also true on the first valid block (m = -inf)
-        rescale_o = (m != -INFINITY) && i > 0;
+        rescale_o = (m != -INFINITY) && i > wg;
         alpha = ex2_approx(m - mb);
         l *= alpha;
         m = mb;
       }
-      // p = 2^(s*c - m) packed to bf16 pairs; a masked block gives 0
-      uint32_t pk[32];
+      // The two warpgroups take turns on the exponentials (the MUFU pipe is the scarce unit):
+      // step i waits until the other warpgroup has finished those of step i-1, so one
+      // warpgroup's exponentials overlap the other's MMAs instead of competing with them.
+      if (i >= 1) wait_or_abort(&bars[B_XDONE + (wg ^ 1)], ((i - 1) >> 1) & 1, abort_flag, prm.ws, 10);
+      // p = 2^(s*c - m) as bf16 pairs over the consumed S columns (32 keys per store).  A
+      // masked block uses the factor 0 and the offset -inf, so it gives exact zeros without a
+      // branch (x is finite).
       float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
+      for (int q = 0; q < 4; ++q) {
+        const bool v = q < 2 ? va : vb;
+        const float cs = v ? c : 0.f, ms = v ? -m : -INFINITY;
+        uint32_t pk[16];
 #pragma unroll
         for (int e2 = 0; e2 < 16; ++e2) {
-          float p0 = 0.f, p1 = 0.f;
-          if (v) {
-            p0 = ex2_approx(fmaf(__uint_as_float(x[q][2 * e2]), c, -m));
-            p1 = ex2_approx(fmaf(__uint_as_float(x[q][2 * e2 + 1]), c, -m));
-          }
-          ls[e2 & 3] += p0 + p1;
-          pk[q * 16 + e2] = pack_bf16(p0, p1);
+          float a0, a1, p0, p1;
+          ffma2(__uint_as_float(x[q][2 * e2]), __uint_as_float(x[q][2 * e2 + 1]), cs, ms, a0, a1);
+          p0 = ex2_approx(a0);
+          p1 = ex2_approx(a1);
+          if (e2 & 1) fadd2(ls[2], ls[3], p0, p1);
+          else fadd2(ls[0], ls[1], p0, p1);
+          pk[e2] = pack_bf16(p0, p1);
         }
+        tmem_st16(tS + q * 16, pk);
       }
       l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-      // P over the S columns just read (the previous user of this buffer, PV(i-2), finished
-      // before S_i was produced)
-      tmem_st32(tS, pk);
-      // O_w may only be rescaled once PV_w(i-1) has completed; tcgen05.ld/st are
-      // warp-collective, so the warp rescales if any of its rows must
+      if (i + 1 < nsteps) mbar_arrive(&bars[B_XDONE + wg]);
+      // PV(i-2), the last MMA into O_w, completed before S(i) was signalled.  tcgen05.ld/st
+      // are warp-collective, so the warp rescales if any of its rows must.
       if (__any_sync(0xffffffffu, rescale_o)) {
-        wait_or_abort(&bars[B_PVDONE + wg], (i - 1) & 1, abort_flag, prm.ws, 8);
         if (!rescale_o) alpha = 1.f;
-        tc_fence_after();
 #pragma unroll 1
         for (int q = 0; q < 4; ++q) {
           uint32_t ov[32];
@@ -367,7 +458,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bars[B_PFULL + 2 * wg + (i & 1)]);
+      mbar_arrive(&bars[B_PFULL + wg]);
     }
     // epilogue: combine the two streams, O = (O_0 2^(m0-M) + O_1 2^(m1-M)) / L.  The
     // all-MMAs-done barrier has a single phase, so this wait cannot alias.
@@ -393,14 +484,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
         uint32_t oa[32], ob[32];
-        if (nsteps > 0) {
-          tmem_ld32(tmem + lane_off + 256 + wg * 64 + q * 32, oa);
-          tmem_ld32(tmem + lane_off + 384 + wg * 64 + q * 32, ob);
-          tmem_wait_ld();
-        } else {
 #pragma unroll
-          for (int e2 = 0; e2 < 32; ++e2) oa[e2] = ob[e2] = 0u;
-        }
+        for (int e2 = 0; e2 < 32; ++e2) oa[e2] = ob[e2] = 0u;
+        if (nsteps > 0) tmem_ld32(tmem + lane_off + 256 + wg * 64 + q * 32, oa);
+        if (nsteps > 1) tmem_ld32(tmem + lane_off + 384 + wg * 64 + q * 32, ob);   // O_1 is written from step 1 on
+        tmem_wait_ld();
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
           uint32_t wv[4];
