@@ -187,8 +187,10 @@ def algorithmic_bytes(w, ncopy: int):
     reps_q = H * nq * d * 4
     nwin = w.window_frames * bpf
     return {
-        "blockify_q": tok + reps_q,
-        "score_select": reps_q + H * nwin * d * 4 + H * nq * (w.capacity + w.topk) * 4 + H * w.capacity * 4,
+        # fused blockify(Q) + score + top-k: Q read once, q reps written, window reps read,
+        # lists written, persistent prefix read
+        "blockify_score_select": tok + reps_q + H * nwin * d * 4 + H * nq * (w.capacity + w.topk) * 4
+        + H * w.capacity * 4,
         "commit_blockify_kv": 2 * (tok + tok) + 2 * reps_q,
         # scores/softmax: q reps + pool reps + p matrix (write, read); copies: K+V+reps per promotion
         "memory_update": reps_q + H * (w.capacity + w.chunk_frames * bpf) * d * 4
@@ -324,7 +326,11 @@ def run_pbsa(args, w, rank, world, local_rank):
     _check_device(P, cache.ws, "during warm-up")
     flops = step.flops()
 
-    groups = ["blockify_q", "score_select", "attend", "commit_blockify_kv", "memory_update"]
+    # kernel groups by the in-graph marks they lie between (marks 1 and 2 are adjacent: the
+    # fused blockify + select is one kernel)
+    spans = {"blockify_score_select": (0, 2), "attend": (2, 3), "commit_blockify_kv": (3, 4),
+             "memory_update": (4, 5)}
+    groups = list(spans)
     per_runs = {g: [] for g in groups}
     step_runs = []
     if world > 1:
@@ -334,8 +340,8 @@ def run_pbsa(args, w, rank, world, local_rank):
         for s in range(args.steps):
             one()
             torch.cuda.synchronize(dev)
-            for i, g in enumerate(groups):
-                per_runs[g].append(marks[i].elapsed_time(marks[i + 1]))
+            for g, (a, b) in spans.items():
+                per_runs[g].append(marks[a].elapsed_time(marks[b]))
             step_runs.append(marks[0].elapsed_time(marks[5]))
     if world > 1:
         torch.distributed.barrier()
@@ -400,7 +406,7 @@ def run_pbsa(args, w, rank, world, local_rank):
                            "dense_21_frames_per_layer": 2 * w.heads * 21 * w.tokens_per_frame * w.head_dim * 2},
         "e2e": {"value": world * flops / (e2e_ms_max * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "ms_per_step": e2e_ms_max, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": P.ChunkDecodeStep.LAUNCHES * args.steps,
+        "gpu_launches": step.LAUNCHES * args.steps,
         "clocks": clk.summary(),
     }
     if not args.no_train:

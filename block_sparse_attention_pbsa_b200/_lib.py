@@ -54,6 +54,8 @@ _SIGS = {
     "pbsa_blockify": (_I, [ctypes.POINTER(Geom), _P, _I, _P, _I, _P, _P, _I, _P, _P]),
     "pbsa_score_select": (_I, [ctypes.POINTER(Geom), _P, _I, _P, _I, _P, _P, _I, _I, _P, _P, _I,
                                _P, _P, _I, _P, _P, _P]),
+    "pbsa_blockify_score_select": (_I, [ctypes.POINTER(Geom), _P, _I, _P, _P, _I, _P, _P, _I, _I, _P,
+                                        _P, _I, _P, _P, _I, _P, _P, _P]),
     "pbsa_attend": (_I, [ctypes.POINTER(Geom), _P, _I, _P, _P, _I, _P, _P, _I, _P, _P, _P, _P]),
     "pbsa_memory_update": (_I, [ctypes.POINTER(Geom), _P, _I, _P, _P, _P, _I, _P, _P, _I, _I, _P,
                                 _P, _I, ctypes.c_float, _P, _P, _P, _P]),
@@ -132,6 +134,18 @@ def pbsa_score_select(g: Geom, q_reps, nq, k_reps, pool_slots, cand_slot, cand_g
                       out_score=None, ws=None, stream=None):
     _check("pbsa_score_select", load().pbsa_score_select(
         ctypes.byref(g), _ptr(q_reps, torch.float32, "q_reps"), nq,
+        _ptr(k_reps, torch.float32, "k_reps"), pool_slots, _ptr(cand_slot, torch.int32, "cand_slot"),
+        _ptr(cand_gid, torch.int32, "cand_gid"), ncand, k, _ptr(prefix_slot, torch.int32, "prefix_slot"),
+        _ptr(prefix_cnt, torch.int32, "prefix_cnt"), prefix_ld, _ptr(out_slot, torch.int32, "out_slot"),
+        _ptr(out_cnt, torch.int32, "out_cnt"), out_ld, _ptr(out_score, torch.float32, "out_score"),
+        _ptr(ws, None, "ws"), _stream(stream)))
+
+
+def pbsa_blockify_score_select(g: Geom, q, q_frames, q_reps, k_reps, pool_slots, cand_slot, cand_gid,
+                               ncand, k, prefix_slot, prefix_cnt, prefix_ld, out_slot, out_cnt, out_ld,
+                               out_score=None, ws=None, stream=None):
+    _check("pbsa_blockify_score_select", load().pbsa_blockify_score_select(
+        ctypes.byref(g), _ptr(q, _tok_dtype(g), "q"), q_frames, _ptr(q_reps, torch.float32, "q_reps"),
         _ptr(k_reps, torch.float32, "k_reps"), pool_slots, _ptr(cand_slot, torch.int32, "cand_slot"),
         _ptr(cand_gid, torch.int32, "cand_gid"), ncand, k, _ptr(prefix_slot, torch.int32, "prefix_slot"),
         _ptr(prefix_cnt, torch.int32, "prefix_cnt"), prefix_ld, _ptr(out_slot, torch.int32, "out_slot"),

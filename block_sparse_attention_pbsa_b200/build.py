@@ -20,7 +20,7 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libpbsa.so")
 
-SOURCES = ["api.cu", "blockify.cu", "score_select.cu", "attend_f32.cu", "attend_tc.cu",
+SOURCES = ["api.cu", "blockify.cu", "score_select.cu", "blockify_select.cu", "attend_f32.cu", "attend_tc.cu",
            "memory_update.cu", "noalloc.cu", "attend_bwd.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",

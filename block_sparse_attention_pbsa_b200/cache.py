@@ -156,6 +156,21 @@ class PBSALayerCache:
                                 self.kv_ld_own, ws=self.ws, stream=stream)
         return self.kv_slot, self.kv_cnt, self.kv_ld_own
 
+    def query_select(self, q: torch.Tensor, stream=None):
+        """a1 + a2 in one launch: q_reps of the chunk and, per query block, persistent slots +
+        top-k local slots -> (q_reps, kv_slot, kv_cnt, kv_ld)."""
+        c = self.cfg
+        nf = self.frames_of(q)
+        nq = nf * c.bpf
+        self.q_reps = self._q_reps_buf[:c.heads * nq * c.head_dim].view(c.heads, nq, c.head_dim)
+        self.kv_slot = self._kv_slot_buf[:c.heads * nq * self.kv_ld_own].view(c.heads, nq, self.kv_ld_own)
+        self.kv_cnt = self._kv_cnt_buf[:c.heads * nq].view(c.heads, nq)
+        cs, cg, n = self._cand
+        L.pbsa_blockify_score_select(self.geom, q, nf, self.q_reps, self.k_reps, self.pool_slots, cs, cg, n,
+                                     c.topk if n else 0, self.p_list, self.p_cnt, c.capacity, self.kv_slot,
+                                     self.kv_cnt, self.kv_ld_own, ws=self.ws, stream=stream)
+        return self.q_reps, self.kv_slot, self.kv_cnt, self.kv_ld_own
+
     def attend(self, q, kv_slot, kv_cnt, kv_ld, o=None, lse=None, stream=None):
         """a3: fine attention over the listed slots."""
         if o is None:
@@ -172,19 +187,20 @@ class PBSALayerCache:
         """
         if self._cand is None:
             self._refresh_window()
+        if self.hist > 0:
+            _, kv_slot, kv_cnt, kv_ld = self.query_select(q, stream)
+            return self.attend(q, kv_slot, kv_cnt, kv_ld, o, lse, stream)
+        # empty history: the chunk attends its own blocks
+        if k is None or v is None:
+            raise ValueError("the first chunk attends its own blocks: pass its k and v")
         q_reps = self.query_reps(q, stream)
-        if self.hist == 0:
-            if k is None or v is None:
-                raise ValueError("the first chunk attends its own blocks: pass its k and v")
-            self._write_chunk(k, v, stream)
-            nq = q_reps.shape[1]
-            own = self._ints([[self.ring_slot(b // self.cfg.bpf, b % self.cfg.bpf) for b in range(nq)]] * nq)
-            kv_slot = torch.zeros((self.cfg.heads, nq, nq), dtype=torch.int32, device=self.device)
-            kv_slot[:] = own.view(nq, nq)
-            kv_cnt = torch.full((self.cfg.heads, nq), nq, dtype=torch.int32, device=self.device)
-            return self.attend(q, kv_slot, kv_cnt, nq, o, lse, stream)
-        kv_slot, kv_cnt, kv_ld = self.select(q_reps, stream)
-        return self.attend(q, kv_slot, kv_cnt, kv_ld, o, lse, stream)
+        self._write_chunk(k, v, stream)
+        nq = q_reps.shape[1]
+        own = self._ints([[self.ring_slot(b // self.cfg.bpf, b % self.cfg.bpf) for b in range(nq)]] * nq)
+        kv_slot = torch.zeros((self.cfg.heads, nq, nq), dtype=torch.int32, device=self.device)
+        kv_slot[:] = own.view(nq, nq)
+        kv_cnt = torch.full((self.cfg.heads, nq), nq, dtype=torch.int32, device=self.device)
+        return self.attend(q, kv_slot, kv_cnt, nq, o, lse, stream)
 
     def _write_chunk(self, k, v, stream=None):
         n = self.frames_of(k)
@@ -285,11 +301,13 @@ class ChunkDecodeStep:
     step can be replayed on a restored state (see ``snapshot``/``restore``).
     """
 
-    LAUNCHES = 8   # kernels per run(): 1 + 1 + 1 + 2 + 3
-
-    def __init__(self, cache: PBSALayerCache, q_frames: int | None = None):
+    def __init__(self, cache: PBSALayerCache, q_frames: int | None = None, fused_select: bool = True):
         c = cache.cfg
         self.cache = cache
+        self.fused_select = fused_select
+        # kernels per run(): [blockify(Q) + select] (1 fused or 2) + attend + blockify K, V (2)
+        # + memory update (3)
+        self.LAUNCHES = (1 if fused_select else 2) + 1 + 2 + 3
         self.q_frames = q_frames or c.chunk_frames
         if cache._cand is None:
             cache._refresh_window()
@@ -330,13 +348,19 @@ class ChunkDecodeStep:
             mk = lambda i: marks[i].record(ev_stream)  # noqa: E731
         else:
             mk = lambda i: None  # noqa: E731
-        mk(0)
-        L.pbsa_blockify(g, q, self.q_frames, self.q_reps, self.nq, ws=ws, stream=stream)
-        mk(1)
         cs, cg, n = ca._cand
-        L.pbsa_score_select(g, self.q_reps, self.nq, ca.k_reps, ps, cs, cg, n, c.topk if n else 0,
-                            ca.p_list, ca.p_cnt, c.capacity, self.kv_slot, self.kv_cnt, ca.kv_ld,
-                            ws=ws, stream=stream)
+        mk(0)
+        if self.fused_select:
+            L.pbsa_blockify_score_select(g, q, self.q_frames, self.q_reps, ca.k_reps, ps, cs, cg, n,
+                                         c.topk if n else 0, ca.p_list, ca.p_cnt, c.capacity, self.kv_slot,
+                                         self.kv_cnt, ca.kv_ld, ws=ws, stream=stream)
+            mk(1)
+        else:
+            L.pbsa_blockify(g, q, self.q_frames, self.q_reps, self.nq, ws=ws, stream=stream)
+            mk(1)
+            L.pbsa_score_select(g, self.q_reps, self.nq, ca.k_reps, ps, cs, cg, n, c.topk if n else 0,
+                                ca.p_list, ca.p_cnt, c.capacity, self.kv_slot, self.kv_cnt, ca.kv_ld,
+                                ws=ws, stream=stream)
         mk(2)
         L.pbsa_attend(g, q, self.q_frames, ca.k_pool, ca.v_pool, ps, self.kv_slot, self.kv_cnt, ca.kv_ld,
                       o, lse, ws=ws, stream=stream)

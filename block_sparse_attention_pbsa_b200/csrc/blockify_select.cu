@@ -1,0 +1,260 @@
+// a1 + a2 fused -- blockify of the query chunk, coarse scores and top-k in one pass.
+//
+// Sparse Forcing (gist.science, English 2.C "Local Sparsity" and 2.E "PBSA Kernel"; Chinese
+// 2.2 "块化压缩"): each query block is summarised by the mean of its 64 tokens and routed
+// to the top-k local blocks by the score scale * <qbar, kbar>.  Blockify and selection are
+// the same two steps as pbsa_blockify + pbsa_score_select; here one CTA does both for one
+// (query block, head), so Q is read from HBM once and qbar never makes a round trip.
+//
+// One CTA of 256 threads per (query block, head):
+//  1. every thread issues its 16-byte loads of the block's tokens (same row/column split
+//     and summation order as the blockify kernel, so qbar is bit-identical to it) together
+//     with the candidate list;
+//  2. qbar is reduced in shared memory in a fixed order and written to q_reps;
+//  3. warp w scores candidates w, w+8, ...: each lane holds d/32 elements of qbar and of the
+//     candidate's kbar row (coalesced row loads, several candidates in flight), and a
+//     butterfly shuffle sums the lane partials (fixed order: deterministic);
+//  4. ranks on (score desc, gid asc, position asc): lists of up to 256 candidates are sorted
+//     by a bitonic network in shared memory (one element per thread), longer ones ranked by
+//     counting; the first k are written behind the copied prefix.
+#include <math.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace pbsa {
+namespace {
+
+constexpr int BS_THREADS = 256;
+constexpr int BS_BATCH = 9;   // candidates per warp in flight (144 candidates: two rounds)
+constexpr int SORT_N = 256;   // candidate lists up to this long are ranked by a bitonic sort
+
+template <typename T>
+__device__ __forceinline__ void add_chunk16(float* acc, const uint4& v);
+template <>
+__device__ __forceinline__ void add_chunk16<float>(float* acc, const uint4& v) {
+  acc[0] += __uint_as_float(v.x);
+  acc[1] += __uint_as_float(v.y);
+  acc[2] += __uint_as_float(v.z);
+  acc[3] += __uint_as_float(v.w);
+}
+template <>
+__device__ __forceinline__ void add_chunk16<__nv_bfloat16>(float* acc, const uint4& v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    acc[2 * i] += __uint_as_float(w[i] << 16);
+    acc[2 * i + 1] += __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+// d/32 consecutive fp32 values of a row, as one vector load
+template <int N> struct Vec;
+template <> struct Vec<4> { using type = float4; };
+template <> struct Vec<2> { using type = float2; };
+template <> struct Vec<1> { using type = float; };
+__device__ __forceinline__ void vec_to(const float4& v, float* o) { o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w; }
+__device__ __forceinline__ void vec_to(const float2& v, float* o) { o[0] = v.x; o[1] = v.y; }
+__device__ __forceinline__ void vec_to(const float& v, float* o) { o[0] = v; }
+
+template <typename T, int D>
+__global__ void __launch_bounds__(BS_THREADS) blockify_select_kernel(
+    const T* __restrict__ x, Geo g, int nq, float* __restrict__ q_reps,
+    const float* __restrict__ k_reps, int pool_slots, const int* __restrict__ cand_slot,
+    const int* __restrict__ cand_gid, int ncand, int k, const int* __restrict__ prefix_slot,
+    const int* __restrict__ prefix_cnt, int prefix_ld, int* __restrict__ out_slot,
+    int* __restrict__ out_cnt, int out_ld, float* __restrict__ out_score, void* ws) {
+  constexpr int VEC = 16 / sizeof(T);   // token elements per 16-byte chunk
+  constexpr int CPR = D / VEC;          // chunks per token row
+  constexpr int RPP = BS_THREADS / CPR; // rows per pass
+  constexpr int PASSES = BT / RPP;
+  constexpr int PL = D / 32;            // qbar / kbar elements per lane
+  using V = typename Vec<PL>::type;
+  __shared__ float part[RPP][D];
+  __shared__ float qb[D];
+  extern __shared__ uint64_t dyn[];
+  uint64_t* key = dyn;                                          // [ncand]
+  float* sc = reinterpret_cast<float*>(key + ncand);            // [ncand]
+  int* gid = reinterpret_cast<int*>(sc + ncand);                // [ncand]
+  int* slot = gid + ncand;                                      // [ncand]
+
+  const int r = blockIdx.x, h = blockIdx.y;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  // ---- 1. loads: the block's tokens and the candidate list
+  const int f = r / g.bpf, rem = r - f * g.bpf;
+  const int ty = rem / g.tpr, tx = rem - ty * g.tpr;
+  const int c = tid % CPR, rg = tid / CPR;
+  uint4 v[PASSES];
+#pragma unroll
+  for (int p = 0; p < PASSES; ++p) {
+    const int row = rg + p * RPP;
+    const int ly = row / g.tw, lx = row - ly * g.tw;
+    const size_t t = (size_t)f * g.tpf + (size_t)(ty * g.th + ly) * g.fw + tx * g.tw + lx;
+    v[p] = __ldg(reinterpret_cast<const uint4*>(x + (t * g.H + h) * D) + c);
+  }
+  for (int j = tid; j < ncand; j += BS_THREADS) {
+    gid[j] = cand_gid[(size_t)h * ncand + j];
+    slot[j] = cand_slot[(size_t)h * ncand + j];
+  }
+  // ---- 2. qbar (fixed-order sums, as in the blockify kernel)
+  float acc[VEC];
+#pragma unroll
+  for (int i = 0; i < VEC; ++i) acc[i] = 0.f;
+#pragma unroll
+  for (int p = 0; p < PASSES; ++p) add_chunk16<T>(acc, v[p]);
+#pragma unroll
+  for (int i = 0; i < VEC; ++i) part[rg][c * VEC + i] = acc[i];
+  __syncthreads();
+  for (int e = tid; e < D; e += BS_THREADS) {
+    float s = 0.f;
+#pragma unroll 4
+    for (int q = 0; q < RPP; ++q) s += part[q][e];
+    s *= (1.0f / BT);
+    qb[e] = s;
+    q_reps[((size_t)h * nq + r) * D + e] = s;
+  }
+  __syncthreads();
+
+  // ---- 3. scores: warp per candidate, lanes over d, BS_BATCH candidates in flight
+  float ql[PL];
+#pragma unroll
+  for (int i = 0; i < PL; ++i) ql[i] = qb[lane * PL + i];
+  constexpr int NW = BS_THREADS / 32;
+  for (int c0 = warp; c0 < ncand; c0 += NW * BS_BATCH) {
+    float kv[BS_BATCH][PL];
+    bool ok[BS_BATCH];
+#pragma unroll
+    for (int b = 0; b < BS_BATCH; ++b) {
+      const int cc = c0 + b * NW;
+      const int s = cc < ncand ? slot[cc] : -1;
+      ok[b] = cc < ncand && s >= 0 && s < pool_slots;
+      if (ok[b]) {
+        const V w = __ldg(reinterpret_cast<const V*>(k_reps + ((size_t)h * pool_slots + s) * D) + lane);
+        vec_to(w, kv[b]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < PL; ++i) kv[b][i] = 0.f;
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < BS_BATCH; ++b) {
+      const int cc = c0 + b * NW;
+      float a = 0.f;
+#pragma unroll
+      for (int i = 0; i < PL; ++i) a = fmaf(ql[i], kv[b][i], a);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+      if (lane == 0 && cc < ncand) {
+        float val = a * g.scale;
+        if (!ok[b]) {
+          if (r == 0) record_error(ws, PBSA_ERR_DEVICE_INDEX, slot[cc], K_SCORE);
+          val = -INFINITY;
+        }
+        if (isnan(val)) val = -INFINITY;
+        sc[cc] = val;
+        key[cc] = rank_key(val, gid[cc]);
+      }
+    }
+  }
+
+  // ---- 4. prefix, count, ranks
+  int pc = prefix_cnt ? prefix_cnt[h] : 0;
+  if (pc < 0 || pc > prefix_ld) {
+    if (tid == 0 && r == 0) record_error(ws, PBSA_ERR_DEVICE_INDEX, pc, K_SCORE);
+    pc = pc < 0 ? 0 : prefix_ld;
+  }
+  const size_t o = (size_t)h * nq + r;
+  for (int j = tid; j < pc; j += BS_THREADS) out_slot[o * out_ld + j] = prefix_slot[(size_t)h * prefix_ld + j];
+  const int kk = min(k, ncand);
+  if (tid == 0) out_cnt[o] = pc + kk;
+  __syncthreads();
+  if (ncand <= SORT_N) {
+    // bitonic sort, descending on (key, -position); padding sorts last
+    __shared__ uint64_t skey[SORT_N];
+    __shared__ int spos[SORT_N];
+    skey[tid] = tid < ncand ? key[tid] : 0ull;
+    spos[tid] = tid < ncand ? tid : SORT_N + tid;
+    __syncthreads();
+    for (int kk2 = 2; kk2 <= SORT_N; kk2 <<= 1) {
+      for (int j = kk2 >> 1; j > 0; j >>= 1) {
+        const int ixj = tid ^ j;
+        const uint64_t a = skey[tid], b = skey[ixj];
+        const int pa = spos[tid], pb = spos[ixj];
+        // does (b, pb) come before (a, pa) in the descending order?
+        const bool b_first = b > a || (b == a && pb < pa);
+        const bool lower = tid < ixj;
+        const bool desc = (tid & kk2) == 0;   // this subsequence is sorted descending
+        const bool take_b = (lower == desc) ? b_first : !b_first;
+        __syncthreads();
+        if (take_b) {
+          skey[tid] = b;
+          spos[tid] = pb;
+        }
+        __syncthreads();
+      }
+    }
+    if (tid < kk) {
+      const int cc = spos[tid];
+      out_slot[o * out_ld + pc + tid] = slot[cc];
+      if (out_score) out_score[o * k + tid] = sc[cc];
+    }
+  } else {
+    for (int cc = tid; cc < ncand; cc += BS_THREADS) {
+      const uint64_t kc = key[cc];
+      int rank = 0;
+#pragma unroll 8
+      for (int c2 = 0; c2 < ncand; ++c2) {
+        const uint64_t k2 = key[c2];
+        rank += (int)(k2 > kc) | ((int)(k2 == kc) & (int)(c2 < cc));
+      }
+      if (rank < kk) {
+        out_slot[o * out_ld + pc + rank] = slot[cc];
+        if (out_score) out_score[o * k + rank] = sc[cc];
+      }
+    }
+  }
+}
+
+template <typename T, int D>
+cudaError_t launch_t(const Geo& g, const void* x, int q_frames, float* q_reps, const float* k_reps,
+                     int pool_slots, const int* cand_slot, const int* cand_gid, int ncand, int k,
+                     const int* prefix_slot, const int* prefix_cnt, int prefix_ld, int* out_slot,
+                     int* out_cnt, int out_ld, float* out_score, void* ws, cudaStream_t st) {
+  const int nq = q_frames * g.bpf;
+  const size_t smem = (size_t)ncand * (8 + 4 + 4 + 4);
+  auto kern = blockify_select_kernel<T, D>;
+  cudaError_t e = set_smem_once((const void*)kern, (int)(smem > 0 ? smem : 8));
+  if (e != cudaSuccess) return e;
+  kern<<<dim3(nq, g.H), BS_THREADS, smem, st>>>(static_cast<const T*>(x), g, nq, q_reps, k_reps,
+                                                 pool_slots, cand_slot, cand_gid, ncand, k,
+                                                 prefix_slot, prefix_cnt, prefix_ld, out_slot,
+                                                 out_cnt, out_ld, out_score, ws);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_blockify_select(const Geo& g, const void* x, int q_frames, float* q_reps,
+                                   const float* k_reps, int pool_slots, const int* cand_slot,
+                                   const int* cand_gid, int ncand, int k, const int* prefix_slot,
+                                   const int* prefix_cnt, int prefix_ld, int* out_slot,
+                                   int* out_cnt, int out_ld, float* out_score, void* ws,
+                                   cudaStream_t st) {
+#define PBSA_BS(TT, DD)                                                                         \
+  return launch_t<TT, DD>(g, x, q_frames, q_reps, k_reps, pool_slots, cand_slot, cand_gid,     \
+                          ncand, k, prefix_slot, prefix_cnt, prefix_ld, out_slot, out_cnt,     \
+                          out_ld, out_score, ws, st);
+  if (g.dtype == PBSA_BF16) {
+    if (g.d == 128) { PBSA_BS(__nv_bfloat16, 128) }
+    if (g.d == 64) { PBSA_BS(__nv_bfloat16, 64) }
+  } else {
+    if (g.d == 128) { PBSA_BS(float, 128) }
+    if (g.d == 64) { PBSA_BS(float, 64) }
+    if (g.d == 32) { PBSA_BS(float, 32) }
+  }
+#undef PBSA_BS
+  return cudaErrorNotSupported;
+}
+
+}  // namespace pbsa

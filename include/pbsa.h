@@ -111,6 +111,25 @@ PBSA_API pbsa_status pbsa_score_select(const pbsa_geom* g, const float* q_reps, 
                               int* out_slot, int* out_cnt, int out_ld, float* out_score,
                               void* ws, void* stream);
 
+/* a1 + a2 fused -- blockify of a query chunk and top-k selection in one pass (the
+ * "lightweight coarse routing" of English 2.C "Local Sparsity" over the blockified latent
+ * space of 2.E; Chinese 2.2 "块化压缩").  Same results as pbsa_blockify(q, q_frames,
+ * q_reps, nq, NULL, NULL, ...) followed by pbsa_score_select(q_reps, nq, ...) with the
+ * same arguments, except that the scores are summed in a different (fixed) order, so
+ * candidates whose scores differ only in the last bits may rank the other way:
+ *   q_reps[h][r] = mean of query block r's 64 tokens (bit-identical to pbsa_blockify)
+ *   out_slot / out_cnt / out_score as for pbsa_score_select.
+ *  q      [q_frames*frame_h*frame_w][H][d] raster, geometry dtype (16-byte aligned);
+ *         nq = q_frames*bpf query blocks.
+ *  q_reps out [H][nq][d] fp32.
+ *  Other arguments as for pbsa_score_select (ncand <= 1024). */
+PBSA_API pbsa_status pbsa_blockify_score_select(const pbsa_geom* g, const void* q, int q_frames,
+                                       float* q_reps, const float* k_reps, int pool_slots,
+                                       const int* cand_slot, const int* cand_gid, int ncand, int k,
+                                       const int* prefix_slot, const int* prefix_cnt, int prefix_ld,
+                                       int* out_slot, int* out_cnt, int out_ld, float* out_score,
+                                       void* ws, void* stream);
+
 /* a3 -- fine attention over the selected blocks (the hybrid mask of the Chinese
  * explainer 2.2 "掩码机制"; English 2.C "Global Access" + "Local Sparsity"):
  * for every token i of query block r of head h,

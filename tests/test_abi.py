@@ -52,3 +52,6 @@ def test_host_side_checks_without_gpu(lib):
                                    None, None) == 1
     odd = P.make_geom(12, 96, 32, 48, 8, 8, 0.1, "bf16")          # head_dim 96 is not built
     assert _lib.load().pbsa_blockify(ctypes.byref(odd), None, 1, None, 1, None, None, 0, None, None) == 2
+    # the fused blockify + select entry point checks its pointers the same way
+    assert _lib.load().pbsa_blockify_score_select(ctypes.byref(g), None, 1, None, None, 10, None, None, 0,
+                                                  0, None, None, 0, None, None, 0, None, None, None) == 1

@@ -108,6 +108,69 @@ def test_score_select(ncand, k, dup):
     assert ncand == 0 or checked >= H * nq // 2
 
 
+# ----------------------------------------------------------------------------- fused blockify + select
+@pytest.mark.parametrize("wname,ncand,k,dup", [("decode", 144, 32, False), ("decode", 48, 32, False),
+                                               ("decode", 300, 16, False), ("decode", 144, 32, True),
+                                               ("decode", 0, 8, False), ("tiny", 8, 4, False),
+                                               ("tile4x16", 20, 32, False)])
+def test_blockify_score_select(wname, ncand, k, dup):
+    """pbsa_blockify_score_select: q reps = the oracle's block means (and bit-identical to
+    pbsa_blockify), selection = the oracle's top-k of its own coarse scores outside near ties."""
+    base = {"decode": dataclasses.replace(I.DECODE_5S, heads=3), "tiny": I.TINY,
+            "tile4x16": dataclasses.replace(I.DECODE_5S, heads=2, tile_h=4, tile_w=16)}[wname]
+    w = base
+    g = geom_for(w)
+    H, d, n_frames = w.heads, w.head_dim, 2
+    nq = n_frames * w.blocks_per_frame
+    x = I.tokens(w, n_frames, 21 + ncand)
+    gen = torch.Generator().manual_seed(5 + ncand)
+    pool, prefix = 400, 20
+    kr = torch.randn((H, pool, d), generator=gen) * 0.3
+    if dup:
+        kr[:] = kr[:, :1]
+    cs = torch.stack([torch.randperm(pool, generator=gen)[:ncand] for _ in range(H)]).to(torch.int32)
+    cg = torch.stack([torch.randperm(5000, generator=gen)[:ncand] for _ in range(H)]).to(torch.int32)
+    ps = torch.randint(0, pool, (H, prefix), generator=gen, dtype=torch.int32)
+    pc = torch.tensor([prefix - h for h in range(H)], dtype=torch.int32)
+    out_ld = prefix + k + 3
+    out = torch.full((H, nq, out_ld), -7, dtype=torch.int32, device=DEV)
+    cnt = torch.zeros((H, nq), dtype=torch.int32, device=DEV)
+    sc = torch.zeros((H, nq, max(k, 1)), device=DEV)
+    qr = torch.zeros((H, nq, d), device=DEV)
+    ws = ws_for(g)
+    xd = x.to(DEV)
+    P.pbsa_blockify_score_select(g, xd, n_frames, qr, kr.to(DEV), pool, cs.to(DEV) if ncand else None,
+                                 cg.to(DEV) if ncand else None, ncand, k, ps.to(DEV), pc.to(DEV), prefix,
+                                 out, cnt, out_ld, sc, ws)
+    check_no_device_error(ws)
+    qr_sep = torch.zeros_like(qr)
+    P.pbsa_blockify(g, xd, n_frames, qr_sep, nq, ws=ws)
+    assert torch.equal(qr, qr_sep)
+    want_q = O.block_reps(f64(x), geom_dict(w), n_frames)
+    np.testing.assert_allclose(f64(qr), want_q, rtol=0, atol=2e-6)
+    out, cnt, sc = out.cpu(), cnt.cpu(), sc.cpu()
+    kk = min(k, ncand)
+    checked = 0
+    for h in range(H):
+        for r in range(nq):
+            p = int(pc[h])
+            assert int(cnt[h, r]) == p + kk
+            assert out[h, r, :p].tolist() == ps[h, :p].tolist()
+            if ncand == 0:
+                continue
+            s64 = O.coarse_scores(want_q[h, r:r + 1], f64(kr[h][cs[h].long()]), w.scale)[0]
+            s32 = s64.astype(np.float32)
+            want_pos = O.topk_select(s32, cg[h].tolist(), k)
+            got_slots = out[h, r, p:p + kk].tolist()
+            np.testing.assert_allclose(sc[h, r, :kk].numpy(), s32[want_pos], rtol=0, atol=2e-5)
+            if dup or O.kth_gap(s32, cg[h].tolist(), k) > NEAR_TIE:
+                assert set(got_slots) == {int(cs[h, i]) for i in want_pos}
+                checked += 1
+            else:
+                assert len(set(got_slots)) == kk and set(got_slots) <= set(cs[h].tolist())
+    assert ncand == 0 or checked >= H * nq // 2
+
+
 # ----------------------------------------------------------------------------- attend
 def _attend_case(w, q_frames, slots, lists, seed):
     gen = torch.Generator().manual_seed(seed)
