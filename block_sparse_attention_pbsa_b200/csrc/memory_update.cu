@@ -6,15 +6,15 @@
 // are dropped, and the sink blocks are always kept.  The scoring rule is fixed as an EMA of
 // each block's mean (over the chunk's query blocks) softmaxed coarse score.
 //
-// Three launches on the caller's stream:
-//   1. mu_score_kernel  -- one CTA per (head, 8 query blocks): coarse scores against every
-//      pool entry (representatives staged in shared memory) and the per-row softmax,
-//      written to the workspace;
-//   2. mu_select_kernel -- one CTA per head: a_b = mean_r p_{r,b} (coalesced, fixed-order
-//      sums), the EMA, the rank of every non-sink block, the new slot table and a copy
-//      list in the workspace;
-//   3. mu_copy_kernel   -- one CTA per (copy, head, K|V): promoted blocks are copied from
-//      their window slots into the freed persistent slots (HBM-bound 16-byte copies).
+// Two launches on the caller's stream:
+//   1. mu_score_select_kernel -- one CTA per (head, 4 query blocks): coarse scores against
+//      every pool entry (warp per entry, lanes over d), the per-row softmax, and the column
+//      sums of its rows written to the workspace.  The last CTA of each head to finish
+//      (an atomic count in the workspace, reset by that CTA) then sums the column partials
+//      in a fixed order (a_b = mean_r p_{r,b}), applies the EMA, ranks every non-sink block,
+//      and writes the new slot table, the persistent list and a copy list;
+//   2. mu_copy_kernel -- one CTA per (copy, head, K|V): promoted blocks are copied from their
+//      window slots into the freed persistent slots (HBM-bound 16-byte copies).
 // All reductions run in a fixed order, so the update is deterministic.
 #include <math.h>
 
@@ -28,21 +28,24 @@ constexpr int MU_THREADS = 256;
 
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+constexpr int MU_RQ = 4;       // query rows per score CTA
+constexpr int MU_BATCH = 12;   // pool entries per warp in flight
+
 struct MuLayout {
-  size_t p_off, copy_off, ncopy_off, end;
+  size_t part_off, copy_off, ncopy_off, count_off, end;
 };
+// part [H][ceil(nq / MU_RQ)][nb] column partial sums; copy list [H][nb][2]; ncopy [H];
+// count [H] finished score CTAs per head (zero between calls)
 __host__ __device__ inline MuLayout mu_layout(int H, int nq, int nb) {
   MuLayout L;
-  L.p_off = WS_HEADER_BYTES;
-  L.copy_off = L.p_off + align256((size_t)H * nq * nb * sizeof(float));
+  const size_t nqb = (size_t)(nq + MU_RQ - 1) / MU_RQ;
+  L.part_off = WS_HEADER_BYTES;
+  L.copy_off = L.part_off + align256((size_t)H * nqb * nb * sizeof(float));
   L.ncopy_off = L.copy_off + align256((size_t)H * nb * 2 * sizeof(int));
-  L.end = L.ncopy_off + align256((size_t)H * sizeof(int));
+  L.count_off = L.ncopy_off + align256((size_t)H * sizeof(int));
+  L.end = L.count_off + align256((size_t)H * sizeof(int));
   return L;
 }
-
-constexpr int MU_RC = 8;       // query rows per score CTA
-constexpr int MU_CH = 128;     // pool entries staged per pass
-constexpr int MU_SEL_THREADS = 512;
 
 // Pool entry j of head h: j < C is persistent slot j (empty when its gid < 0), j >= C is
 // candidate j - C, which must live outside the persistent region.  Returns the gid (-1 for
@@ -64,132 +67,50 @@ __device__ __forceinline__ int entry_of(int j, int h, int C, int ncand, int pool
   return g;
 }
 
-template <int D>
-__global__ void __launch_bounds__(MU_THREADS) mu_score_kernel(
-    const float* __restrict__ q_reps, int nq, const float* __restrict__ k_reps, int pool_slots,
-    const int* __restrict__ slot_gid, int C, const int* __restrict__ cand_slot,
-    const int* __restrict__ cand_gid, int ncand, float scale, float* __restrict__ p_out, void* ws) {
-  constexpr int DP = D + 1;
-  extern __shared__ float smem[];
-  const int h = blockIdx.y, r0 = blockIdx.x * MU_RC, nb = C + ncand;
-  const int nr = min(MU_RC, nq - r0);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  float* ks = smem;                          // [MU_CH][DP]
-  float* qs = ks + MU_CH * DP;               // [MU_RC][D]
-  float* sc = qs + MU_RC * D;                // [MU_RC][nb]
-  int* gid = reinterpret_cast<int*>(sc + MU_RC * nb);   // [nb]
-  int* eslot = gid + nb;                                 // [nb]
+template <int N> struct MuVec;
+template <> struct MuVec<4> { using type = float4; };
+template <> struct MuVec<2> { using type = float2; };
+template <> struct MuVec<1> { using type = float; };
+__device__ __forceinline__ void mu_vec_to(const float4& v, float* o) { o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w; }
+__device__ __forceinline__ void mu_vec_to(const float2& v, float* o) { o[0] = v.x; o[1] = v.y; }
+__device__ __forceinline__ void mu_vec_to(const float& v, float* o) { o[0] = v; }
 
-  for (int j = tid; j < nb; j += MU_THREADS) {
-    int sl;
-    gid[j] = entry_of(j, h, C, ncand, pool_slots, slot_gid, cand_slot, cand_gid, &sl, ws, blockIdx.x == 0);
-    eslot[j] = sl;
-  }
-  for (int i = tid; i < MU_RC * D; i += MU_THREADS) {
-    const int r = i / D;
-    qs[i] = r < nr ? q_reps[((size_t)h * nq + r0 + r) * D + (i - r * D)] : 0.f;
-  }
-  for (int base = 0; base < nb; base += MU_CH) {
-    const int nc = min(MU_CH, nb - base);
-    __syncthreads();   // metadata ready / previous pass done with ks
-    stage_rows<D, DP, MU_THREADS>(ks, nc, [&](int c) -> const float* {
-      return gid[base + c] >= 0 ? k_reps + ((size_t)h * pool_slots + eslot[base + c]) * D : nullptr;
-    });
-    __syncthreads();
-    for (int p = tid; p < nc * (MU_RC / 4); p += MU_THREADS) {
-      const int c = p % nc, rg = (p / nc) * 4;
-      float a4[4] = {0.f, 0.f, 0.f, 0.f};
-      const float* kr = ks + c * DP;
-#pragma unroll 8
-      for (int e = 0; e < D; ++e) {
-        const float kv = kr[e];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) a4[j] = fmaf(qs[(rg + j) * D + e], kv, a4[j]);
-      }
-      const bool ok = gid[base + c] >= 0;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) sc[(rg + j) * nb + base + c] = ok ? a4[j] * scale : -INFINITY;
-    }
-  }
-  __syncthreads();
-  // softmax of each row over the pool (one warp per row, fixed-order reductions)
-  for (int r = warp; r < nr; r += MU_THREADS / 32) {
-    const float* row = sc + r * nb;
-    float m = -INFINITY;
-    for (int j = lane; j < nb; j += 32) m = fmaxf(m, row[j]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    float sum = 0.f;
-    for (int j = lane; j < nb; j += 32) sum += row[j] == -INFINITY ? 0.f : expf(row[j] - m);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    const float inv = sum > 0.f ? 1.0f / sum : 0.f;
-    float* prow = p_out + ((size_t)h * nq + r0 + r) * nb;
-    for (int j = lane; j < nb; j += 32) prow[j] = row[j] == -INFINITY ? 0.f : expf(row[j] - m) * inv;
-  }
-}
-
-__global__ void __launch_bounds__(MU_SEL_THREADS) mu_select_kernel(
-    const float* __restrict__ p_in, int nq, int pool_slots, int* __restrict__ slot_gid,
-    float* __restrict__ slot_ema, int C, int n_sink_gid, const int* __restrict__ cand_slot,
-    const int* __restrict__ cand_gid, int ncand, float gamma, int* __restrict__ copy_list,
-    int* __restrict__ ncopy, int* __restrict__ p_list, int* __restrict__ p_cnt, void* ws) {
-  constexpr int NW = MU_SEL_THREADS / 32;
-  extern __shared__ float smem[];
-  const int h = blockIdx.x, nb = C + ncand;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  float* part = smem;                        // [NW][nb] per-warp partial sums over rows
-  float* ema = part + NW * nb;               // [nb]
-  int* gid = reinterpret_cast<int*>(ema + nb);   // [nb]
-  int* eslot = gid + nb;                         // [nb]
-  int* rank = eslot + nb;                        // [nb]
-  int* by_rank = rank + nb;                      // [nb]
-  int* filled = by_rank + nb;                    // [nb]
-  int* flist = filled + nb;                      // [nb] freed persistent slots, ascending
-  int* plist2 = flist + nb;                      // [nb] promoted entries, in promotion order
+// The selection of one head from its a_b (in ema[], overwritten by the EMA): ranks, slot
+// assignment, slot table, copy list, persistent list.  Run by one CTA (all threads).
+__device__ void mu_select_head(int h, int nb, int pool_slots, int* __restrict__ slot_gid,
+                               float* __restrict__ slot_ema, int C, int n_sink_gid, float gamma,
+                               const int* gid, const int* eslot, float* ema, uint64_t* key, int* rank,
+                               int* by_rank, int* filled, int* flist, int* plist2, int* __restrict__ copy_list,
+                               int* __restrict__ ncopy, int* __restrict__ p_list, int* __restrict__ p_cnt,
+                               void* ws) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, NT = blockDim.x;
   __shared__ int n_sink_s, n_free_s, n_promo_s;
   if (tid == 0) n_sink_s = 0;
-  for (int j = tid; j < nb; j += MU_SEL_THREADS) {
-    int sl;
-    gid[j] = entry_of(j, h, C, ncand, pool_slots, slot_gid, cand_slot, cand_gid, &sl, ws, false);
-    eslot[j] = sl;
+  __syncthreads();
+  for (int j = tid; j < nb; j += NT) {
+    const int g = gid[j];
+    const float a = ema[j];
+    const float e = (g >= 0 && j < C) ? fmaf(gamma, slot_ema[(size_t)h * C + j], (1.0f - gamma) * a) : a;
+    ema[j] = e;
+    // ranking key of a non-sink block: larger EMA first, then the lower gid; empty entries
+    // and sinks get 0, below every ranked key
+    key[j] = g >= n_sink_gid ? rank_key(e, g) : 0ull;
+    if (g >= 0 && g < n_sink_gid) atomicAdd(&n_sink_s, 1);
     by_rank[j] = -1;
     filled[j] = 0;
   }
-  // warp w sums rows w, w + NW, ...; lanes walk consecutive entries (coalesced)
-  const float* pbase = p_in + (size_t)h * nq * nb;
-  for (int j0 = 0; j0 < nb; j0 += 32) {
-    const int j = j0 + lane;
-    float a = 0.f;
-    if (j < nb) {
-#pragma unroll 4
-      for (int r = warp; r < nq; r += NW) a += pbase[(size_t)r * nb + j];
-      part[warp * nb + j] = a;
-    }
-  }
-  __syncthreads();
-  const float inv_nq = 1.0f / (float)nq;
-  for (int j = tid; j < nb; j += MU_SEL_THREADS) {
-    float a = 0.f;
-    for (int w = 0; w < NW; ++w) a += part[w * nb + j];
-    a *= inv_nq;
-    const int g = gid[j];
-    ema[j] = (g >= 0 && j < C) ? fmaf(gamma, slot_ema[(size_t)h * C + j], (1.0f - gamma) * a) : a;
-    if (g >= 0 && g < n_sink_gid) atomicAdd(&n_sink_s, 1);
-  }
   __syncthreads();
   const int free_places = max(0, C - n_sink_s);
-  for (int j = tid; j < nb; j += MU_SEL_THREADS) {
-    const int g = gid[j];
+  // rank = #ranked keys above this one, plus equal keys at a lower entry (branch-free)
+  for (int j = tid; j < nb; j += NT) {
+    const uint64_t kj = key[j];
     int rk = -1;
-    if (g >= n_sink_gid) {
-      const float e = ema[j];
+    if (kj != 0ull) {
       rk = 0;
+#pragma unroll 8
       for (int j2 = 0; j2 < nb; ++j2) {
-        const int g2 = gid[j2];
-        if (g2 < n_sink_gid) continue;  // empty entries and sinks are not ranked
-        const float e2 = ema[j2];
-        rk += (e2 > e) || (e2 == e && (g2 < g || (g2 == g && j2 < j)));
+        const uint64_t k2 = key[j2];
+        rk += (int)(k2 > kj) | ((int)(k2 == kj) & (int)(j2 < j));
       }
       if (rk < free_places) by_rank[rk] = j;
     }
@@ -235,7 +156,7 @@ __global__ void __launch_bounds__(MU_SEL_THREADS) mu_select_kernel(
   }
   __syncthreads();
   const int n_promo = n_promo_s, n_free = n_free_s;
-  for (int t = tid; t < n_promo; t += MU_SEL_THREADS) {
+  for (int t = tid; t < n_promo; t += NT) {
     const int j = plist2[t];
     if (t >= n_free) {
       record_error(ws, PBSA_ERR_INVALID_ARG, j, K_MU_SELECT);
@@ -251,7 +172,7 @@ __global__ void __launch_bounds__(MU_SEL_THREADS) mu_select_kernel(
   if (tid == 0) ncopy[h] = min(n_promo, n_free);
   __syncthreads();
   // kept persistent entries take their new EMA; slots neither kept nor refilled are cleared
-  for (int j = tid; j < C; j += MU_SEL_THREADS) {
+  for (int j = tid; j < C; j += NT) {
     if (stays(j)) {
       slot_ema[(size_t)h * C + j] = ema[j];
     } else if (!filled[j]) {
@@ -271,6 +192,134 @@ __global__ void __launch_bounds__(MU_SEL_THREADS) mu_select_kernel(
     }
     if (lane == 0 && p_cnt) p_cnt[h] = n;
   }
+}
+
+template <int D>
+__global__ void __launch_bounds__(MU_THREADS) mu_score_select_kernel(
+    const float* __restrict__ q_reps, int nq, const float* __restrict__ k_reps, int pool_slots,
+    int* __restrict__ slot_gid, float* __restrict__ slot_ema, int C, int n_sink_gid,
+    const int* __restrict__ cand_slot, const int* __restrict__ cand_gid, int ncand, float gamma,
+    float scale, float* __restrict__ part, int* __restrict__ copy_list, int* __restrict__ ncopy,
+    int* __restrict__ count, int* __restrict__ p_list, int* __restrict__ p_cnt, void* ws) {
+  constexpr int PL = D / 32;          // elements of a row per lane
+  constexpr int NW = MU_THREADS / 32;
+  using V = typename MuVec<PL>::type;
+  extern __shared__ float smem[];
+  const int h = blockIdx.y, r0 = blockIdx.x * MU_RQ, nb = C + ncand;
+  const int nr = min(MU_RQ, nq - r0);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  int* gid = reinterpret_cast<int*>(smem);          // [nb]
+  int* eslot = gid + nb;                             // [nb]
+  float* qs = reinterpret_cast<float*>(eslot + nb);  // [MU_RQ][D]
+  float* sc = qs + MU_RQ * D;                        // [MU_RQ][nb] scores, then p
+  __shared__ int last_s;
+
+  for (int j = tid; j < nb; j += MU_THREADS) {
+    int sl;
+    gid[j] = entry_of(j, h, C, ncand, pool_slots, slot_gid, cand_slot, cand_gid, &sl, ws, blockIdx.x == 0);
+    eslot[j] = sl;
+  }
+  for (int i = tid; i < MU_RQ * D; i += MU_THREADS) {
+    const int r = i / D;
+    qs[i] = r < nr ? q_reps[((size_t)h * nq + r0 + r) * D + (i - r * D)] : 0.f;
+  }
+  __syncthreads();
+
+  // ---- scores: warp per pool entry, lanes over d, MU_BATCH entries in flight
+  float ql[MU_RQ][PL];
+#pragma unroll
+  for (int r = 0; r < MU_RQ; ++r)
+#pragma unroll
+    for (int i = 0; i < PL; ++i) ql[r][i] = qs[r * D + lane * PL + i];
+  for (int j0 = warp; j0 < nb; j0 += NW * MU_BATCH) {
+    float kv[MU_BATCH][PL];
+#pragma unroll
+    for (int b = 0; b < MU_BATCH; ++b) {
+      const int j = j0 + b * NW;
+      if (j < nb && gid[j] >= 0) {
+        const V w = __ldg(reinterpret_cast<const V*>(k_reps + ((size_t)h * pool_slots + eslot[j]) * D) + lane);
+        mu_vec_to(w, kv[b]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < PL; ++i) kv[b][i] = 0.f;
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < MU_BATCH; ++b) {
+      const int j = j0 + b * NW;
+      float a[MU_RQ];
+#pragma unroll
+      for (int r = 0; r < MU_RQ; ++r) {
+        a[r] = 0.f;
+#pragma unroll
+        for (int i = 0; i < PL; ++i) a[r] = fmaf(ql[r][i], kv[b][i], a[r]);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int r = 0; r < MU_RQ; ++r) a[r] += __shfl_xor_sync(0xffffffffu, a[r], o);
+      if (lane == 0 && j < nb) {
+        const bool ok = gid[j] >= 0;
+#pragma unroll
+        for (int r = 0; r < MU_RQ; ++r) sc[r * nb + j] = ok ? a[r] * scale : -INFINITY;
+      }
+    }
+  }
+  __syncthreads();
+  // ---- softmax of each row over the pool (one warp per row, fixed-order reductions)
+  for (int r = warp; r < nr; r += NW) {
+    float* row = sc + r * nb;
+    float m = -INFINITY;
+    for (int j = lane; j < nb; j += 32) m = fmaxf(m, row[j]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float sum = 0.f;
+    for (int j = lane; j < nb; j += 32) sum += row[j] == -INFINITY ? 0.f : expf(row[j] - m);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    const float inv = sum > 0.f ? 1.0f / sum : 0.f;
+    __syncwarp();
+    for (int j = lane; j < nb; j += 32) row[j] = row[j] == -INFINITY ? 0.f : expf(row[j] - m) * inv;
+  }
+  __syncthreads();
+  // ---- column sums of this CTA's rows (row order), then count this CTA as done
+  float* my_part = part + ((size_t)h * gridDim.x + blockIdx.x) * nb;
+  for (int j = tid; j < nb; j += MU_THREADS) {
+    float a = 0.f;
+    for (int r = 0; r < nr; ++r) a += sc[r * nb + j];
+    my_part[j] = a;
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) last_s = atomicAdd(&count[h], 1) == (int)gridDim.x - 1;
+  __syncthreads();
+  if (!last_s) return;
+  __threadfence();
+  // ---- the last CTA of head h: a_b = mean over all rows, summed over the partials in order
+  float* ema = sc;                                    // [nb]
+  uint64_t* key = reinterpret_cast<uint64_t*>(sc + 2 * ((nb + 1) / 2) + 2);  // [nb], 8-byte aligned
+  int* rank = reinterpret_cast<int*>(key + nb);       // [nb]
+  int* by_rank = rank + nb;                           // [nb]
+  int* filled = by_rank + nb;                         // [nb]
+  int* flist = filled + nb;                           // [nb] freed persistent slots, ascending
+  int* plist2 = flist + nb;                           // [nb] promoted entries, in promotion order
+  const float* hpart = part + (size_t)h * gridDim.x * nb;
+  const float inv_nq = 1.0f / (float)nq;
+  const int nparts = (int)gridDim.x;
+  for (int j = tid; j < nb; j += MU_THREADS) {
+    float a = 0.f;
+    for (int b0 = 0; b0 < nparts; b0 += 8) {   // eight loads in flight, summed in order
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = b0 + u < nparts ? __ldcg(hpart + (size_t)(b0 + u) * nb + j) : 0.f;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) a += v[u];
+    }
+    ema[j] = a * inv_nq;
+  }
+  mu_select_head(h, nb, pool_slots, slot_gid, slot_ema, C, n_sink_gid, gamma, gid, eslot, ema, key, rank,
+                 by_rank, filled, flist, plist2, copy_list, ncopy, p_list, p_cnt, ws);
+  if (tid == 0) count[h] = 0;   // ready for the next call
 }
 
 template <typename T, int D>
@@ -313,21 +362,20 @@ cudaError_t launch_mu(const Geo& g, const float* q_reps, int nq, float* k_reps, 
   const int nb = C + ncand;
   const MuLayout L = mu_layout(g.H, nq, nb);
   char* base = static_cast<char*>(ws);
+  float* part = reinterpret_cast<float*>(base + L.part_off);
   int* copy_list = reinterpret_cast<int*>(base + L.copy_off);
   int* ncopy = reinterpret_cast<int*>(base + L.ncopy_off);
+  int* count = reinterpret_cast<int*>(base + L.count_off);
   cudaError_t e;
 
-  float* p = reinterpret_cast<float*>(base + L.p_off);
-  const size_t smem1 = ((size_t)MU_CH * (D + 1) + (size_t)MU_RC * D + (size_t)MU_RC * nb) * 4 + (size_t)nb * 8;
-  if ((e = set_smem_once((const void*)mu_score_kernel<D>, (int)smem1)) != cudaSuccess) return e;
-  mu_score_kernel<D><<<dim3((nq + MU_RC - 1) / MU_RC, g.H), MU_THREADS, smem1, st>>>(
-      q_reps, nq, k_reps, pool_slots, slot_gid, C, cand_slot, cand_gid, ncand, g.scale, p, ws);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const size_t smem2 = ((size_t)(MU_SEL_THREADS / 32) * nb + nb) * 4 + (size_t)nb * 7 * sizeof(int);
-  if ((e = set_smem_once((const void*)mu_select_kernel, (int)smem2)) != cudaSuccess) return e;
-  mu_select_kernel<<<g.H, MU_SEL_THREADS, smem2, st>>>(p, nq, pool_slots, slot_gid, slot_ema, C, n_sink_gid,
-                                                        cand_slot, cand_gid, ncand, gamma, copy_list, ncopy,
-                                                        p_list, p_cnt, ws);
+  // smem: gid, eslot [nb] + q rows [MU_RQ][D] + max(scores [MU_RQ][nb], select arrays: 6 x 4
+  // bytes + 8-byte keys per entry, plus alignment)
+  const size_t sel = (size_t)14 * nb * 4 + 16, sco = (size_t)MU_RQ * nb * 4;
+  const size_t smem = (size_t)2 * nb * 4 + (size_t)MU_RQ * D * 4 + (sel > sco ? sel : sco);
+  if ((e = set_smem_once((const void*)mu_score_select_kernel<D>, (int)smem)) != cudaSuccess) return e;
+  mu_score_select_kernel<D><<<dim3((nq + MU_RQ - 1) / MU_RQ, g.H), MU_THREADS, smem, st>>>(
+      q_reps, nq, k_reps, pool_slots, slot_gid, slot_ema, C, n_sink_gid, cand_slot, cand_gid, ncand,
+      gamma, g.scale, part, copy_list, ncopy, count, p_list, p_cnt, ws);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
   const int max_copies = C < nb ? C : nb;

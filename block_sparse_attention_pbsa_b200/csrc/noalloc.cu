@@ -13,8 +13,10 @@
 // cudaGetSymbolAddress (the array's name in host code is only a stand-in, never a
 // device address) and caches the pointer; make that first call before any stream
 // capture.  Every call shares the array and finds the previous call's contents in it:
-// the error word is cleared on the caller's stream at the start of each call, and the
-// kernels write every other scratch byte they read.  Two calls whose work overlaps on
+// the error word is cleared on the caller's stream at the start of each call, the
+// per-head completion counts of the score kernel start at zero (the array is zero when the
+// library loads) and every call leaves them at zero, and the kernels write every other
+// scratch byte they read.  Two calls whose work overlaps on
 // the GPU (different streams, or the same stream from two threads without ordering)
 // race on the array.  Device-side index errors found by this variant are recorded in
 // the scratch and not reported to the caller.
