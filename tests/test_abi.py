@@ -43,7 +43,9 @@ def test_host_side_checks_without_gpu(lib):
     P.load()
     assert P.pbsa_status_string(0) == "ok" and P.pbsa_status_string(5).startswith("index")
     g = P.make_geom(12, 128, 32, 48, 8, 8, 128 ** -0.5, "bf16")
-    assert P.pbsa_workspace_bytes(g, 72, 360) >= 256 + 12 * 72 * 360 * 4
+    # error word + per-head column partial sums of four-row groups (18 for 72 query blocks)
+    assert P.pbsa_workspace_bytes(g, 72, 360) >= 256 + 12 * 18 * 360 * 4
+    assert P.pbsa_workspace_bytes(g, 72, 360) >= P.pbsa_workspace_bytes(g, 8, 40) > 256
     bad = P.make_geom(12, 128, 32, 48, 8, 7, 0.1, "bf16")        # tile is not 64 tokens
     assert _lib.load().pbsa_blockify(ctypes.byref(bad), None, 1, None, 1, None, None, 0, None, None) == 1
     assert _lib.load().pbsa_workspace_bytes(ctypes.byref(bad), 1, 1) == 0
