@@ -21,6 +21,7 @@ from __future__ import annotations
 
 import argparse
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -260,6 +261,96 @@ def run_train(P, I, dev, steps: int, peaks):
                     "the deterministic kernels recompute S and dP in both the dQ and the dK/dV passes"}
 
 
+def run_rollout(P, I, dev, w, max_chunks=None):
+    """A whole rollout through the layer caches: ``w.layers`` layers, ``w.steps`` denoising
+    steps per chunk sharing the persistent memory, the memory update once per finished chunk.
+
+    Inputs are fresh N(0,1) tokens per (chunk, step, layer, tensor) plus per-tile offsets
+    (i.i.d. per chunk, or an AR(1) drift across frames for ``w.ar_rho`` > 0), drawn on the
+    device before each chunk's timed region.  Each chunk (all layers and steps, then the
+    commits) is timed with CUDA events around eager launches on one stream.
+    """
+    H, d, bpf = w.heads, w.head_dim, w.blocks_per_frame
+    cfg = P.LayerConfig(H, d, w.frame_h, w.frame_w, w.tile_h, w.tile_w, w.capacity, w.window_frames,
+                        w.chunk_frames, w.topk, w.gamma, w.dtype, 0)
+    torch.cuda.synchronize(dev)
+    base_alloc = torch.cuda.memory_allocated(dev)
+    caches = [P.PBSALayerCache(cfg, dev) for _ in range(w.layers)]
+    kv_alloc = torch.cuda.memory_allocated(dev) - base_alloc
+    chunks = I.rollout_chunks(w)[:max_chunks]
+    ty, tx = w.frame_h // w.tile_h, w.frame_w // w.tile_w
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(I.stream_seed(w.seed, 7000))
+    s_off = w.block_offset_std
+    ar = None
+    if w.ar_rho > 0:   # AR(1) tile offsets per (layer, tensor), stepped once per frame
+        ar = torch.randn((w.layers, 3, ty, tx, H, d), generator=gen, device=dev) * s_off
+    c_ar = math.sqrt(max(0.0, 1.0 - w.ar_rho ** 2))
+
+    def draw(nf):
+        """[steps][layers] lists of (q, k, v) for a chunk of nf frames."""
+        nonlocal ar
+        if ar is not None:
+            offs = []
+            for _ in range(nf):
+                ar = w.ar_rho * ar + c_ar * s_off * torch.randn(ar.shape, generator=gen, device=dev)
+                offs.append(ar)
+            off = torch.stack(offs, 2)                                 # [L, 3, nf, ty, tx, H, d]
+        out = []
+        for _ in range(w.steps):
+            if ar is None:
+                off = torch.randn((w.layers, 3, nf, ty, tx, H, d), generator=gen, device=dev) * s_off
+            x = torch.randn((w.layers, 3, nf, ty, w.tile_h, tx, w.tile_w, H, d), generator=gen, device=dev)
+            x = (x + off[:, :, :, :, None, :, None]).view(w.layers, 3, nf * w.tokens_per_frame, H, d)
+            x = x.to(torch.bfloat16)
+            out.append([(x[l, 0], x[l, 1], x[l, 2]) for l in range(w.layers)])
+        return out
+
+    stream = torch.cuda.current_stream(dev)
+    per_chunk, flops_chunk, o = [], [], None
+    peak_alloc = 0
+    for c, (f0, nf) in enumerate(chunks):
+        inp = draw(nf)
+        if o is None or o.shape[0] != nf * w.tokens_per_frame:
+            o = torch.empty((nf * w.tokens_per_frame, H, d), dtype=torch.bfloat16, device=dev)
+        torch.cuda.synchronize(dev)
+        torch.cuda.reset_peak_memory_stats(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for s in range(w.steps):
+            for l in range(w.layers):
+                q, k, v = inp[s][l]
+                caches[l].decode_step(q, k, v, o=o)
+        cnt_layer0 = caches[0].kv_cnt.clone() if caches[0].hist > 0 else None
+        for l in range(w.layers):
+            q, k, v = inp[w.steps - 1][l]
+            caches[l].commit(k, v)
+        e1.record(stream)
+        e1.synchronize()
+        per_chunk.append(e0.elapsed_time(e1))
+        peak_alloc = max(peak_alloc, torch.cuda.max_memory_allocated(dev) - base_alloc)
+        blocks = int(cnt_layer0.sum().item()) if cnt_layer0 is not None else H * (nf * bpf) ** 2
+        flops_chunk.append(4.0 * 64 * 64 * d * blocks * w.steps * w.layers)
+        del inp
+        _check_device(P, caches[0].ws, f"in rollout chunk {c}")
+    kv_bytes = sum(ca.kv_bytes for ca in caches)
+    dense = 2 * w.layers * H * w.total_frames * w.tokens_per_frame * d * 2
+    steady = [i for i in range(len(chunks)) if i >= min(4, len(chunks) - 1)]
+    ms_steady = statistics.mean(per_chunk[i] for i in steady)
+    tf_steady = sum(flops_chunk[i] for i in steady) / (sum(per_chunk[i] for i in steady) * 1e-3) / 1e12
+    return {
+        "workload": w.name, "layers": w.layers, "steps_per_chunk": w.steps, "chunks": len(chunks),
+        "ms_per_chunk": [round(x, 3) for x in per_chunk],
+        "ms_per_chunk_steady": ms_steady, "steady_chunks": f"{steady[0]}..{steady[-1]}",
+        "selected_tflops_steady": tf_steady,
+        "kv_cache_bytes": {"pbsa_all_layers": kv_bytes, "dense_all_frames_all_layers": dense,
+                           "ratio": kv_bytes / dense, "allocated_by_caches": kv_alloc,
+                           "peak_allocated_during_chunks": peak_alloc},
+        "timing": "CUDA events around each chunk's eager launches (all layers x steps, then commits)",
+        "inputs": "device-drawn N(0,1) + per-tile offsets" + (" (AR(1) drift)" if w.ar_rho > 0 else ""),
+    }
+
+
 def rank_workload(w, rank: int):
     """Weak scaling: every rank decodes its own independent layer (same shapes, its own seed)."""
     import dataclasses
@@ -411,6 +502,8 @@ def run_pbsa(args, w, rank, world, local_rank):
     }
     if not args.no_train:
         line["train"] = run_train(P, I, dev, 5, peaks)
+    if not args.no_rollout:
+        line["rollouts"] = [run_rollout(P, I, dev, I.ROLLOUT_5S), run_rollout(P, I, dev, I.ROLLOUT_1MIN)]
     if world == 1 and not args.no_cpu_baseline:
         t, desc, threads = oracle_sample(w, q, k, v, units=24)
         line["cpu_baseline"] = {"value": flops / t / 1e12, "unit": "TFLOP/s", "cores": threads,
@@ -427,6 +520,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-train", action="store_true", help="skip the forward+backward training workload")
     ap.add_argument("--train-only", action="store_true", help="only the training workload (for profiling)")
+    ap.add_argument("--no-rollout", action="store_true", help="skip the 30-layer 5 s and 1-minute rollouts")
     args = ap.parse_args()
     from block_sparse_attention_pbsa_b200 import inputs as I
     w = I.DECODE_5S

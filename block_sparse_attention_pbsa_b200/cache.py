@@ -97,6 +97,24 @@ class PBSALayerCache:
         t = torch.tensor(rows, dtype=torch.int32).pin_memory()
         return t.to(self.device, non_blocking=True)
 
+    # Candidate lists depend only on the ring geometry and the frame schedule, which every
+    # layer of a model shares: they are built once per (device, heads, ring, list) and reused.
+    _LIST_MEMO: dict = {}
+
+    def _list_pair(self, pairs) -> tuple[torch.Tensor, torch.Tensor]:
+        """Device tensors [H, n] of the slots and gids of ``pairs`` (a list of (slot, gid))."""
+        H = self.cfg.heads
+        key = (str(self.device), H, self.ring_frames, self.cfg.bpf, self.ring_base, tuple(pairs))
+        hit = PBSALayerCache._LIST_MEMO.get(key)
+        if hit is None:
+            n = len(pairs)
+            hit = (self._ints([[s for s, _ in pairs]] * H).view(H, n),
+                   self._ints([[g for _, g in pairs]] * H).view(H, n))
+            if len(PBSALayerCache._LIST_MEMO) > 4096:
+                PBSALayerCache._LIST_MEMO.clear()
+            PBSALayerCache._LIST_MEMO[key] = hit
+        return hit
+
     def _frames_dst(self, first: int, n: int) -> torch.Tensor:
         key = (first % self.ring_frames, n)
         if key not in self._dst_cache:
@@ -108,13 +126,12 @@ class PBSALayerCache:
     def _refresh_window(self):
         bpf, H = self.cfg.bpf, self.cfg.heads
         frames = self.window_frames()
-        slots = [self.ring_slot(f, t) for f in frames for t in range(bpf)]
-        gids = [f * bpf + t for f in frames for t in range(bpf)]
-        n = len(slots)
-        if n == 0:
+        pairs = [(self.ring_slot(f, t), f * bpf + t) for f in frames for t in range(bpf)]
+        if not pairs:
             self._cand = (None, None, 0)
             return
-        self._cand = (self._ints([slots] * H).view(H, n), self._ints([gids] * H).view(H, n), n)
+        cs, cg = self._list_pair(pairs)
+        self._cand = (cs, cg, len(pairs))
 
     @property
     def kv_bytes(self) -> int:
@@ -243,11 +260,7 @@ class PBSALayerCache:
     def _update(self, q_reps, cand, stream=None):
         c, H = self.cfg, self.cfg.heads
         ncand = len(cand)
-        if ncand:
-            cs = self._ints([[s for s, _ in cand]] * H).view(H, ncand)
-            cg = self._ints([[g for _, g in cand]] * H).view(H, ncand)
-        else:
-            cs = cg = None
+        cs, cg = self._list_pair(cand) if ncand else (None, None)
         L.pbsa_memory_update(self.geom, q_reps, q_reps.shape[1], self.k_reps, self.k_pool, self.v_pool,
                              self.pool_slots, self.slot_gid, self.slot_ema, c.capacity, c.bpf, cs, cg,
                              ncand, c.gamma, self.p_list, self.p_cnt, ws=self.ws, stream=stream)
