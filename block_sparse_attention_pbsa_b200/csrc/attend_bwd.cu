@@ -211,9 +211,12 @@ __device__ int merge_pair(const int* la, int cA, const int* lb, int cB, int* msl
 }
 
 // ---------------------------------------------------------------------------- 4. dQ
-// smem: Q | dO (2 panels x [128 rows][128 B] each) | K ring (2) | V ring (2) | barriers | lists
-constexpr uint32_t Q_SM_Q = 0, Q_SM_DO = 32768, Q_SM_K = 65536, Q_SM_V = Q_SM_K + 2 * 32768;
-constexpr uint32_t Q_SM_BAR = Q_SM_V + 2 * 32768;
+// smem: Q | dO (2 panels x [128 rows][128 B] each) | K ring (3) | V (1) | barriers | lists.
+// K(i) is read by S(i) and again by dQ(i) (the B operand), so its ring is the deeper one;
+// V(i) is free as soon as dP(i) is done.
+constexpr int QK_STAGES = 3;
+constexpr uint32_t Q_SM_Q = 0, Q_SM_DO = 32768, Q_SM_K = 65536, Q_SM_V = Q_SM_K + QK_STAGES * 32768;
+constexpr uint32_t Q_SM_BAR = Q_SM_V + 32768;
 constexpr uint32_t Q_SM_MISC = Q_SM_BAR + 256;
 constexpr uint32_t Q_SM_SLOT = Q_SM_MISC + 64;
 constexpr uint32_t Q_SM_FLAG = Q_SM_SLOT + 4 * 1024;
@@ -221,8 +224,10 @@ constexpr uint32_t Q_SM_LA = Q_SM_FLAG + 1024;
 constexpr uint32_t Q_SM_LB = Q_SM_LA + 4 * 512;
 constexpr uint32_t Q_SM_ONLYB = Q_SM_LB + 4 * 512;
 constexpr uint32_t Q_SMEM_BYTES = Q_SM_ONLYB + 512 + 1024;
-enum { QB_QFULL = 0, QB_KFULL = 1, QB_KEMPTY = 3, QB_VFULL = 5, QB_VEMPTY = 7, QB_SFULL = 9,
-       QB_PFULL = 11 /* [w][i&1] */, QB_MMADONE = 15, QB_NUM = 16 };
+enum { QB_QFULL = 0, QB_KFULL = 1, QB_KEMPTY = QB_KFULL + QK_STAGES, QB_VFULL = QB_KEMPTY + QK_STAGES,
+       QB_VEMPTY = QB_VFULL + 1, QB_SFULL = QB_VEMPTY + 1 /* [i&1] */,
+       QB_PFULL = QB_SFULL + 2 /* [w][i&1], 128 arrivals */, QB_DPFREE = QB_PFULL + 4 /* 256 arrivals */,
+       QB_MMADONE = QB_DPFREE + 1, QB_NUM = QB_MMADONE + 1 };
 
 struct DqParams {
   BwdGeo g;
@@ -258,6 +263,7 @@ __global__ void __launch_bounds__(NT, 1)
   if (tid == 0) {
     for (int i = 0; i < QB_NUM; ++i) mbar_init(&bars[i], 1);
     for (int i = 0; i < 4; ++i) mbar_init(&bars[QB_PFULL + i], 128);
+    mbar_init(&bars[QB_DPFREE], 256);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -291,12 +297,19 @@ __global__ void __launch_bounds__(NT, 1)
 
   if (warp < 4) {
     setmaxnreg_dec<REG_CTRL>();
+    auto load_pair = [&](const CUtensorMap* map, uint8_t* dst, uint64_t* bar, int i) {
+      for (int b = 0; b < 2; ++b) {
+        const int e = 2 * i + b;
+        const int slot = e < n ? mslot[e] : -1;
+        const int row0 = slot >= 0 ? (h * g.pool_slots + slot) * 64 : prm.kv_rows;
+        for (int p = 0; p < 2; ++p) tma_load_2d(dst + p * 16384 + b * 8192, map, bar, p * 64, row0);
+      }
+    };
     if (warp == 0 && lane == 0 && nsteps > 0) {
-      // ---- producer: Q and dO once, then K, V of each step
+      // ---- producer: Q and dO once, then the K ring
       tma_prefetch_desc(&qmap);
       tma_prefetch_desc(&domap);
       tma_prefetch_desc(&kmap);
-      tma_prefetch_desc(&vmap);
       mbar_arrive_expect_tx(&bars[QB_QFULL], 65536);
       for (int half = 0; half < 2; ++half) {
         const int r = (half == 1 && hasB) ? rB : rA;
@@ -307,82 +320,94 @@ __global__ void __launch_bounds__(NT, 1)
           tma_load_5d(sm + Q_SM_DO + p * 16384 + half * 8192, &domap, &bars[QB_QFULL], p * 64, h, tx * g.tw, ty * g.th, f);
         }
       }
-      auto load_pair = [&](const CUtensorMap* map, uint8_t* dst, uint64_t* bar, int i) {
-        for (int b = 0; b < 2; ++b) {
-          const int e = 2 * i + b;
-          const int slot = e < n ? mslot[e] : -1;
-          const int row0 = slot >= 0 ? (h * g.pool_slots + slot) * 64 : prm.kv_rows;
-          for (int p = 0; p < 2; ++p) tma_load_2d(dst + p * 16384 + b * 8192, map, bar, p * 64, row0);
-        }
-      };
-      int kiss = 0, viss = 0;
+      int kiss = 0;
       for (int i = 0; i < nsteps; ++i) {
-        const int s = i & 1;
-        wait_or_abort(&bars[QB_KEMPTY + s], ((i >> 1) & 1) ^ 1, abort_flag, prm.ws, 1, K_BWD_Q);
+        const int s = i % QK_STAGES;
+        wait_or_abort(&bars[QB_KEMPTY + s], ((i / QK_STAGES) & 1) ^ 1, abort_flag, prm.ws, 1, K_BWD_Q);
         if (*abort_flag) break;
         mbar_arrive_expect_tx(&bars[QB_KFULL + s], 32768);
         load_pair(&kmap, sm + Q_SM_K + s * 32768, &bars[QB_KFULL + s], i);
         kiss = i + 1;
-        wait_or_abort(&bars[QB_VEMPTY + s], ((i >> 1) & 1) ^ 1, abort_flag, prm.ws, 2, K_BWD_Q);
-        if (*abort_flag) break;
-        mbar_arrive_expect_tx(&bars[QB_VFULL + s], 32768);
-        load_pair(&vmap, sm + Q_SM_V + s * 32768, &bars[QB_VFULL + s], i);
-        viss = i + 1;
       }
       if (*abort_flag) {
         mbar_wait(&bars[QB_QFULL], 0, kWaitLimitNs);
-        for (int i = (kiss > 2 ? kiss - 2 : 0); i < kiss; ++i) mbar_wait(&bars[QB_KFULL + (i & 1)], (i >> 1) & 1, kWaitLimitNs);
-        for (int i = (viss > 2 ? viss - 2 : 0); i < viss; ++i) mbar_wait(&bars[QB_VFULL + (i & 1)], (i >> 1) & 1, kWaitLimitNs);
+        for (int i = (kiss > QK_STAGES ? kiss - QK_STAGES : 0); i < kiss; ++i)
+          mbar_wait(&bars[QB_KFULL + i % QK_STAGES], (i / QK_STAGES) & 1, kWaitLimitNs);
       }
+    }
+    if (warp == 2 && lane == 0 && nsteps > 0) {
+      // ---- producer: V of each step (one stage)
+      tma_prefetch_desc(&vmap);
+      int viss = 0;
+      for (int i = 0; i < nsteps; ++i) {
+        wait_or_abort(&bars[QB_VEMPTY], (i & 1) ^ 1, abort_flag, prm.ws, 2, K_BWD_Q);
+        if (*abort_flag) break;
+        mbar_arrive_expect_tx(&bars[QB_VFULL], 32768);
+        load_pair(&vmap, sm + Q_SM_V, &bars[QB_VFULL], i);
+        viss = i + 1;
+      }
+      if (*abort_flag && viss > 0) mbar_wait(&bars[QB_VFULL], (viss - 1) & 1, kWaitLimitNs);
     }
     if (warp == 1 && lane == 0 && nsteps > 0) {
       // ---- MMA issuer.  TMEM: S[i&1] at 128*(i&1), dP at 256, dQ at 384.
-      const uint32_t q_base = smem_u32(sm + Q_SM_Q), do_base = smem_u32(sm + Q_SM_DO);
-      const uint32_t k_base = smem_u32(sm + Q_SM_K), v_base = smem_u32(sm + Q_SM_V);
-      auto issue_dq = [&](int j) {
-        const int s = j & 1;
-        for (int w = 0; w < 2; ++w) {
-          wait_or_abort(&bars[QB_PFULL + 2 * w + (j & 1)], (j >> 1) & 1, abort_flag, prm.ws, 3, K_BWD_Q);
-          if (*abort_flag) return;
-          tc_fence_after();
+      // Per step: the next S and, as soon as the warpgroups have read dP(i) into registers,
+      // the next dP; then dQ += dS(i) K(i) once dS(i) is in TMEM.  So the tensor pipe computes
+      // S(i+1) and dP(i+1) while the warpgroups form dS(i).
+      const uint64_t dq_ = sw128_desc(smem_u32(sm + Q_SM_Q), 16, 1024);
+      const uint64_t ddo = sw128_desc(smem_u32(sm + Q_SM_DO), 16, 1024);
+      const uint64_t dk = sw128_desc(smem_u32(sm + Q_SM_K), 16, 1024);
+      const uint64_t dv = sw128_desc(smem_u32(sm + Q_SM_V), 16, 1024);
+      const uint64_t dk_mn = sw128_desc(smem_u32(sm + Q_SM_K), 16384, 1024);
+      auto issue_s = [&](int i) {   // S(i) = Q K(i)^T into S[i&1]
+        const int sk = i % QK_STAGES;
+        wait_or_abort(&bars[QB_KFULL + sk], (i / QK_STAGES) & 1, abort_flag, prm.ws, 5, K_BWD_Q);
+        if (*abort_flag) return;
+        tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t b = sw128_desc(k_base + s * 32768 + w * 8192 + kk * 2048, 16384, 1024);
-            mma_bf16_ts(tmem + 384, tmem + (j & 1) * 128 + w * 64 + kk * 8, b, IDESC_BMN,
-                        (j > 0 || w > 0 || kk > 0) ? 1u : 0u);
-          }
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+          mma_bf16_ss(tmem + (i & 1) * 128, dq_ + off, dk + ((sk * 32768) >> 4) + off, IDESC_KMAJ,
+                      kk > 0 ? 1u : 0u);
         }
-        mma_commit(&bars[QB_KEMPTY + s]);
+      };
+      auto issue_dp = [&](int i) {  // dP(i) = dO V(i)^T, then V's stage is free
+        wait_or_abort(&bars[QB_VFULL], i & 1, abort_flag, prm.ws, 6, K_BWD_Q);
+        if (*abort_flag) return;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+          mma_bf16_ss(tmem + 256, ddo + off, dv + off, IDESC_KMAJ, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&bars[QB_VEMPTY]);
       };
       wait_or_abort(&bars[QB_QFULL], 0, abort_flag, prm.ws, 4, K_BWD_Q);
+      issue_s(0);
+      issue_dp(0);
+      mma_commit(&bars[QB_SFULL + 0]);
       for (int i = 0; i < nsteps && !*abort_flag; ++i) {
-        const int s = i & 1;
-        wait_or_abort(&bars[QB_KFULL + s], (i >> 1) & 1, abort_flag, prm.ws, 5, K_BWD_Q);
-        if (*abort_flag) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t a = sw128_desc(q_base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-          const uint64_t b = sw128_desc(k_base + s * 32768 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-          mma_bf16_ss(tmem + (i & 1) * 128, a, b, IDESC_KMAJ, kk > 0 ? 1u : 0u);
+        const int s = i & 1, sk = i % QK_STAGES;
+        if (i + 1 < nsteps) {
+          issue_s(i + 1);
+          wait_or_abort(&bars[QB_DPFREE], i & 1, abort_flag, prm.ws, 9, K_BWD_Q);
+          issue_dp(i + 1);
+          mma_commit(&bars[QB_SFULL + ((i + 1) & 1)]);
+          if (*abort_flag) break;
         }
-        // dS(i-1) has been consumed by the softmax side once its P-full arrives; that also
-        // frees the single dP buffer for dP(i)
-        if (i >= 1) issue_dq(i - 1);
-        if (*abort_flag) break;
-        wait_or_abort(&bars[QB_VFULL + s], (i >> 1) & 1, abort_flag, prm.ws, 6, K_BWD_Q);
-        if (*abort_flag) break;
-        tc_fence_after();
+        // dQ += dS(i) K(i): dS(i) (bf16 pairs) sits over S[s], warpgroup w's 64 keys in its
+        // half; K(i) is the B operand (keys x d, d contiguous)
+        for (int w = 0; w < 2; ++w) {
+          wait_or_abort(&bars[QB_PFULL + 2 * w + s], (i >> 1) & 1, abort_flag, prm.ws, 3, K_BWD_Q);
+          if (*abort_flag) break;
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t a = sw128_desc(do_base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-          const uint64_t b = sw128_desc(v_base + s * 32768 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-          mma_bf16_ss(tmem + 256, a, b, IDESC_KMAJ, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16_ts(tmem + 384, tmem + s * 128 + w * 64 + kk * 8,
+                        dk_mn + ((sk * 32768 + w * 8192 + kk * 2048) >> 4), IDESC_BMN,
+                        (i > 0 || w > 0 || kk > 0) ? 1u : 0u);
         }
-        mma_commit(&bars[QB_SFULL + (i & 1)]);
-        mma_commit(&bars[QB_VEMPTY + s]);
+        mma_commit(&bars[QB_KEMPTY + sk]);
       }
-      if (!*abort_flag) issue_dq(nsteps - 1);
       mma_commit(&bars[QB_MMADONE]);
       mbar_wait(&bars[QB_MMADONE], 0, kWaitLimitNs);
     }
@@ -406,26 +431,29 @@ __global__ void __launch_bounds__(NT, 1)
       wait_or_abort(&bars[QB_SFULL + (i & 1)], (i >> 1) & 1, abort_flag, prm.ws, 7, K_BWD_Q);
       if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
       tc_fence_after();
+      // every column holds a finite value (a block that does not exist was loaded as
+      // zeros), so all are read and masking is arithmetic
       uint32_t xs[2][32], xp[2][32];
-      if (__any_sync(0xffffffffu, v)) {
-        tmem_ld32(tS, xs[0]);
-        tmem_ld32(tS + 32, xs[1]);
-        tmem_ld32(tP, xp[0]);
-        tmem_ld32(tP + 32, xp[1]);
-        tmem_wait_ld();
-      }
+      tmem_ld32(tS, xs[0]);
+      tmem_ld32(tS + 32, xs[1]);
+      tmem_ld32(tP, xp[0]);
+      tmem_ld32(tP + 32, xp[1]);
+      tmem_wait_ld();
+      // dP(i) is in registers: the issuer may overwrite its TMEM with dP(i+1)
+      tc_fence_before();
+      mbar_arrive(&bars[QB_DPFREE]);
+      // dS = P * (dP - D), P = 2^(s*c - lse2); a masked block uses the factor 0 and the offset
+      // -inf, so P (and dS) are exact zeros without a branch
+      const float cs = v ? c : 0.f, ms = v ? -lse2 : -INFINITY;
       uint32_t pk[32];
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
 #pragma unroll
         for (int e2 = 0; e2 < 16; ++e2) {
-          float d0 = 0.f, d1 = 0.f;
-          if (v) {
-            const float p0 = ex2_approx(fmaf(__uint_as_float(xs[q][2 * e2]), c, -lse2));
-            const float p1 = ex2_approx(fmaf(__uint_as_float(xs[q][2 * e2 + 1]), c, -lse2));
-            d0 = p0 * (__uint_as_float(xp[q][2 * e2]) - dd);
-            d1 = p1 * (__uint_as_float(xp[q][2 * e2 + 1]) - dd);
-          }
+          float a0, a1, t0, t1, d0, d1;
+          ffma2(__uint_as_float(xs[q][2 * e2]), __uint_as_float(xs[q][2 * e2 + 1]), cs, ms, a0, a1);
+          ffma2(__uint_as_float(xp[q][2 * e2]), __uint_as_float(xp[q][2 * e2 + 1]), 1.f, -dd, t0, t1);
+          fmul2(ex2_approx(a0), ex2_approx(a1), t0, t1, d0, d1);
           pk[q * 16 + e2] = pack_bf16(d0, d1);
         }
       }
@@ -472,12 +500,14 @@ __global__ void __launch_bounds__(NT, 1)
 
 
 // ---------------------------------------------------------------------------- 5. dK, dV
-// smem: K pair | V pair (2 panels x [128 keys][128 B] each) | 2 stages x (Q, dO tiles of two
-// query blocks, their log2-LSE and D rows) | barriers | lists
-constexpr uint32_t KV_SM_K = 0, KV_SM_V = 32768, KV_SM_Q = 65536;    // Q stage s at +65536*s
-constexpr uint32_t KV_STAGE = 65536;                                 // Q (32 KB) + dO (32 KB)
-constexpr uint32_t KV_SM_VEC = KV_SM_Q + 2 * KV_STAGE;               // 2 stages x [lse2 | D] x 2 blocks x 64 f32
-constexpr uint32_t KV_SM_BAR = KV_SM_VEC + 2 * 1024;
+// smem: K pair | V pair (2 panels x [128 keys][128 B] each) | KV_QST stages x (Q, dO tiles of one
+// query block: 2 panels x [64 rows][128 B] each) | KV_QST x [log2-LSE | D] x 64 f32 | barriers |
+// lists
+constexpr int KV_QST = 4;                                            // query-block stages
+constexpr uint32_t KV_SM_K = 0, KV_SM_V = 32768, KV_SM_Q = 65536;    // Q stage s at +KV_STAGE*s
+constexpr uint32_t KV_STAGE = 32768;                                 // Q (16 KB) + dO (16 KB)
+constexpr uint32_t KV_SM_VEC = KV_SM_Q + KV_QST * KV_STAGE;          // [stage][lse2 | D][64] f32
+constexpr uint32_t KV_SM_BAR = KV_SM_VEC + KV_QST * 512;
 constexpr uint32_t KV_SM_MISC = KV_SM_BAR + 256;
 constexpr uint32_t KV_SM_SLOT = KV_SM_MISC + 64;
 constexpr uint32_t KV_SM_FLAG = KV_SM_SLOT + 4 * 1024;
@@ -486,8 +516,9 @@ constexpr uint32_t KV_SM_LB = KV_SM_LA + 4 * 512;
 constexpr uint32_t KV_SM_ONLYB = KV_SM_LB + 4 * 512;
 constexpr uint32_t KV_SM_TMP = KV_SM_ONLYB + 512;                    // int[512] sort scratch
 constexpr uint32_t KV_SMEM_BYTES = KV_SM_TMP + 4 * 512 + 1024;
-enum { KB_KVFULL = 0, KB_QFULL = 1, KB_QEMPTY = 3, KB_SFULL = 5, KB_PFULL = 6 /* [w] */,
-       KB_MMADONE = 8, KB_NUM = 9 };
+enum { KB_KVFULL = 0, KB_QFULL = 1, KB_QEMPTY = KB_QFULL + KV_QST, KB_SFULL = KB_QEMPTY + KV_QST /* [b] */,
+       KB_PFULL = KB_SFULL + 2 /* [b], 128 arrivals */, KB_MMADONE = KB_PFULL + 2, KB_NUM = KB_MMADONE + 1 };
+constexpr uint32_t IDESC_N64 = idesc_bf16_f32(128, 64, 0, 0);   // S^T, dP^T of one query block
 
 struct DkvParams {
   BwdGeo g;
@@ -572,13 +603,14 @@ __global__ void __launch_bounds__(NT, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const int nsteps = (n + 1) >> 1;
-  float* vecs = reinterpret_cast<float*>(sm + KV_SM_VEC);  // [stage][lse2 blk0, lse2 blk1, D blk0, D blk1][64]
+  // one step per merged query block j; warpgroup (j & 1) forms P^T and dS^T of step j
+  const int nsteps = n;
+  float* vecs = reinterpret_cast<float*>(sm + KV_SM_VEC);  // [stage][lse2 | D][64]
 
   if (warp < 4) {
     setmaxnreg_dec<REG_CTRL>();
     if (warp == 0 && lane == 0 && nsteps > 0) {
-      // ---- producer: the K, V pair once; then Q, dO, log2-LSE, D of two query blocks per step
+      // ---- producer: the K, V pair once; then Q, dO, log2-LSE, D of one query block per step
       tma_prefetch_desc(&qmap);
       tma_prefetch_desc(&domap);
       tma_prefetch_desc(&kmap);
@@ -592,68 +624,72 @@ __global__ void __launch_bounds__(NT, 1)
         }
       }
       int iss = 0;
-      for (int i = 0; i < nsteps; ++i) {
-        const int s = i & 1;
-        wait_or_abort(&bars[KB_QEMPTY + s], ((i >> 1) & 1) ^ 1, abort_flag, prm.ws, 1, K_BWD_KV);
+      for (int j = 0; j < nsteps; ++j) {
+        const int s = j % KV_QST;
+        wait_or_abort(&bars[KB_QEMPTY + s], ((j / KV_QST) & 1) ^ 1, abort_flag, prm.ws, 1, K_BWD_KV);
         if (*abort_flag) break;
-        mbar_arrive_expect_tx(&bars[KB_QFULL + s], KV_STAGE + 4 * 256);
+        mbar_arrive_expect_tx(&bars[KB_QFULL + s], KV_STAGE + 512);
         uint8_t* qdst = sm + KV_SM_Q + s * KV_STAGE;
-        float* vdst = vecs + s * 256;
-        for (int b = 0; b < 2; ++b) {
-          const int e = 2 * i + b;
-          const bool real = e < n;
-          const int r = real ? mslot[e] : mslot[2 * i];
-          const int f = real ? r / g.bpf : prm.q_frames;   // a missing block is loaded out of bounds
-          const int rem = r - (r / g.bpf) * g.bpf;
-          const int ty = rem / g.tpr, tx = rem - ty * g.tpr;
-          for (int p = 0; p < 2; ++p) {
-            tma_load_5d(qdst + p * 16384 + b * 8192, &qmap, &bars[KB_QFULL + s], p * 64, h, tx * g.tw, ty * g.th, f);
-            tma_load_5d(qdst + 32768 + p * 16384 + b * 8192, &domap, &bars[KB_QFULL + s], p * 64, h, tx * g.tw,
-                        ty * g.th, f);
-          }
-          const size_t bi = ((size_t)h * g.nq + r) * BT;
-          bulk_load(vdst + b * 64, prm.lvec + bi, 256, &bars[KB_QFULL + s]);
-          bulk_load(vdst + 128 + b * 64, prm.dvec + bi, 256, &bars[KB_QFULL + s]);
+        const int r = mslot[j];
+        const int f = r / g.bpf, rem = r - f * g.bpf;
+        const int ty = rem / g.tpr, tx = rem - ty * g.tpr;
+        for (int p = 0; p < 2; ++p) {
+          tma_load_5d(qdst + p * 8192, &qmap, &bars[KB_QFULL + s], p * 64, h, tx * g.tw, ty * g.th, f);
+          tma_load_5d(qdst + 16384 + p * 8192, &domap, &bars[KB_QFULL + s], p * 64, h, tx * g.tw, ty * g.th, f);
         }
-        iss = i + 1;
+        const size_t bi = ((size_t)h * g.nq + r) * BT;
+        bulk_load(vecs + s * 128, prm.lvec + bi, 256, &bars[KB_QFULL + s]);
+        bulk_load(vecs + s * 128 + 64, prm.dvec + bi, 256, &bars[KB_QFULL + s]);
+        iss = j + 1;
       }
       if (*abort_flag) {
         mbar_wait(&bars[KB_KVFULL], 0, kWaitLimitNs);
-        for (int i = (iss > 2 ? iss - 2 : 0); i < iss; ++i) mbar_wait(&bars[KB_QFULL + (i & 1)], (i >> 1) & 1, kWaitLimitNs);
+        for (int j = (iss > KV_QST ? iss - KV_QST : 0); j < iss; ++j)
+          mbar_wait(&bars[KB_QFULL + j % KV_QST], (j / KV_QST) & 1, kWaitLimitNs);
       }
     }
     if (warp == 1 && lane == 0 && nsteps > 0) {
-      // ---- MMA issuer.  TMEM: S^T at 0, dP^T at 128, dV at 256, dK at 384 (keys on lanes).
-      const uint32_t k_base = smem_u32(sm + KV_SM_K), v_base = smem_u32(sm + KV_SM_V);
+      // ---- MMA issuer (one thread, so dV and dK accumulate in a fixed order).
+      // TMEM: S^T[b] at 64 b, dP^T[b] at 128 + 64 b (keys on lanes, 64 queries each), dV at 256,
+      // dK at 384.  Step j uses buffer b = j & 1; S^T/dP^T(j+2) go into it right behind the
+      // dV/dK MMAs of step j, while the other warpgroup works on step j+1.
+      const uint64_t dk = sw128_desc(smem_u32(sm + KV_SM_K), 16, 1024);
+      const uint64_t dv = sw128_desc(smem_u32(sm + KV_SM_V), 16, 1024);
+      auto issue_sdp = [&](int j) {   // S^T = K Q_j^T, dP^T = V dO_j^T (M = 128 keys, N = 64)
+        const int s = j % KV_QST, b = j & 1;
+        wait_or_abort(&bars[KB_QFULL + s], (j / KV_QST) & 1, abort_flag, prm.ws, 3, K_BWD_KV);
+        if (*abort_flag) return;
+        tc_fence_after();
+        const uint64_t dq_ = sw128_desc(smem_u32(sm + KV_SM_Q + s * KV_STAGE), 16, 1024);
+        const uint64_t ddo = sw128_desc(smem_u32(sm + KV_SM_Q + s * KV_STAGE + 16384), 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t ka = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;   // K/V: 128-row panels
+          const uint32_t kb = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;    // Q/dO: 64-row panels
+          mma_bf16_ss(tmem + b * 64, dk + ka, dq_ + kb, IDESC_N64, kk > 0 ? 1u : 0u);
+          mma_bf16_ss(tmem + 128 + b * 64, dv + ka, ddo + kb, IDESC_N64, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&bars[KB_SFULL + b]);
+      };
       wait_or_abort(&bars[KB_KVFULL], 0, abort_flag, prm.ws, 2, K_BWD_KV);
-      for (int i = 0; i < nsteps && !*abort_flag; ++i) {
-        const int s = i & 1;
-        const uint32_t q_base = smem_u32(sm + KV_SM_Q + s * KV_STAGE), do_base = q_base + 32768;
-        wait_or_abort(&bars[KB_QFULL + s], (i >> 1) & 1, abort_flag, prm.ws, 3, K_BWD_KV);
+      issue_sdp(0);
+      if (nsteps > 1) issue_sdp(1);
+      for (int j = 0; j < nsteps && !*abort_flag; ++j) {
+        const int s = j % KV_QST, b = j & 1;
+        wait_or_abort(&bars[KB_PFULL + b], (j >> 1) & 1, abort_flag, prm.ws, 4, K_BWD_KV);
         if (*abort_flag) break;
         tc_fence_after();
+        // dV += P^T dO_j, dK += dS^T Q_j: A from TMEM (bf16 pairs over S^T[b] / dP^T[b]), B =
+        // the query block's 64 rows (d contiguous, two 64-column panels 8 KB apart)
+        const uint32_t q_base = smem_u32(sm + KV_SM_Q + s * KV_STAGE), do_base = q_base + 16384;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {   // S^T = K Q^T and dP^T = V dO^T (M = 128 keys, N = 128 queries)
-          const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_bf16_ss(tmem + 0, sw128_desc(k_base + ko, 16, 1024), sw128_desc(q_base + ko, 16, 1024),
-                      IDESC_KMAJ, kk > 0 ? 1u : 0u);
-          mma_bf16_ss(tmem + 128, sw128_desc(v_base + ko, 16, 1024), sw128_desc(do_base + ko, 16, 1024),
-                      IDESC_KMAJ, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(&bars[KB_SFULL]);
-        for (int w = 0; w < 2; ++w) {
-          wait_or_abort(&bars[KB_PFULL + w], i & 1, abort_flag, prm.ws, 4, K_BWD_KV);
-          if (*abort_flag) break;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {   // dV += P^T dO_w, dK += dS^T Q_w (queries of block w)
-            const uint32_t bo = w * 8192 + kk * 2048;
-            const uint32_t acc = (i > 0 || w > 0 || kk > 0) ? 1u : 0u;
-            mma_bf16_ts(tmem + 256, tmem + 0 + w * 64 + kk * 8, sw128_desc(do_base + bo, 16384, 1024), IDESC_BMN, acc);
-            mma_bf16_ts(tmem + 384, tmem + 128 + w * 64 + kk * 8, sw128_desc(q_base + bo, 16384, 1024), IDESC_BMN, acc);
-          }
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
+          mma_bf16_ts(tmem + 256, tmem + b * 64 + kk * 8, sw128_desc(do_base + kk * 2048, 8192, 1024), IDESC_BMN, acc);
+          mma_bf16_ts(tmem + 384, tmem + 128 + b * 64 + kk * 8, sw128_desc(q_base + kk * 2048, 8192, 1024), IDESC_BMN, acc);
         }
         mma_commit(&bars[KB_QEMPTY + s]);
+        if (j + 2 < nsteps) issue_sdp(j + 2);
       }
       mma_commit(&bars[KB_MMADONE]);
       mbar_wait(&bars[KB_MMADONE], 0, kWaitLimitNs);
@@ -661,44 +697,44 @@ __global__ void __launch_bounds__(NT, 1)
     __syncwarp();
   } else {
     setmaxnreg_inc<REG_WORK>();
-    // ---- P^T and dS^T for the query block of the step this warpgroup owns; lanes are keys
+    // ---- P^T and dS^T of the steps j = wg (mod 2); lanes are keys
     const int wg = (warp - 4) >> 2, wq = warp & 3;
     const int row = wq * 32 + lane, kh = row >> 6;   // key row, which slot of the pair
     const bool row_valid = kh == 0 || hasB;
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const float c = prm.scale_log2;
-    for (int i = 0; i < nsteps; ++i) {
-      const int e = 2 * i + wg;
-      const bool v = row_valid && e < n && ((mflag[e] >> kh) & 1);
-      const uint32_t tS = tmem + lane_off + wg * 64, tD = tmem + lane_off + 128 + wg * 64;
-      const float* lse2 = vecs + (i & 1) * 256 + wg * 64;
-      const float* dd = vecs + (i & 1) * 256 + 128 + wg * 64;
+    const uint32_t tS = tmem + lane_off + wg * 64, tD = tmem + lane_off + 128 + wg * 64;
+    for (int j = wg; j < nsteps; j += 2) {
+      const bool v = row_valid && ((mflag[j] >> kh) & 1);
+      const float* lse2 = vecs + (j % KV_QST) * 128;
+      const float* dd = lse2 + 64;
       // the step's log2-LSE / D rows arrived with its Q-full barrier (TMA bulk copies)
-      wait_or_abort(&bars[KB_QFULL + (i & 1)], (i >> 1) & 1, abort_flag, prm.ws, 7, K_BWD_KV);
-      wait_or_abort(&bars[KB_SFULL], i & 1, abort_flag, prm.ws, 5, K_BWD_KV);
+      wait_or_abort(&bars[KB_QFULL + j % KV_QST], (j / KV_QST) & 1, abort_flag, prm.ws, 7, K_BWD_KV);
+      wait_or_abort(&bars[KB_SFULL + wg], (j >> 1) & 1, abort_flag, prm.ws, 5, K_BWD_KV);
       if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
       tc_fence_after();
+      // every column is finite (a missing block was loaded as zeros): read all, mask arithmetically
       uint32_t xs[2][32], xp[2][32];
-      if (__any_sync(0xffffffffu, v)) {
-        tmem_ld32(tS, xs[0]);
-        tmem_ld32(tS + 32, xs[1]);
-        tmem_ld32(tD, xp[0]);
-        tmem_ld32(tD + 32, xp[1]);
-        tmem_wait_ld();
-      }
+      tmem_ld32(tS, xs[0]);
+      tmem_ld32(tS + 32, xs[1]);
+      tmem_ld32(tD, xp[0]);
+      tmem_ld32(tD + 32, xp[1]);
+      tmem_wait_ld();
+      const float cs = v ? c : 0.f;
       uint32_t pp[32], pd[32];
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
 #pragma unroll
         for (int e2 = 0; e2 < 16; ++e2) {
           const int c0 = q * 32 + 2 * e2;
-          float p0 = 0.f, p1 = 0.f, d0 = 0.f, d1 = 0.f;
-          if (v) {
-            p0 = ex2_approx(fmaf(__uint_as_float(xs[q][2 * e2]), c, -lse2[c0]));
-            p1 = ex2_approx(fmaf(__uint_as_float(xs[q][2 * e2 + 1]), c, -lse2[c0 + 1]));
-            d0 = p0 * (__uint_as_float(xp[q][2 * e2]) - dd[c0]);
-            d1 = p1 * (__uint_as_float(xp[q][2 * e2 + 1]) - dd[c0 + 1]);
-          }
+          const float m0 = v ? -lse2[c0] : -INFINITY, m1 = v ? -lse2[c0 + 1] : -INFINITY;
+          float a0, a1, t0, t1, d0, d1;
+          a0 = fmaf(__uint_as_float(xs[q][2 * e2]), cs, m0);
+          a1 = fmaf(__uint_as_float(xs[q][2 * e2 + 1]), cs, m1);
+          const float p0 = ex2_approx(a0), p1 = ex2_approx(a1);
+          t0 = __uint_as_float(xp[q][2 * e2]) - dd[c0];
+          t1 = __uint_as_float(xp[q][2 * e2 + 1]) - dd[c0 + 1];
+          fmul2(p0, p1, t0, t1, d0, d1);
           pp[q * 16 + e2] = pack_bf16(p0, p1);
           pd[q * 16 + e2] = pack_bf16(d0, d1);
         }

@@ -87,26 +87,6 @@ struct Params {
   void* ws;
 };
 
-// ---------------------------------------------------------------- softmax arithmetic
-// Two fp32 lanes per instruction (sm_100 packed f32x2): a = x * c + m.
-__device__ __forceinline__ void ffma2(float x0, float x1, float c, float m, float& a0, float& a1) {
-  asm("{\n\t.reg .b64 x, c, m, a;\n\t"
-      "mov.b64 x, {%2, %3};\n\tmov.b64 c, {%4, %4};\n\tmov.b64 m, {%5, %5};\n\t"
-      "fma.rn.f32x2 a, x, c, m;\n\tmov.b64 {%0, %1}, a;\n\t}"
-      : "=f"(a0), "=f"(a1) : "f"(x0), "f"(x1), "f"(c), "f"(m));
-}
-// (s0, s1) += (y0, y1)
-__device__ __forceinline__ void fadd2(float& s0, float& s1, float y0, float y1) {
-  asm("{\n\t.reg .b64 s, y;\n\t"
-      "mov.b64 s, {%0, %1};\n\tmov.b64 y, {%2, %3};\n\t"
-      "add.rn.f32x2 s, s, y;\n\tmov.b64 {%0, %1}, s;\n\t}"
-      : "+f"(s0), "+f"(s1) : "f"(y0), "f"(y1));
-}
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-  float d;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-  return d;
-}
 __device__ __forceinline__ void wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                               void* ws, int where) {
   if (*abort_flag) return;
