@@ -105,6 +105,44 @@ def kth_gap(scores: np.ndarray, gids, k: int) -> float:
     return abs(float(scores[order[k - 1]]) - float(scores[order[k]]))
 
 
+# --------------------------------------------------------------------------- hierarchical selection
+def hsa_select(q_rep, cand_reps, cand_gids, bpf: int, top_frames: int, n_recent: int, k: int,
+               scale: float):
+    """Two-level (frame, then block) choice of the local blocks one query block attends.
+
+    The hierarchical sparse attention of *Light Forcing* (papernotes.org notes, "方法详解",
+    HSA, steps (1)-(3)), used as the selection policy over PBSA's local window:
+      1. token compression: a frame's representative is the mean of its tokens, i.e. the mean
+         of its block representatives (every block holds the same number of tokens);
+      2. frame level: p(t) = scale * <qbar, frame rep of t>; the chosen frames are the
+         always-on ones (here the ``n_recent`` latest candidate frames: the sinks already sit in
+         the persistent memory, and the current chunk is not attended at inference) plus the
+         ``top_frames`` best other frames (score descending, the earlier frame on ties);
+      3. block level: o(b) = scale * <qbar, kbar_b> over the blocks of the chosen frames, the
+         ``k`` best (score descending, the lower gid on ties).
+    Candidates come in whole frames: candidate c belongs to frame slot c // bpf, frame slots in
+    time order.  Returns (candidate positions best first, frame-level gap, block-level gap); a
+    gap is |score at the cut - score just past it| (inf when nothing is cut).
+    """
+    reps = np.asarray(cand_reps, np.float64)
+    q = np.asarray(q_rep, np.float64)
+    n = reps.shape[0]
+    nf = n // bpf
+    frame_rep = reps.reshape(nf, bpf, -1).mean(axis=1)
+    p = scale * (frame_rep @ q)
+    always = list(range(max(0, nf - n_recent), nf))
+    others = sorted((t for t in range(nf) if t not in always), key=lambda t: (-float(p[t]), t))
+    chosen = set(always) | set(others[:max(0, top_frames)])
+    frame_gap = float("inf")
+    if 0 < top_frames < len(others):
+        frame_gap = abs(float(p[others[top_frames - 1]]) - float(p[others[top_frames]]))
+    elig = [c for c in range(n) if c // bpf in chosen]
+    o = scale * (reps[elig] @ q)
+    gids = [int(cand_gids[c]) for c in elig]
+    pos = topk_select(o, gids, k)
+    return [elig[i] for i in pos], frame_gap, kth_gap(o, gids, k)
+
+
 # --------------------------------------------------------------------------- a3: fine attention
 def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float):
     """Softmax attention of query rows over key/value rows; returns (out [n, d], lse [n]).

@@ -245,3 +245,56 @@ def test_train_masks_shape():
     assert len(m[12]) == 4 + 2 + 12 and set(m[12][:4]) == set(range(4))
     assert set(m[12][4:6]) <= set(range(4, 12))
     assert set(m[30][4:6]) <= set(range(4, 24))
+
+
+# ------------------------------------------------------------------ hierarchical (frame -> block) selection
+def test_hsa_frames_ranked_by_mean_not_by_best_block():
+    """Hand-built case: frame 0 holds the single best block but the lowest mean, frame 1 the
+    best mean; frame 2 is the always-on latest frame.  With one extra frame the selection is
+    frame 1's blocks then frame 2's, and frame 0's best block is left out."""
+    bpf, scale = 2, 1.0
+    q = np.array([1.0, 0.0])
+    block_score = [10.0, -9.0, 2.0, 2.0, 0.0, 0.0]     # frame means 0.5, 2.0, 0.0
+    reps = np.array([[s, 7.0] for s in block_score])
+    gids = [100, 101, 102, 103, 104, 105]
+    pos, fgap, bgap = O.hsa_select(q, reps, gids, bpf, top_frames=1, n_recent=1, k=3, scale=scale)
+    assert pos == [2, 3, 4]                 # scores 2, 2 (lower gid first), then 0 (gid 104 < 105)
+    assert fgap == pytest.approx(1.5)       # frame 1 (2.0) vs frame 0 (0.5)
+    assert bgap == 0.0                      # 4th best ties with the 3rd (0 vs 0)
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_hsa_reduces_to_flat_topk(seed):
+    """Every frame chosen (enough extra frames, or every frame always-on) is the flat top-k."""
+    rng = np.random.default_rng(seed)
+    bpf, nf, d, k = 4, 6, 8, 7
+    q = rng.normal(size=d)
+    reps = rng.normal(size=(nf * bpf, d))
+    gids = rng.permutation(1000)[:nf * bpf]
+    flat = O.topk_select(O.coarse_scores(q[None], reps, 0.3)[0], gids, k)
+    for top_frames, n_recent in [(nf, 1), (nf - 1, 1), (0, nf), (3, nf)]:
+        pos, _, _ = O.hsa_select(q, reps, gids, bpf, top_frames, n_recent, k, 0.3)
+        assert pos == flat
+
+
+def test_hsa_brute_force_small():
+    """Against an exhaustive restatement: frame sets by frame-mean score, then the best blocks."""
+    rng = np.random.default_rng(5)
+    bpf, nf, d = 3, 5, 4
+    for trial in range(20):
+        q = rng.normal(size=d)
+        reps = rng.normal(size=(nf * bpf, d))
+        gids = list(range(nf * bpf))
+        top_frames, n_recent, k = int(rng.integers(0, nf)), int(rng.integers(0, 3)), int(rng.integers(1, 8))
+        pos, _, _ = O.hsa_select(q, reps, gids, bpf, top_frames, n_recent, k, 1.0)
+        fmean = [float(np.mean([reps[t * bpf + b] @ q for b in range(bpf)])) for t in range(nf)]
+        always = set(range(max(0, nf - n_recent), nf))
+        others = [t for t in range(nf) if t not in always]
+        # the best subset of other frames of size top_frames by total mean score (ties unlikely)
+        best = max(itertools.combinations(others, min(top_frames, len(others))),
+                   key=lambda c: sum(fmean[t] for t in c), default=())
+        frames = always | set(best)
+        cands = sorted((c for c in range(nf * bpf) if c // bpf in frames), key=lambda c: -(reps[c] @ q))
+        assert pos == cands[:k]
+        # selected blocks lie in chosen frames, the latest n_recent frames are always available
+        assert all(c // bpf in frames for c in pos)
