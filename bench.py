@@ -351,6 +351,51 @@ def run_rollout(P, I, dev, w, max_chunks=None):
     }
 
 
+def run_variant(P, I, dev, w, steps: int, **cfg_changes):
+    """The chunk decode of ``run_pbsa`` under a different layer policy (e.g. the hierarchical
+    selection), on the same inputs: graph-captured, L2 flushed before each step, in-graph events."""
+    q, k, v = I.single_step(w)
+    kc = I.tokens(w, w.chunk_frames, I.stream_seed(w.seed, 4))
+    vc = I.tokens(w, w.chunk_frames, I.stream_seed(w.seed, 5))
+    bpf = w.blocks_per_frame
+    cfg = P.LayerConfig(w.heads, w.head_dim, w.frame_h, w.frame_w, w.tile_h, w.tile_w, w.capacity,
+                        w.window_frames, w.chunk_frames, w.topk, w.gamma, w.dtype,
+                        (w.hist_frames - w.window_frames) * bpf, **cfg_changes)
+    cache = P.PBSALayerCache(cfg, dev)
+    qd, kcd, vcd = q.to(dev), kc.to(dev), vc.to(dev)
+    cache.prefill(k.to(dev), v.to(dev), w.hist_frames, cache.query_reps(qd))
+    step = P.ChunkDecodeStep(cache)
+    o = torch.empty_like(qd)
+    snap = step.snapshot()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(2):
+        step.restore(snap)
+        step.run(qd, kcd, vcd, o)
+    torch.cuda.synchronize(dev)
+    marks = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(6)]
+    graph = step.capture(qd, kcd, vcd, o, marks=marks)
+    spans = {"blockify_select": (0, 2), "attend": (2, 3), "commit_blockify_kv": (3, 4), "memory_update": (4, 5)}
+    runs = {g: [] for g in spans}
+    total = []
+    for s in range(steps + 3):
+        step.restore(snap)
+        flush.fill_(1)
+        graph.replay()
+        torch.cuda.synchronize(dev)
+        if s >= 3:
+            for g, (a, b) in spans.items():
+                runs[g].append(marks[a].elapsed_time(marks[b]))
+            total.append(marks[0].elapsed_time(marks[5]))
+    _check_device(P, cache.ws, "in a variant run")
+    flops = step.flops()
+    per = {g: statistics.mean(x) for g, x in runs.items()}
+    ms = statistics.mean(total)
+    del graph
+    return {"policy": cfg_changes, "ms_per_chunk_decode": ms, "kernels_ms": per,
+            "selected_flops": flops, "value_tflops": flops / (ms * 1e-3) / 1e12,
+            "attend_tflops": flops / (per["attend"] * 1e-3) / 1e12}
+
+
 def rank_workload(w, rank: int):
     """Weak scaling: every rank decodes its own independent layer (same shapes, its own seed)."""
     import dataclasses
@@ -502,6 +547,7 @@ def run_pbsa(args, w, rank, world, local_rank):
     }
     if not args.no_train:
         line["train"] = run_train(P, I, dev, 5, peaks)
+    line["variants"] = [run_variant(P, I, dev, w, max(5, args.steps // 2), hsa_top_frames=3, hsa_recent=1)]
     if not args.no_rollout:
         line["rollouts"] = [run_rollout(P, I, dev, I.ROLLOUT_5S), run_rollout(P, I, dev, I.ROLLOUT_1MIN)]
     if world == 1 and not args.no_cpu_baseline:

@@ -38,6 +38,11 @@ class LayerConfig:
     dtype: str = "bf16"           # "bf16" or "f32"
     staging_blocks: int = 0       # extra slots for prefill (history beyond the ring)
     scale: float | None = None
+    # local selection policy: -1 = flat top-k over the window; >= 0 = two-level (hierarchical)
+    # selection: the hsa_recent latest window frames + the hsa_top_frames best other frames,
+    # then the top-k blocks of those frames
+    hsa_top_frames: int = -1
+    hsa_recent: int = 1
 
     @property
     def bpf(self) -> int:
@@ -182,11 +187,21 @@ class PBSALayerCache:
         self.q_reps = self._q_reps_buf[:c.heads * nq * c.head_dim].view(c.heads, nq, c.head_dim)
         self.kv_slot = self._kv_slot_buf[:c.heads * nq * self.kv_ld_own].view(c.heads, nq, self.kv_ld_own)
         self.kv_cnt = self._kv_cnt_buf[:c.heads * nq].view(c.heads, nq)
-        cs, cg, n = self._cand
-        L.pbsa_blockify_score_select(self.geom, q, nf, self.q_reps, self.k_reps, self.pool_slots, cs, cg, n,
-                                     c.topk if n else 0, self.p_list, self.p_cnt, c.capacity, self.kv_slot,
-                                     self.kv_cnt, self.kv_ld_own, ws=self.ws, stream=stream)
+        self._select_fused(q, nf, self.q_reps, self.kv_slot, self.kv_cnt, self.kv_ld_own, stream)
         return self.q_reps, self.kv_slot, self.kv_cnt, self.kv_ld_own
+
+    def _select_fused(self, q, nf, q_reps, kv_slot, kv_cnt, kv_ld, stream=None):
+        """The one-launch blockify + selection of the configured policy."""
+        c = self.cfg
+        cs, cg, n = self._cand
+        if c.hsa_top_frames >= 0 and n:
+            L.pbsa_blockify_hsa_select(self.geom, q, nf, q_reps, self.k_reps, self.pool_slots, cs, cg, n,
+                                       c.hsa_top_frames, c.hsa_recent, c.topk, self.p_list, self.p_cnt,
+                                       c.capacity, kv_slot, kv_cnt, kv_ld, ws=self.ws, stream=stream)
+        else:
+            L.pbsa_blockify_score_select(self.geom, q, nf, q_reps, self.k_reps, self.pool_slots, cs, cg, n,
+                                         c.topk if n else 0, self.p_list, self.p_cnt, c.capacity, kv_slot,
+                                         kv_cnt, kv_ld, ws=self.ws, stream=stream)
 
     def attend(self, q, kv_slot, kv_cnt, kv_ld, o=None, lse=None, stream=None):
         """a3: fine attention over the listed slots."""
@@ -308,7 +323,7 @@ class ChunkDecodeStep:
     """One chunk decode plus its commit, with every device-side index array prepared up front.
 
     ``run(q, k, v)`` issues only C-ABI launches on one stream -- blockify(Q), score+top-k,
-    attend, blockify(K), blockify(V) into the chunk's ring positions, memory update (3
+    attend, blockify(K), blockify(V) into the chunk's ring positions, memory update (2
     kernels) -- with no host synchronisation or allocation, so it can be timed per kernel
     or captured in a CUDA graph.  It does not advance the cache's host bookkeeping: the same
     step can be replayed on a restored state (see ``snapshot``/``restore``).
@@ -319,8 +334,8 @@ class ChunkDecodeStep:
         self.cache = cache
         self.fused_select = fused_select
         # kernels per run(): [blockify(Q) + select] (1 fused or 2) + attend + blockify K, V (2)
-        # + memory update (3)
-        self.LAUNCHES = (1 if fused_select else 2) + 1 + 2 + 3
+        # + memory update (2)
+        self.LAUNCHES = (1 if fused_select else 2) + 1 + 2 + 2
         self.q_frames = q_frames or c.chunk_frames
         if cache._cand is None:
             cache._refresh_window()
@@ -364,9 +379,7 @@ class ChunkDecodeStep:
         cs, cg, n = ca._cand
         mk(0)
         if self.fused_select:
-            L.pbsa_blockify_score_select(g, q, self.q_frames, self.q_reps, ca.k_reps, ps, cs, cg, n,
-                                         c.topk if n else 0, ca.p_list, ca.p_cnt, c.capacity, self.kv_slot,
-                                         self.kv_cnt, ca.kv_ld, ws=ws, stream=stream)
+            ca._select_fused(q, self.q_frames, self.q_reps, self.kv_slot, self.kv_cnt, ca.kv_ld, stream)
             mk(1)
         else:
             L.pbsa_blockify(g, q, self.q_frames, self.q_reps, self.nq, ws=ws, stream=stream)

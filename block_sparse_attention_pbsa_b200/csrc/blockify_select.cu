@@ -17,6 +17,13 @@
 //  4. ranks on (score desc, gid asc, position asc): lists of up to 256 candidates are sorted
 //     by a bitonic network in shared memory (one element per thread), longer ones ranked by
 //     counting; the first k are written behind the copied prefix.
+//
+// Hierarchical variant (Light Forcing, papernotes.org notes, "方法详解" HSA, steps (1)-(3), as a
+// selection policy over the local window): between 3 and 4, the candidates (whole frames,
+// frame slot = position / bpf) get frame scores = the mean of their blocks' scores (the score
+// of the frame's mean-pooled representative, by linearity), summed in block order; the
+// n_recent latest frames are always chosen, plus the top_frames best others (score
+// descending, the earlier frame on ties); blocks of the other frames leave the ranking.
 #include <math.h>
 
 #include "common.cuh"
@@ -28,6 +35,7 @@ namespace {
 constexpr int BS_THREADS = 256;
 constexpr int BS_BATCH = 9;   // candidates per warp in flight (144 candidates: two rounds)
 constexpr int SORT_N = 256;   // candidate lists up to this long are ranked by a bitonic sort
+constexpr int HSA_MAX_FRAMES = 256;
 
 template <typename T>
 __device__ __forceinline__ void add_chunk16(float* acc, const uint4& v);
@@ -57,13 +65,14 @@ __device__ __forceinline__ void vec_to(const float4& v, float* o) { o[0] = v.x; 
 __device__ __forceinline__ void vec_to(const float2& v, float* o) { o[0] = v.x; o[1] = v.y; }
 __device__ __forceinline__ void vec_to(const float& v, float* o) { o[0] = v; }
 
-template <typename T, int D>
+template <typename T, int D, bool HSA>
 __global__ void __launch_bounds__(BS_THREADS) blockify_select_kernel(
     const T* __restrict__ x, Geo g, int nq, float* __restrict__ q_reps,
     const float* __restrict__ k_reps, int pool_slots, const int* __restrict__ cand_slot,
     const int* __restrict__ cand_gid, int ncand, int k, const int* __restrict__ prefix_slot,
     const int* __restrict__ prefix_cnt, int prefix_ld, int* __restrict__ out_slot,
-    int* __restrict__ out_cnt, int out_ld, float* __restrict__ out_score, void* ws) {
+    int* __restrict__ out_cnt, int out_ld, float* __restrict__ out_score, int top_frames,
+    int n_recent, void* ws) {
   constexpr int VEC = 16 / sizeof(T);   // token elements per 16-byte chunk
   constexpr int CPR = D / VEC;          // chunks per token row
   constexpr int RPP = BS_THREADS / CPR; // rows per pass
@@ -166,9 +175,37 @@ __global__ void __launch_bounds__(BS_THREADS) blockify_select_kernel(
   }
   const size_t o = (size_t)h * nq + r;
   for (int j = tid; j < pc; j += BS_THREADS) out_slot[o * out_ld + j] = prefix_slot[(size_t)h * prefix_ld + j];
-  const int kk = min(k, ncand);
-  if (tid == 0) out_cnt[o] = pc + kk;
+  int kk = min(k, ncand);
   __syncthreads();
+  if (HSA) {
+    // frame level: mean of each frame's block scores (block order), rank the non-recent
+    // frames, drop the blocks of frames not chosen from the ranking (key 0 sorts last)
+    __shared__ float fsc[HSA_MAX_FRAMES];
+    __shared__ int fchosen[HSA_MAX_FRAMES], n_elig_s;
+    const int bpf = g.bpf, nf = ncand / bpf, first_recent = max(0, nf - n_recent);
+    for (int t = tid; t < nf; t += BS_THREADS) {
+      float a = 0.f;
+      for (int b = 0; b < bpf; ++b) a += sc[t * bpf + b];
+      fsc[t] = a * (1.0f / (float)bpf);
+    }
+    __syncthreads();
+    for (int t = tid; t < nf; t += BS_THREADS) {
+      int rank = 0;
+      if (t < first_recent)
+        for (int t2 = 0; t2 < first_recent; ++t2)
+          rank += (fsc[t2] > fsc[t]) | ((fsc[t2] == fsc[t]) & (t2 < t));
+      fchosen[t] = t >= first_recent || rank < top_frames;
+    }
+    if (tid == 0) n_elig_s = 0;
+    __syncthreads();
+    for (int cc = tid; cc < ncand; cc += BS_THREADS) {
+      if (fchosen[cc / bpf]) atomicAdd(&n_elig_s, 1);
+      else key[cc] = 0ull;
+    }
+    __syncthreads();
+    kk = min(k, n_elig_s);
+  }
+  if (tid == 0) out_cnt[o] = pc + kk;
   if (ncand <= SORT_N) {
     // bitonic sort, descending on (key, -position); padding sorts last
     __shared__ uint64_t skey[SORT_N];
@@ -216,20 +253,21 @@ __global__ void __launch_bounds__(BS_THREADS) blockify_select_kernel(
   }
 }
 
-template <typename T, int D>
+template <typename T, int D, bool HSA>
 cudaError_t launch_t(const Geo& g, const void* x, int q_frames, float* q_reps, const float* k_reps,
                      int pool_slots, const int* cand_slot, const int* cand_gid, int ncand, int k,
                      const int* prefix_slot, const int* prefix_cnt, int prefix_ld, int* out_slot,
-                     int* out_cnt, int out_ld, float* out_score, void* ws, cudaStream_t st) {
+                     int* out_cnt, int out_ld, float* out_score, int top_frames, int n_recent,
+                     void* ws, cudaStream_t st) {
   const int nq = q_frames * g.bpf;
   const size_t smem = (size_t)ncand * (8 + 4 + 4 + 4);
-  auto kern = blockify_select_kernel<T, D>;
+  auto kern = blockify_select_kernel<T, D, HSA>;
   cudaError_t e = set_smem_once((const void*)kern, (int)(smem > 0 ? smem : 8));
   if (e != cudaSuccess) return e;
   kern<<<dim3(nq, g.H), BS_THREADS, smem, st>>>(static_cast<const T*>(x), g, nq, q_reps, k_reps,
                                                  pool_slots, cand_slot, cand_gid, ncand, k,
                                                  prefix_slot, prefix_cnt, prefix_ld, out_slot,
-                                                 out_cnt, out_ld, out_score, ws);
+                                                 out_cnt, out_ld, out_score, top_frames, n_recent, ws);
   return cudaGetLastError();
 }
 
@@ -239,12 +277,17 @@ cudaError_t launch_blockify_select(const Geo& g, const void* x, int q_frames, fl
                                    const float* k_reps, int pool_slots, const int* cand_slot,
                                    const int* cand_gid, int ncand, int k, const int* prefix_slot,
                                    const int* prefix_cnt, int prefix_ld, int* out_slot,
-                                   int* out_cnt, int out_ld, float* out_score, void* ws,
-                                   cudaStream_t st) {
-#define PBSA_BS(TT, DD)                                                                         \
-  return launch_t<TT, DD>(g, x, q_frames, q_reps, k_reps, pool_slots, cand_slot, cand_gid,     \
-                          ncand, k, prefix_slot, prefix_cnt, prefix_ld, out_slot, out_cnt,     \
-                          out_ld, out_score, ws, st);
+                                   int* out_cnt, int out_ld, float* out_score, int top_frames,
+                                   int n_recent, void* ws, cudaStream_t st) {
+  const bool hsa = top_frames >= 0;
+#define PBSA_BS(TT, DD)                                                                          \
+  return hsa ? launch_t<TT, DD, true>(g, x, q_frames, q_reps, k_reps, pool_slots, cand_slot,     \
+                                      cand_gid, ncand, k, prefix_slot, prefix_cnt, prefix_ld,   \
+                                      out_slot, out_cnt, out_ld, out_score, top_frames,         \
+                                      n_recent, ws, st)                                         \
+             : launch_t<TT, DD, false>(g, x, q_frames, q_reps, k_reps, pool_slots, cand_slot,    \
+                                       cand_gid, ncand, k, prefix_slot, prefix_cnt, prefix_ld,  \
+                                       out_slot, out_cnt, out_ld, out_score, 0, 0, ws, st);
   if (g.dtype == PBSA_BF16) {
     if (g.d == 128) { PBSA_BS(__nv_bfloat16, 128) }
     if (g.d == 64) { PBSA_BS(__nv_bfloat16, 64) }

@@ -130,6 +130,26 @@ PBSA_API pbsa_status pbsa_blockify_score_select(const pbsa_geom* g, const void* 
                                        int* out_slot, int* out_cnt, int out_ld, float* out_score,
                                        void* ws, void* stream);
 
+/* a1 + a2 fused, hierarchical selection -- as pbsa_blockify_score_select, but the candidates
+ * are chosen in two levels, after the hierarchical sparse attention of the related Light
+ * Forcing method (papernotes.org notes, "方法详解", HSA steps (1)-(3)):
+ *   frame score(t)  = mean of the scores of frame t's blocks (= the score of its mean-pooled
+ *                     representative), summed in block order;
+ *   chosen frames   = the n_recent_frames latest frames + the top_frames best other frames
+ *                     (score descending, the earlier frame on ties);
+ *   selection       = the k best blocks of the chosen frames (score descending, then the lower
+ *                     cand_gid, then the lower position).
+ *  The candidates must come in whole frames in time order: ncand = nf * bpf, candidate c in
+ *  frame slot c / bpf (nf <= 256).  out_cnt[h][r] = pc + min(k, blocks of the chosen frames).
+ *  Other arguments, outputs and limits as for pbsa_blockify_score_select. */
+PBSA_API pbsa_status pbsa_blockify_hsa_select(const pbsa_geom* g, const void* q, int q_frames,
+                                     float* q_reps, const float* k_reps, int pool_slots,
+                                     const int* cand_slot, const int* cand_gid, int ncand,
+                                     int top_frames, int n_recent_frames, int k,
+                                     const int* prefix_slot, const int* prefix_cnt, int prefix_ld,
+                                     int* out_slot, int* out_cnt, int out_ld, float* out_score,
+                                     void* ws, void* stream);
+
 /* a3 -- fine attention over the selected blocks (the hybrid mask of the Chinese
  * explainer 2.2 "掩码机制"; English 2.C "Global Access" + "Local Sparsity"):
  * for every token i of query block r of head h,

@@ -16,22 +16,30 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def layer_cfg(w, staging=0):
+def layer_cfg(w, staging=0, hsa=None):
+    top, recent = hsa if hsa is not None else (-1, 1)
     return P.LayerConfig(w.heads, w.head_dim, w.frame_h, w.frame_w, w.tile_h, w.tile_w, w.capacity,
-                         w.window_frames, w.chunk_frames, w.topk, w.gamma, w.dtype, staging)
+                         w.window_frames, w.chunk_frames, w.topk, w.gamma, w.dtype, staging,
+                         hsa_top_frames=top, hsa_recent=recent)
 
 
-def _decode_single_step(w, sample_units=None):
+def _decode_single_step(w, sample_units=None, hsa=None):
+    """One chunk decode against the oracle's plan.  ``hsa`` = (top_frames, recent frames)
+    selects with the two-level policy (through the one-launch blockify + selection);
+    otherwise the flat top-k through the two-call path."""
     q, k, v = I.single_step(w)
     kc = I.tokens(w, w.chunk_frames, I.stream_seed(w.seed, 4))
     vc = I.tokens(w, w.chunk_frames, I.stream_seed(w.seed, 5))
     bpf = w.blocks_per_frame
-    cache = P.PBSALayerCache(layer_cfg(w, (w.hist_frames - w.window_frames) * bpf))
+    cache = P.PBSALayerCache(layer_cfg(w, (w.hist_frames - w.window_frames) * bpf, hsa))
     qd = q.to(DEV)
     q_reps = cache.query_reps(qd)
     cache.prefill(k.to(DEV), v.to(DEV), w.hist_frames, q_reps)
     P_gpu = cache.persistent_gids()
-    kv_slot, kv_cnt, ld = cache.select(q_reps)
+    if hsa is None:
+        kv_slot, kv_cnt, ld = cache.select(q_reps)
+    else:
+        _, kv_slot, kv_cnt, ld = cache.query_select(qd)
     lse = torch.zeros((w.heads, qd.shape[0]), device=DEV)
     o = cache.attend(qd, kv_slot, kv_cnt, ld, lse=lse)
     s2g = cache.slot_to_gid()
@@ -46,6 +54,13 @@ def _decode_single_step(w, sample_units=None):
     gd = geom_dict(w)
     plan = O.single_step_plan(q64, k64, gd, w.hist_frames, w.chunk_frames, w.capacity,
                               w.window_frames, w.topk, w.gamma, k_chunk=f64(kc))
+    if hsa is not None:   # replace the flat selections by the two-level ones
+        qr64, kr64, local = O.block_reps(q64, gd, w.chunk_frames), O.block_reps(k64, gd, w.hist_frames), plan["local"]
+        for h in range(w.heads):
+            for r in range(qr64.shape[1]):
+                pos, fgap, bgap = O.hsa_select(qr64[h, r], kr64[h][local], local, bpf, hsa[0], hsa[1], w.topk, gd["scale"])
+                plan["sel"][h][r] = [local[i] for i in pos]
+                plan["sel_gap"][h][r] = min(fgap, bgap)
     nq = w.chunk_frames * bpf
     units = [(h, r) for h in range(w.heads) for r in range(nq)]
     if sample_units is not None:
@@ -85,6 +100,14 @@ def test_decode_tiny_f32():
 
 def test_decode_5s_last_chunk_bf16():
     _decode_single_step(I.DECODE_5S, sample_units=24)
+
+
+def test_decode_5s_last_chunk_hierarchical_selection():
+    _decode_single_step(I.DECODE_5S, sample_units=24, hsa=(3, 1))
+
+
+def test_decode_tiny_hierarchical_selection():
+    _decode_single_step(I.TINY, hsa=(0, 1))
 
 
 def _rollout(w, n_chunks, sample_every=3):

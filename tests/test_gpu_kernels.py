@@ -171,6 +171,61 @@ def test_blockify_score_select(wname, ncand, k, dup):
     assert ncand == 0 or checked >= H * nq // 2
 
 
+@pytest.mark.parametrize("wname,nf,top_frames,n_recent,k", [
+    ("decode", 6, 3, 1, 32), ("decode", 6, 0, 1, 32), ("decode", 6, 5, 1, 32), ("decode", 6, 2, 0, 16),
+    ("decode", 12, 4, 2, 40), ("tiny", 4, 1, 1, 4)])
+def test_blockify_hsa_select(wname, nf, top_frames, n_recent, k):
+    """pbsa_blockify_hsa_select against the oracle's two-level (frame, then block) selection;
+    sets compared where neither cut-off is a near tie."""
+    w = {"decode": dataclasses.replace(I.DECODE_5S, heads=3), "tiny": I.TINY}[wname]
+    g = geom_for(w)
+    H, d, bpf, n_frames = w.heads, w.head_dim, w.blocks_per_frame, 2
+    nq = n_frames * bpf
+    ncand = nf * bpf
+    x = I.tokens(w, n_frames, 41 + nf + top_frames)
+    gen = torch.Generator().manual_seed(9 + nf + 10 * top_frames + n_recent)
+    pool, prefix = ncand + 50, 12
+    # window reps: one offset per frame so that frames differ, plus block noise
+    kr = torch.randn((H, pool, d), generator=gen) * 0.3
+    frame_off = torch.randn((H, nf, d), generator=gen) * 0.3
+    cs = torch.stack([torch.randperm(pool, generator=gen)[:ncand] for _ in range(H)]).to(torch.int32)
+    for h in range(H):
+        for c in range(ncand):
+            kr[h, int(cs[h, c])] += frame_off[h, c // bpf]
+    first_frame = 3
+    cg = torch.tensor([[(first_frame + c // bpf) * bpf + c % bpf for c in range(ncand)]] * H, dtype=torch.int32)
+    ps = torch.randint(0, pool, (H, prefix), generator=gen, dtype=torch.int32)
+    pc = torch.tensor([prefix - h for h in range(H)], dtype=torch.int32)
+    out_ld = prefix + k + 3
+    out = torch.full((H, nq, out_ld), -7, dtype=torch.int32, device=DEV)
+    cnt = torch.zeros((H, nq), dtype=torch.int32, device=DEV)
+    qr = torch.zeros((H, nq, d), device=DEV)
+    ws = ws_for(g)
+    P.pbsa_blockify_hsa_select(g, x.to(DEV), n_frames, qr, kr.to(DEV), pool, cs.to(DEV), cg.to(DEV), ncand,
+                               top_frames, n_recent, k, ps.to(DEV), pc.to(DEV), prefix, out, cnt, out_ld, None, ws)
+    check_no_device_error(ws)
+    want_q = O.block_reps(f64(x), geom_dict(w), n_frames)
+    np.testing.assert_allclose(f64(qr), want_q, rtol=0, atol=2e-6)
+    out, cnt = out.cpu(), cnt.cpu()
+    nchosen = min(nf, n_recent + top_frames) * bpf
+    checked = 0
+    for h in range(H):
+        reps_h = f64(kr[h][cs[h].long()])
+        for r in range(nq):
+            p = int(pc[h])
+            kk = min(k, nchosen)
+            assert int(cnt[h, r]) == p + kk
+            assert out[h, r, :p].tolist() == ps[h, :p].tolist()
+            pos, fgap, bgap = O.hsa_select(want_q[h, r], reps_h, cg[h].tolist(), bpf, top_frames, n_recent,
+                                           k, w.scale)
+            got = out[h, r, p:p + kk].tolist()
+            assert len(set(got)) == kk and set(got) <= set(cs[h].tolist())
+            if fgap > NEAR_TIE and bgap > NEAR_TIE:
+                assert set(got) == {int(cs[h, c]) for c in pos}, (h, r)
+                checked += 1
+    assert checked >= H * nq // 2
+
+
 # ----------------------------------------------------------------------------- attend
 def _attend_case(w, q_frames, slots, lists, seed):
     gen = torch.Generator().manual_seed(seed)
