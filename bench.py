@@ -374,7 +374,10 @@ def run_variant(P, I, dev, w, steps: int, **cfg_changes):
     torch.cuda.synchronize(dev)
     marks = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(6)]
     graph = step.capture(qd, kcd, vcd, o, marks=marks)
-    spans = {"blockify_select": (0, 2), "attend": (2, 3), "commit_blockify_kv": (3, 4), "memory_update": (4, 5)}
+    if cfg.own_chunk:   # the chunk's K, V are written before the selection
+        spans = {"commit_blockify_kv": (0, 1), "blockify_select": (1, 2), "attend": (2, 3), "memory_update": (4, 5)}
+    else:
+        spans = {"blockify_select": (0, 2), "attend": (2, 3), "commit_blockify_kv": (3, 4), "memory_update": (4, 5)}
     runs = {g: [] for g in spans}
     total = []
     for s in range(steps + 3):
@@ -547,7 +550,8 @@ def run_pbsa(args, w, rank, world, local_rank):
     }
     if not args.no_train:
         line["train"] = run_train(P, I, dev, 5, peaks)
-    line["variants"] = [run_variant(P, I, dev, w, max(5, args.steps // 2), hsa_top_frames=3, hsa_recent=1)]
+    line["variants"] = [run_variant(P, I, dev, w, max(5, args.steps // 2), hsa_top_frames=3, hsa_recent=1),
+                        run_variant(P, I, dev, w, max(5, args.steps // 2), own_chunk=True)]
     if not args.no_rollout:
         line["rollouts"] = [run_rollout(P, I, dev, I.ROLLOUT_5S), run_rollout(P, I, dev, I.ROLLOUT_1MIN)]
     if world == 1 and not args.no_cpu_baseline:

@@ -43,6 +43,10 @@ class LayerConfig:
     # then the top-k blocks of those frames
     hsa_top_frames: int = -1
     hsa_recent: int = 1
+    # own-chunk variant: every query block also attends the chunk's own blocks, written into
+    # their ring positions at the current step before the selection (the chunk-wise
+    # self-attention of the trainable path, applied at inference)
+    own_chunk: bool = False
 
     @property
     def bpf(self) -> int:
@@ -77,7 +81,7 @@ class PBSALayerCache:
         self.max_pool_entries = C + max(self.ring_frames * bpf, cfg.staging_blocks)
         self.ws = torch.zeros(L.pbsa_workspace_bytes(self.geom, nq, self.max_pool_entries),
                               dtype=torch.uint8, device=dev)
-        self.kv_ld = C + max(cfg.topk, 0)
+        self.kv_ld = C + max(cfg.topk, 0) + (nq if cfg.own_chunk else 0)
         self.kv_ld_own = max(self.kv_ld, nq)
         # flat buffers, viewed per call as [H, nq, ...] for chunks of up to chunk_frames frames
         self._q_reps_buf = torch.zeros(H * nq * d, dtype=torch.float32, device=dev)
@@ -191,17 +195,16 @@ class PBSALayerCache:
         return self.q_reps, self.kv_slot, self.kv_cnt, self.kv_ld_own
 
     def _select_fused(self, q, nf, q_reps, kv_slot, kv_cnt, kv_ld, stream=None):
-        """The one-launch blockify + selection of the configured policy."""
+        """The one-launch blockify + selection of the configured policy (and, for the own-chunk
+        variant, the chunk's ring slots appended to every row)."""
         c = self.cfg
         cs, cg, n = self._cand
-        if c.hsa_top_frames >= 0 and n:
-            L.pbsa_blockify_hsa_select(self.geom, q, nf, q_reps, self.k_reps, self.pool_slots, cs, cg, n,
-                                       c.hsa_top_frames, c.hsa_recent, c.topk, self.p_list, self.p_cnt,
-                                       c.capacity, kv_slot, kv_cnt, kv_ld, ws=self.ws, stream=stream)
-        else:
-            L.pbsa_blockify_score_select(self.geom, q, nf, q_reps, self.k_reps, self.pool_slots, cs, cg, n,
-                                         c.topk if n else 0, self.p_list, self.p_cnt, c.capacity, kv_slot,
-                                         kv_cnt, kv_ld, ws=self.ws, stream=stream)
+        top = c.hsa_top_frames if (c.hsa_top_frames >= 0 and n) else -1
+        own = self._frames_dst(self.hist, nf) if c.own_chunk else None
+        L.pbsa_blockify_select_ex(self.geom, q, nf, q_reps, self.k_reps, self.pool_slots, cs, cg, n,
+                                  c.topk if n else 0, top, c.hsa_recent, self.p_list, self.p_cnt, c.capacity,
+                                  own, own.numel() if own is not None else 0, kv_slot, kv_cnt, kv_ld,
+                                  ws=self.ws, stream=stream)
 
     def attend(self, q, kv_slot, kv_cnt, kv_ld, o=None, lse=None, stream=None):
         """a3: fine attention over the listed slots."""
@@ -220,6 +223,10 @@ class PBSALayerCache:
         if self._cand is None:
             self._refresh_window()
         if self.hist > 0:
+            if self.cfg.own_chunk:
+                if k is None or v is None:
+                    raise ValueError("the own-chunk variant attends the chunk's blocks: pass its k and v")
+                self._write_chunk(k, v, stream)
             _, kv_slot, kv_cnt, kv_ld = self.query_select(q, stream)
             return self.attend(q, kv_slot, kv_cnt, kv_ld, o, lse, stream)
         # empty history: the chunk attends its own blocks
@@ -367,8 +374,10 @@ class ChunkDecodeStep:
         return 4.0 * 64 * 64 * c.head_dim * cnt
 
     def run(self, q, k, v, o, lse=None, stream=None, marks=None):
-        """``marks``: optional list of torch.cuda.Event recorded after each kernel group
-        (blockify Q, select, attend, commit blockify K+V, memory update)."""
+        """``marks``: optional list of 6 torch.cuda.Event recorded around the kernel groups:
+        0 | blockify Q (+ select) | 1 | select | 2 | attend | 3 | commit blockify K+V | 4 | memory
+        update | 5.  For the own-chunk variant the chunk's blockify K+V runs first (between
+        marks 0 and 1), the fused selection between 1 and 2, and nothing between 3 and 4."""
         ca, c = self.cache, self.cache.cfg
         g, ws, ps = ca.geom, ca.ws, ca.pool_slots
         if marks is not None:
@@ -376,14 +385,21 @@ class ChunkDecodeStep:
             mk = lambda i: marks[i].record(ev_stream)  # noqa: E731
         else:
             mk = lambda i: None  # noqa: E731
-        cs, cg, n = ca._cand
+        own = c.own_chunk
         mk(0)
+        if own:   # the chunk's K, V go to their ring positions first: every row attends them
+            L.pbsa_blockify(g, k, self.q_frames, ca.k_reps, ps, self.dst, ca.k_pool, ps, ws=ws, stream=stream)
+            L.pbsa_blockify(g, v, self.q_frames, self.vreps, ps, self.dst, ca.v_pool, ps, ws=ws, stream=stream)
+            mk(1)
+        cs, cg, n = ca._cand
         if self.fused_select:
             ca._select_fused(q, self.q_frames, self.q_reps, self.kv_slot, self.kv_cnt, ca.kv_ld, stream)
-            mk(1)
+            if not own:
+                mk(1)
         else:
             L.pbsa_blockify(g, q, self.q_frames, self.q_reps, self.nq, ws=ws, stream=stream)
-            mk(1)
+            if not own:
+                mk(1)
             L.pbsa_score_select(g, self.q_reps, self.nq, ca.k_reps, ps, cs, cg, n, c.topk if n else 0,
                                 ca.p_list, ca.p_cnt, c.capacity, self.kv_slot, self.kv_cnt, ca.kv_ld,
                                 ws=ws, stream=stream)
@@ -391,8 +407,9 @@ class ChunkDecodeStep:
         L.pbsa_attend(g, q, self.q_frames, ca.k_pool, ca.v_pool, ps, self.kv_slot, self.kv_cnt, ca.kv_ld,
                       o, lse, ws=ws, stream=stream)
         mk(3)
-        L.pbsa_blockify(g, k, self.q_frames, ca.k_reps, ps, self.dst, ca.k_pool, ps, ws=ws, stream=stream)
-        L.pbsa_blockify(g, v, self.q_frames, self.vreps, ps, self.dst, ca.v_pool, ps, ws=ws, stream=stream)
+        if not own:
+            L.pbsa_blockify(g, k, self.q_frames, ca.k_reps, ps, self.dst, ca.k_pool, ps, ws=ws, stream=stream)
+            L.pbsa_blockify(g, v, self.q_frames, self.vreps, ps, self.dst, ca.v_pool, ps, ws=ws, stream=stream)
         mk(4)
         L.pbsa_memory_update(g, self.q_reps, self.nq, ca.k_reps, ca.k_pool, ca.v_pool, ps, ca.slot_gid,
                              ca.slot_ema, c.capacity, c.bpf, self.cs, self.cg, self.ncand, c.gamma,

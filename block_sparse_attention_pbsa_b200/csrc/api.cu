@@ -120,30 +120,45 @@ pbsa_status pbsa_score_select(const pbsa_geom* gin, const float* q_reps, int nq,
                                        out_ld, out_score, ws, static_cast<cudaStream_t>(stream)));
 }
 
-pbsa_status pbsa_blockify_score_select(const pbsa_geom* gin, const void* q, int q_frames,
-                                       float* q_reps, const float* k_reps, int pool_slots,
-                                       const int* cand_slot, const int* cand_gid, int ncand, int k,
-                                       const int* prefix_slot, const int* prefix_cnt, int prefix_ld,
-                                       int* out_slot, int* out_cnt, int out_ld, float* out_score,
-                                       void* ws, void* stream) {
+pbsa_status pbsa_blockify_select_ex(const pbsa_geom* gin, const void* q, int q_frames, float* q_reps,
+                                    const float* k_reps, int pool_slots, const int* cand_slot,
+                                    const int* cand_gid, int ncand, int k, int top_frames,
+                                    int n_recent_frames, const int* prefix_slot, const int* prefix_cnt,
+                                    int prefix_ld, const int* suffix_slot, int suffix_n, int* out_slot,
+                                    int* out_cnt, int out_ld, float* out_score, void* ws, void* stream) {
   Geo g;
   pbsa_status s = make_geo(gin, &g);
   if (s != PBSA_OK) return s;
   if (q == nullptr || q_reps == nullptr || k_reps == nullptr || out_slot == nullptr ||
       out_cnt == nullptr)
     return PBSA_ERR_INVALID_ARG;
-  if (q_frames <= 0 || ncand < 0 || k < 0 || pool_slots <= 0 || prefix_ld < 0) return PBSA_ERR_INVALID_ARG;
+  if (q_frames <= 0 || ncand < 0 || k < 0 || pool_slots <= 0 || prefix_ld < 0 || suffix_n < 0)
+    return PBSA_ERR_INVALID_ARG;
   if ((int64_t)q_frames * g.bpf > 65535 * 64) return PBSA_ERR_INVALID_ARG;
   if (ncand > 0 && (cand_slot == nullptr || cand_gid == nullptr)) return PBSA_ERR_INVALID_ARG;
   if ((prefix_cnt == nullptr) != (prefix_slot == nullptr)) return PBSA_ERR_INVALID_ARG;
+  if (suffix_n > 0 && suffix_slot == nullptr) return PBSA_ERR_INVALID_ARG;
+  if (top_frames >= 0 && (n_recent_frames < 0 || ncand % g.bpf != 0)) return PBSA_ERR_INVALID_ARG;
   if (prefix_slot == nullptr) prefix_ld = 0;
-  if (out_ld < prefix_ld + k) return PBSA_ERR_INVALID_ARG;
-  if (ncand > 1024) return PBSA_ERR_UNSUPPORTED;
+  if (out_ld < prefix_ld + k + suffix_n) return PBSA_ERR_INVALID_ARG;
+  if (ncand > 1024 || (top_frames >= 0 && ncand / g.bpf > 256)) return PBSA_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(q_reps) || !aligned16(k_reps)) return PBSA_ERR_INVALID_ARG;
   return from_cuda(launch_blockify_select(g, q, q_frames, q_reps, k_reps, pool_slots, cand_slot,
                                           cand_gid, ncand, k, prefix_slot, prefix_cnt, prefix_ld,
-                                          out_slot, out_cnt, out_ld, out_score, -1, 0, ws,
-                                          static_cast<cudaStream_t>(stream)));
+                                          out_slot, out_cnt, out_ld, out_score,
+                                          top_frames < 0 ? -1 : top_frames, n_recent_frames,
+                                          suffix_slot, suffix_n, ws, static_cast<cudaStream_t>(stream)));
+}
+
+pbsa_status pbsa_blockify_score_select(const pbsa_geom* gin, const void* q, int q_frames,
+                                       float* q_reps, const float* k_reps, int pool_slots,
+                                       const int* cand_slot, const int* cand_gid, int ncand, int k,
+                                       const int* prefix_slot, const int* prefix_cnt, int prefix_ld,
+                                       int* out_slot, int* out_cnt, int out_ld, float* out_score,
+                                       void* ws, void* stream) {
+  return pbsa_blockify_select_ex(gin, q, q_frames, q_reps, k_reps, pool_slots, cand_slot, cand_gid, ncand,
+                                 k, -1, 0, prefix_slot, prefix_cnt, prefix_ld, nullptr, 0, out_slot,
+                                 out_cnt, out_ld, out_score, ws, stream);
 }
 
 pbsa_status pbsa_blockify_hsa_select(const pbsa_geom* gin, const void* q, int q_frames, float* q_reps,
@@ -153,25 +168,10 @@ pbsa_status pbsa_blockify_hsa_select(const pbsa_geom* gin, const void* q, int q_
                                      const int* prefix_cnt, int prefix_ld, int* out_slot,
                                      int* out_cnt, int out_ld, float* out_score, void* ws,
                                      void* stream) {
-  Geo g;
-  pbsa_status s = make_geo(gin, &g);
-  if (s != PBSA_OK) return s;
-  if (q == nullptr || q_reps == nullptr || k_reps == nullptr || out_slot == nullptr ||
-      out_cnt == nullptr)
-    return PBSA_ERR_INVALID_ARG;
-  if (q_frames <= 0 || ncand < 0 || k < 0 || pool_slots <= 0 || prefix_ld < 0) return PBSA_ERR_INVALID_ARG;
-  if (top_frames < 0 || n_recent_frames < 0 || ncand % g.bpf != 0) return PBSA_ERR_INVALID_ARG;
-  if ((int64_t)q_frames * g.bpf > 65535 * 64) return PBSA_ERR_INVALID_ARG;
-  if (ncand > 0 && (cand_slot == nullptr || cand_gid == nullptr)) return PBSA_ERR_INVALID_ARG;
-  if ((prefix_cnt == nullptr) != (prefix_slot == nullptr)) return PBSA_ERR_INVALID_ARG;
-  if (prefix_slot == nullptr) prefix_ld = 0;
-  if (out_ld < prefix_ld + k) return PBSA_ERR_INVALID_ARG;
-  if (ncand > 1024 || ncand / g.bpf > 256) return PBSA_ERR_UNSUPPORTED;
-  if (!aligned16(q) || !aligned16(q_reps) || !aligned16(k_reps)) return PBSA_ERR_INVALID_ARG;
-  return from_cuda(launch_blockify_select(g, q, q_frames, q_reps, k_reps, pool_slots, cand_slot,
-                                          cand_gid, ncand, k, prefix_slot, prefix_cnt, prefix_ld,
-                                          out_slot, out_cnt, out_ld, out_score, top_frames,
-                                          n_recent_frames, ws, static_cast<cudaStream_t>(stream)));
+  if (top_frames < 0 || n_recent_frames < 0) return PBSA_ERR_INVALID_ARG;
+  return pbsa_blockify_select_ex(gin, q, q_frames, q_reps, k_reps, pool_slots, cand_slot, cand_gid, ncand,
+                                 k, top_frames, n_recent_frames, prefix_slot, prefix_cnt, prefix_ld,
+                                 nullptr, 0, out_slot, out_cnt, out_ld, out_score, ws, stream);
 }
 
 pbsa_status pbsa_attend(const pbsa_geom* gin, const void* q, int q_frames, const void* k_pool,

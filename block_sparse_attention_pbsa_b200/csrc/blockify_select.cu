@@ -16,7 +16,8 @@
 //     butterfly shuffle sums the lane partials (fixed order: deterministic);
 //  4. ranks on (score desc, gid asc, position asc): lists of up to 256 candidates are sorted
 //     by a bitonic network in shared memory (one element per thread), longer ones ranked by
-//     counting; the first k are written behind the copied prefix.
+//     counting; the first k are written behind the copied prefix, then an optional suffix
+//     list shared by every row (e.g. the chunk's own blocks).
 //
 // Hierarchical variant (Light Forcing, papernotes.org notes, "方法详解" HSA, steps (1)-(3), as a
 // selection policy over the local window): between 3 and 4, the candidates (whole frames,
@@ -72,7 +73,7 @@ __global__ void __launch_bounds__(BS_THREADS) blockify_select_kernel(
     const int* __restrict__ cand_gid, int ncand, int k, const int* __restrict__ prefix_slot,
     const int* __restrict__ prefix_cnt, int prefix_ld, int* __restrict__ out_slot,
     int* __restrict__ out_cnt, int out_ld, float* __restrict__ out_score, int top_frames,
-    int n_recent, void* ws) {
+    int n_recent, const int* __restrict__ suffix_slot, int suffix_n, void* ws) {
   constexpr int VEC = 16 / sizeof(T);   // token elements per 16-byte chunk
   constexpr int CPR = D / VEC;          // chunks per token row
   constexpr int RPP = BS_THREADS / CPR; // rows per pass
@@ -205,7 +206,8 @@ __global__ void __launch_bounds__(BS_THREADS) blockify_select_kernel(
     __syncthreads();
     kk = min(k, n_elig_s);
   }
-  if (tid == 0) out_cnt[o] = pc + kk;
+  if (tid == 0) out_cnt[o] = pc + kk + suffix_n;
+  for (int j = tid; j < suffix_n; j += BS_THREADS) out_slot[o * out_ld + pc + kk + j] = suffix_slot[j];
   if (ncand <= SORT_N) {
     // bitonic sort, descending on (key, -position); padding sorts last
     __shared__ uint64_t skey[SORT_N];
@@ -258,7 +260,7 @@ cudaError_t launch_t(const Geo& g, const void* x, int q_frames, float* q_reps, c
                      int pool_slots, const int* cand_slot, const int* cand_gid, int ncand, int k,
                      const int* prefix_slot, const int* prefix_cnt, int prefix_ld, int* out_slot,
                      int* out_cnt, int out_ld, float* out_score, int top_frames, int n_recent,
-                     void* ws, cudaStream_t st) {
+                     const int* suffix_slot, int suffix_n, void* ws, cudaStream_t st) {
   const int nq = q_frames * g.bpf;
   const size_t smem = (size_t)ncand * (8 + 4 + 4 + 4);
   auto kern = blockify_select_kernel<T, D, HSA>;
@@ -267,7 +269,8 @@ cudaError_t launch_t(const Geo& g, const void* x, int q_frames, float* q_reps, c
   kern<<<dim3(nq, g.H), BS_THREADS, smem, st>>>(static_cast<const T*>(x), g, nq, q_reps, k_reps,
                                                  pool_slots, cand_slot, cand_gid, ncand, k,
                                                  prefix_slot, prefix_cnt, prefix_ld, out_slot,
-                                                 out_cnt, out_ld, out_score, top_frames, n_recent, ws);
+                                                 out_cnt, out_ld, out_score, top_frames, n_recent,
+                                                 suffix_slot, suffix_n, ws);
   return cudaGetLastError();
 }
 
@@ -278,16 +281,18 @@ cudaError_t launch_blockify_select(const Geo& g, const void* x, int q_frames, fl
                                    const int* cand_gid, int ncand, int k, const int* prefix_slot,
                                    const int* prefix_cnt, int prefix_ld, int* out_slot,
                                    int* out_cnt, int out_ld, float* out_score, int top_frames,
-                                   int n_recent, void* ws, cudaStream_t st) {
+                                   int n_recent, const int* suffix_slot, int suffix_n, void* ws,
+                                   cudaStream_t st) {
   const bool hsa = top_frames >= 0;
 #define PBSA_BS(TT, DD)                                                                          \
   return hsa ? launch_t<TT, DD, true>(g, x, q_frames, q_reps, k_reps, pool_slots, cand_slot,     \
                                       cand_gid, ncand, k, prefix_slot, prefix_cnt, prefix_ld,   \
                                       out_slot, out_cnt, out_ld, out_score, top_frames,         \
-                                      n_recent, ws, st)                                         \
+                                      n_recent, suffix_slot, suffix_n, ws, st)                  \
              : launch_t<TT, DD, false>(g, x, q_frames, q_reps, k_reps, pool_slots, cand_slot,    \
                                        cand_gid, ncand, k, prefix_slot, prefix_cnt, prefix_ld,  \
-                                       out_slot, out_cnt, out_ld, out_score, 0, 0, ws, st);
+                                       out_slot, out_cnt, out_ld, out_score, 0, 0, suffix_slot, \
+                                       suffix_n, ws, st);
   if (g.dtype == PBSA_BF16) {
     if (g.d == 128) { PBSA_BS(__nv_bfloat16, 128) }
     if (g.d == 64) { PBSA_BS(__nv_bfloat16, 64) }

@@ -42,7 +42,8 @@ cudaError_t launch_blockify_select(const Geo& g, const void* x, int q_frames, fl
                                    const int* cand_gid, int ncand, int k, const int* prefix_slot,
                                    const int* prefix_cnt, int prefix_ld, int* out_slot,
                                    int* out_cnt, int out_ld, float* out_score, int top_frames,
-                                   int n_recent, void* ws, cudaStream_t st);
+                                   int n_recent, const int* suffix_slot, int suffix_n, void* ws,
+                                   cudaStream_t st);
 
 cudaError_t launch_attend_f32(const Geo& g, const float* q, int q_frames, const float* k_pool,
                               const float* v_pool, int pool_slots, const int* kv_slot,

@@ -150,6 +150,22 @@ PBSA_API pbsa_status pbsa_blockify_hsa_select(const pbsa_geom* g, const void* q,
                                      int* out_slot, int* out_cnt, int out_ld, float* out_score,
                                      void* ws, void* stream);
 
+/* a1 + a2 fused, general form -- pbsa_blockify_score_select (top_frames < 0) or
+ * pbsa_blockify_hsa_select (top_frames >= 0), with an optional suffix: after each row's
+ * selection, suffix_slot[0..suffix_n) (device, shared by every head and query block) is
+ * appended, and out_cnt[h][r] counts it.  The suffix serves lists that every query block
+ * attends besides its selection, e.g. the current chunk's own blocks written into the pool at
+ * the current noise level (the chunk-wise self-attention of the trainable path, English 2.D
+ * "Training Strategy", applied at inference as a variant).  Requires out_ld >= prefix_ld + k +
+ * suffix_n; other arguments, outputs and limits as for the two calls above. */
+PBSA_API pbsa_status pbsa_blockify_select_ex(const pbsa_geom* g, const void* q, int q_frames,
+                                    float* q_reps, const float* k_reps, int pool_slots,
+                                    const int* cand_slot, const int* cand_gid, int ncand, int k,
+                                    int top_frames, int n_recent_frames, const int* prefix_slot,
+                                    const int* prefix_cnt, int prefix_ld, const int* suffix_slot,
+                                    int suffix_n, int* out_slot, int* out_cnt, int out_ld,
+                                    float* out_score, void* ws, void* stream);
+
 /* a3 -- fine attention over the selected blocks (the hybrid mask of the Chinese
  * explainer 2.2 "掩码机制"; English 2.C "Global Access" + "Local Sparsity"):
  * for every token i of query block r of head h,

@@ -16,14 +16,14 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def layer_cfg(w, staging=0, hsa=None):
+def layer_cfg(w, staging=0, hsa=None, own_chunk=False):
     top, recent = hsa if hsa is not None else (-1, 1)
     return P.LayerConfig(w.heads, w.head_dim, w.frame_h, w.frame_w, w.tile_h, w.tile_w, w.capacity,
                          w.window_frames, w.chunk_frames, w.topk, w.gamma, w.dtype, staging,
-                         hsa_top_frames=top, hsa_recent=recent)
+                         hsa_top_frames=top, hsa_recent=recent, own_chunk=own_chunk)
 
 
-def _decode_single_step(w, sample_units=None, hsa=None):
+def _decode_single_step(w, sample_units=None, hsa=None, own_chunk=False):
     """One chunk decode against the oracle's plan.  ``hsa`` = (top_frames, recent frames)
     selects with the two-level policy (through the one-launch blockify + selection);
     otherwise the flat top-k through the two-call path."""
@@ -31,17 +31,21 @@ def _decode_single_step(w, sample_units=None, hsa=None):
     kc = I.tokens(w, w.chunk_frames, I.stream_seed(w.seed, 4))
     vc = I.tokens(w, w.chunk_frames, I.stream_seed(w.seed, 5))
     bpf = w.blocks_per_frame
-    cache = P.PBSALayerCache(layer_cfg(w, (w.hist_frames - w.window_frames) * bpf, hsa))
+    cache = P.PBSALayerCache(layer_cfg(w, (w.hist_frames - w.window_frames) * bpf, hsa, own_chunk))
     qd = q.to(DEV)
     q_reps = cache.query_reps(qd)
     cache.prefill(k.to(DEV), v.to(DEV), w.hist_frames, q_reps)
     P_gpu = cache.persistent_gids()
-    if hsa is None:
-        kv_slot, kv_cnt, ld = cache.select(q_reps)
-    else:
-        _, kv_slot, kv_cnt, ld = cache.query_select(qd)
     lse = torch.zeros((w.heads, qd.shape[0]), device=DEV)
-    o = cache.attend(qd, kv_slot, kv_cnt, ld, lse=lse)
+    if own_chunk:   # the step's K, V (here the chunk's committed ones) are attended as well
+        o = cache.decode_step(qd, kc.to(DEV), vc.to(DEV), lse=lse)
+        kv_slot, kv_cnt = cache.kv_slot, cache.kv_cnt
+    else:
+        if hsa is None:
+            kv_slot, kv_cnt, ld = cache.select(q_reps)
+        else:
+            _, kv_slot, kv_cnt, ld = cache.query_select(qd)
+        o = cache.attend(qd, kv_slot, kv_cnt, ld, lse=lse)
     s2g = cache.slot_to_gid()
     slot_gid = cache.slot_gid.cpu()
     kv_slot, kv_cnt, o, lse = kv_slot.cpu(), kv_cnt.cpu(), o.cpu(), lse.cpu()
@@ -51,6 +55,9 @@ def _decode_single_step(w, sample_units=None, hsa=None):
     assert P.pbsa_get_device_error(cache.ws) == 0
 
     q64, k64, v64 = f64(q), f64(k), f64(v)
+    own = list(range(w.hist_frames * bpf, (w.hist_frames + w.chunk_frames) * bpf)) if own_chunk else []
+    if own_chunk:   # K, V of the history followed by the chunk's
+        k64, v64 = np.concatenate([k64, f64(kc)]), np.concatenate([v64, f64(vc)])
     gd = geom_dict(w)
     plan = O.single_step_plan(q64, k64, gd, w.hist_frames, w.chunk_frames, w.capacity,
                               w.window_frames, w.topk, w.gamma, k_chunk=f64(kc))
@@ -75,12 +82,17 @@ def _decode_single_step(w, sample_units=None, hsa=None):
         for r in range(nq):
             n = int(kv_cnt[h, r])
             slots = kv_slot[h, r, :n].tolist()
-            gids = [pers_slot_gid[s] if s < w.capacity else s2g[s] for s in slots]
+            own_s2g = {int(x): own[i] for i, x in enumerate(cache._frames_dst(w.hist_frames, w.chunk_frames).cpu())} \
+                if own_chunk else {}
+            gids = [pers_slot_gid[s] if s < w.capacity else (own_s2g[s] if s in own_s2g else s2g[s]) for s in slots]
+            if own_chunk:
+                assert gids[len(gids) - len(own):] == own
+                gids = gids[:len(gids) - len(own)]
             sel = set(gids[len(pers_slot_gid):])
             if plan["sel_gap"][h][r] > NEAR_TIE:
                 assert sel == set(plan["sel"][h][r]), (h, r)
             if (h, r) in units and boot_exact and plan["sel_gap"][h][r] > NEAR_TIE:
-                want, wlse = O.attend_gids(q64, k64, v64, gd, h, r, plan["P"][h] + plan["sel"][h][r],
+                want, wlse = O.attend_gids(q64, k64, v64, gd, h, r, plan["P"][h] + plan["sel"][h][r] + own,
                                            q_first_frame=w.hist_frames)
                 rows = block_rows(w, r)
                 if w.dtype == "f32":
@@ -108,6 +120,14 @@ def test_decode_5s_last_chunk_hierarchical_selection():
 
 def test_decode_tiny_hierarchical_selection():
     _decode_single_step(I.TINY, hsa=(0, 1))
+
+
+def test_decode_5s_last_chunk_own_chunk():
+    _decode_single_step(I.DECODE_5S, sample_units=24, own_chunk=True)
+
+
+def test_decode_tiny_own_chunk():
+    _decode_single_step(I.TINY, own_chunk=True)
 
 
 def _rollout(w, n_chunks, sample_every=3):
