@@ -143,6 +143,32 @@ def hsa_select(q_rep, cand_reps, cand_gids, bpf: int, top_frames: int, n_recent:
     return [elig[i] for i in pos], frame_gap, kth_gap(o, gids, k)
 
 
+# --------------------------------------------------------------------------- per-chunk sparsity
+def cag_sparsity(lq, lk, d: int, s_base: float, s_target: float, alpha, n_dense: int = 1):
+    """Chunk-aware growth of the related *Light Forcing* method (papernotes.org notes,
+    "方法详解", CAG): the first ``n_dense`` chunks keep dense attention, chunk i after them gets
+    sparsity s_i = s_base - alpha_i * beta, and beta makes the attention FLOPs of those chunks
+    equal the target:
+        sum_i (1 - s_base + alpha_i beta) lq_i lk_i d = (1 - s_target) sum_i lq_i lk_i d.
+    ``lq``, ``lk``: query and key token counts per chunk; ``alpha``: each chunk's weight
+    (the noise level at which it arrives, on the pages).  Returns (beta, [s_i] per chunk).
+    """
+    n = len(lq)
+    L = [float(lq[i]) * float(lk[i]) * d for i in range(n)]
+    tail = range(n_dense, n)
+    num = (s_base - s_target) * sum(L[i] for i in tail)
+    den = sum(float(alpha[i]) * L[i] for i in tail)
+    beta = num / den if den != 0.0 else 0.0
+    return beta, [0.0 if i < n_dense else s_base - float(alpha[i]) * beta for i in range(n)]
+
+
+def cag_topk(sparsity: float, n_hist_blocks: int, n_persistent: int, n_local: int) -> int:
+    """Local top-k of a chunk whose attention keeps a (1 - sparsity) share of its history blocks,
+    the persistent blocks counted first: clamp(round((1 - s) * n_hist) - n_persistent, 0, n_local)."""
+    keep = int(np.floor((1.0 - sparsity) * n_hist_blocks + 0.5))
+    return max(0, min(n_local, keep - n_persistent))
+
+
 # --------------------------------------------------------------------------- a3: fine attention
 def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float):
     """Softmax attention of query rows over key/value rows; returns (out [n, d], lse [n]).

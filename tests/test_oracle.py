@@ -298,3 +298,37 @@ def test_hsa_brute_force_small():
         assert pos == cands[:k]
         # selected blocks lie in chosen frames, the latest n_recent frames are always available
         assert all(c // bpf in frames for c in pos)
+
+
+# ------------------------------------------------------------------ per-chunk sparsity (chunk-aware growth)
+def test_cag_meets_the_flop_budget():
+    """beta solves the budget equation exactly; the dense chunks stay dense."""
+    lq = [4608] * 7
+    lk = [0, 4608, 9216, 13824, 18432, 23040, 27648]
+    alpha = [1.0, 1.0, 0.8, 0.6, 0.4, 0.2, 0.0]
+    s_base, s_target, d = 0.9, 0.8, 128
+    beta, s = O.cag_sparsity(lq, lk, d, s_base, s_target, alpha, n_dense=1)
+    lhs = sum((1 - s_base + alpha[i] * beta) * lq[i] * lk[i] * d for i in range(1, 7))
+    rhs = (1 - s_target) * sum(lq[i] * lk[i] * d for i in range(1, 7))
+    assert lhs == pytest.approx(rhs, rel=1e-12)
+    assert s[0] == 0.0 and beta > 0
+    # the attended share (1 - s_i) of every later chunk averages, FLOP-weighted, to 1 - s_target
+    w = [lq[i] * lk[i] for i in range(1, 7)]
+    assert sum((1 - s[i]) * w[i - 1] for i in range(1, 7)) / sum(w) == pytest.approx(1 - s_target, rel=1e-12)
+    # larger alpha -> less sparse
+    assert all(s[i] <= s[i + 1] for i in range(1, 6))
+
+
+def test_cag_special_cases():
+    lq, lk = [10, 10, 10], [0, 20, 40]
+    beta, s = O.cag_sparsity(lq, lk, 8, 0.7, 0.7, [0.3, 0.5, 0.9])
+    assert beta == 0.0 and s == [0.0, 0.7, 0.7]              # target = base: no growth
+    beta, s = O.cag_sparsity(lq, lk, 8, 0.9, 0.6, [1.0, 0.5, 0.5])
+    assert s[1] == pytest.approx(0.6) and s[2] == pytest.approx(0.6)   # uniform alpha: every chunk at the target
+
+
+def test_cag_topk_mapping():
+    assert O.cag_topk(0.0, 288, 96, 144) == 144          # dense: every local block
+    assert O.cag_topk(0.5, 288, 96, 144) == 48           # 144 kept - 96 persistent
+    assert O.cag_topk(0.9, 288, 96, 144) == 0            # the persistent blocks already exceed the share
+    assert O.cag_topk(0.75, 100, 10, 200) == 15          # round(25) - 10
