@@ -261,7 +261,7 @@ def run_train(P, I, dev, steps: int, peaks):
                     "the deterministic kernels recompute S and dP in both the dQ and the dK/dV passes"}
 
 
-def run_rollout(P, I, dev, w, max_chunks=None):
+def run_rollout(P, I, dev, w, max_chunks=None, k_schedule=None, label=None):
     """A whole rollout through the layer caches: ``w.layers`` layers, ``w.steps`` denoising
     steps per chunk sharing the persistent memory, the memory update once per finished chunk.
 
@@ -272,7 +272,8 @@ def run_rollout(P, I, dev, w, max_chunks=None):
     """
     H, d, bpf = w.heads, w.head_dim, w.blocks_per_frame
     cfg = P.LayerConfig(H, d, w.frame_h, w.frame_w, w.tile_h, w.tile_w, w.capacity, w.window_frames,
-                        w.chunk_frames, w.topk, w.gamma, w.dtype, 0)
+                        w.chunk_frames, w.topk, w.gamma, w.dtype, 0,
+                        max_topk=w.window_frames * bpf if k_schedule is not None else -1)
     torch.cuda.synchronize(dev)
     base_alloc = torch.cuda.memory_allocated(dev)
     caches = [P.PBSALayerCache(cfg, dev) for _ in range(w.layers)]
@@ -310,6 +311,9 @@ def run_rollout(P, I, dev, w, max_chunks=None):
     per_chunk, flops_chunk, o = [], [], None
     peak_alloc = 0
     for c, (f0, nf) in enumerate(chunks):
+        if k_schedule is not None:
+            for ca in caches:
+                ca.set_topk(k_schedule[c])
         inp = draw(nf)
         if o is None or o.shape[0] != nf * w.tokens_per_frame:
             o = torch.empty((nf * w.tokens_per_frame, H, d), dtype=torch.bfloat16, device=dev)
@@ -338,8 +342,11 @@ def run_rollout(P, I, dev, w, max_chunks=None):
     steady = [i for i in range(len(chunks)) if i >= min(4, len(chunks) - 1)]
     ms_steady = statistics.mean(per_chunk[i] for i in steady)
     tf_steady = sum(flops_chunk[i] for i in steady) / (sum(per_chunk[i] for i in steady) * 1e-3) / 1e12
+    total_ms, total_flops = sum(per_chunk), sum(flops_chunk)
     return {
-        "workload": w.name, "layers": w.layers, "steps_per_chunk": w.steps, "chunks": len(chunks),
+        "workload": w.name + (f" ({label})" if label else ""), "layers": w.layers, "steps_per_chunk": w.steps,
+        "chunks": len(chunks), "local_topk_per_chunk": list(k_schedule) if k_schedule is not None else w.topk,
+        "ms_total": total_ms, "selected_tflop_total": total_flops / 1e12,
         "ms_per_chunk": [round(x, 3) for x in per_chunk],
         "ms_per_chunk_steady": ms_steady, "steady_chunks": f"{steady[0]}..{steady[-1]}",
         "selected_tflops_steady": tf_steady,
@@ -553,7 +560,13 @@ def run_pbsa(args, w, rank, world, local_rank):
     line["variants"] = [run_variant(P, I, dev, w, max(5, args.steps // 2), hsa_top_frames=3, hsa_recent=1),
                         run_variant(P, I, dev, w, max(5, args.steps // 2), own_chunk=True)]
     if not args.no_rollout:
-        line["rollouts"] = [run_rollout(P, I, dev, I.ROLLOUT_5S), run_rollout(P, I, dev, I.ROLLOUT_1MIN)]
+        from block_sparse_attention_pbsa_b200 import schedule as S
+        w5 = I.ROLLOUT_5S
+        ks, _, _ = S.rollout_topk(I.rollout_chunks(w5), w5.tokens_per_frame, w5.blocks_per_frame, w5.head_dim,
+                                  w5.capacity, w5.window_frames, 0.7, 0.5)
+        line["rollouts"] = [run_rollout(P, I, dev, w5), run_rollout(P, I, dev, I.ROLLOUT_1MIN),
+                            run_rollout(P, I, dev, w5, k_schedule=ks,
+                                        label="per-chunk top-k, chunk-aware growth s_base 0.7 -> s_target 0.5")]
     if world == 1 and not args.no_cpu_baseline:
         t, desc, threads = oracle_sample(w, q, k, v, units=24)
         line["cpu_baseline"] = {"value": flops / t / 1e12, "unit": "TFLOP/s", "cores": threads,

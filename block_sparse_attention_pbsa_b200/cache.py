@@ -47,6 +47,8 @@ class LayerConfig:
     # their ring positions at the current step before the selection (the chunk-wise
     # self-attention of the trainable path, applied at inference)
     own_chunk: bool = False
+    # largest local top-k a per-chunk schedule may set (set_topk); -1: topk
+    max_topk: int = -1
 
     @property
     def bpf(self) -> int:
@@ -81,7 +83,9 @@ class PBSALayerCache:
         self.max_pool_entries = C + max(self.ring_frames * bpf, cfg.staging_blocks)
         self.ws = torch.zeros(L.pbsa_workspace_bytes(self.geom, nq, self.max_pool_entries),
                               dtype=torch.uint8, device=dev)
-        self.kv_ld = C + max(cfg.topk, 0) + (nq if cfg.own_chunk else 0)
+        self.topk = cfg.topk
+        self.max_topk = max(cfg.topk, cfg.max_topk)
+        self.kv_ld = C + max(self.max_topk, 0) + (nq if cfg.own_chunk else 0)
         self.kv_ld_own = max(self.kv_ld, nq)
         # flat buffers, viewed per call as [H, nq, ...] for chunks of up to chunk_frames frames
         self._q_reps_buf = torch.zeros(H * nq * d, dtype=torch.float32, device=dev)
@@ -177,10 +181,16 @@ class PBSALayerCache:
                                 self.p_list, self.p_cnt, c.capacity, self.kv_slot, self.kv_cnt,
                                 self.kv_ld_own, ws=self.ws, stream=stream)
         else:
-            L.pbsa_score_select(self.geom, q_reps, nq, self.k_reps, self.pool_slots, cs, cg, n, c.topk,
+            L.pbsa_score_select(self.geom, q_reps, nq, self.k_reps, self.pool_slots, cs, cg, n, self.topk,
                                 self.p_list, self.p_cnt, c.capacity, self.kv_slot, self.kv_cnt,
                                 self.kv_ld_own, ws=self.ws, stream=stream)
         return self.kv_slot, self.kv_cnt, self.kv_ld_own
+
+    def set_topk(self, k: int):
+        """Local top-k of the following selections (a per-chunk schedule; at most max_topk)."""
+        if not 0 <= k <= self.max_topk:
+            raise ValueError(f"top-k must lie in [0, {self.max_topk}], got {k}")
+        self.topk = int(k)
 
     def query_select(self, q: torch.Tensor, stream=None):
         """a1 + a2 in one launch: q_reps of the chunk and, per query block, persistent slots +
@@ -202,7 +212,7 @@ class PBSALayerCache:
         top = c.hsa_top_frames if (c.hsa_top_frames >= 0 and n) else -1
         own = self._frames_dst(self.hist, nf) if c.own_chunk else None
         L.pbsa_blockify_select_ex(self.geom, q, nf, q_reps, self.k_reps, self.pool_slots, cs, cg, n,
-                                  c.topk if n else 0, top, c.hsa_recent, self.p_list, self.p_cnt, c.capacity,
+                                  self.topk if n else 0, top, c.hsa_recent, self.p_list, self.p_cnt, c.capacity,
                                   own, own.numel() if own is not None else 0, kv_slot, kv_cnt, kv_ld,
                                   ws=self.ws, stream=stream)
 
@@ -400,7 +410,7 @@ class ChunkDecodeStep:
             L.pbsa_blockify(g, q, self.q_frames, self.q_reps, self.nq, ws=ws, stream=stream)
             if not own:
                 mk(1)
-            L.pbsa_score_select(g, self.q_reps, self.nq, ca.k_reps, ps, cs, cg, n, c.topk if n else 0,
+            L.pbsa_score_select(g, self.q_reps, self.nq, ca.k_reps, ps, cs, cg, n, ca.topk if n else 0,
                                 ca.p_list, ca.p_cnt, c.capacity, self.kv_slot, self.kv_cnt, ca.kv_ld,
                                 ws=ws, stream=stream)
         mk(2)

@@ -16,11 +16,11 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def layer_cfg(w, staging=0, hsa=None, own_chunk=False):
+def layer_cfg(w, staging=0, hsa=None, own_chunk=False, max_topk=-1):
     top, recent = hsa if hsa is not None else (-1, 1)
     return P.LayerConfig(w.heads, w.head_dim, w.frame_h, w.frame_w, w.tile_h, w.tile_w, w.capacity,
                          w.window_frames, w.chunk_frames, w.topk, w.gamma, w.dtype, staging,
-                         hsa_top_frames=top, hsa_recent=recent, own_chunk=own_chunk)
+                         hsa_top_frames=top, hsa_recent=recent, own_chunk=own_chunk, max_topk=max_topk)
 
 
 def _decode_single_step(w, sample_units=None, hsa=None, own_chunk=False):
@@ -130,11 +130,12 @@ def test_decode_tiny_own_chunk():
     _decode_single_step(I.TINY, own_chunk=True)
 
 
-def _rollout(w, n_chunks, sample_every=3):
+def _rollout(w, n_chunks, sample_every=3, k_schedule=None):
     """Layer-0 rollout: GPU cache vs the oracle state machine, chunk by chunk.  A head whose
-    memory-update boundary was a near tie is compared no further (both outcomes are valid)."""
+    memory-update boundary was a near tie is compared no further (both outcomes are valid).
+    ``k_schedule``: a local top-k per chunk (set on both sides before the chunk)."""
     bpf = w.blocks_per_frame
-    cache = P.PBSALayerCache(layer_cfg(w))
+    cache = P.PBSALayerCache(layer_cfg(w, max_topk=w.window_frames * bpf if k_schedule else -1))
     ro = O.RolloutOracle(geom_dict(w), w.heads, w.capacity, w.window_frames, w.topk, w.gamma)
     gd = geom_dict(w)
     alive = [True] * w.heads
@@ -145,6 +146,9 @@ def _rollout(w, n_chunks, sample_every=3):
     chunks = I.rollout_chunks(w)[:n_chunks]
     for c, (f0, nf) in enumerate(chunks):
         assert nf == w.chunk_frames or c == 0
+        if k_schedule is not None:
+            cache.set_topk(k_schedule[c])
+            ro.k = k_schedule[c]
         wc = dataclasses.replace(w, chunk_frames=nf)
         for s in range(w.steps):
             seeds = [I.stream_seed(w.seed, c, s, t) for t in range(3)]
@@ -204,6 +208,17 @@ def _rollout(w, n_chunks, sample_every=3):
 def test_rollout_5s_layer0():
     w = I.ROLLOUT_5S
     alive = _rollout(w, n_chunks=7)
+    assert sum(alive) >= w.heads // 2
+
+
+def test_rollout_5s_layer0_chunk_topk_schedule():
+    """The 5 s rollout with a per-chunk local top-k from the chunk-aware-growth schedule."""
+    from block_sparse_attention_pbsa_b200 import schedule as S
+    w = I.ROLLOUT_5S
+    ks, _, _ = S.rollout_topk(I.rollout_chunks(w), w.tokens_per_frame, w.blocks_per_frame, w.head_dim,
+                              w.capacity, w.window_frames, 0.7, 0.5)
+    assert len(set(ks[1:])) > 2       # the schedule really varies
+    alive = _rollout(w, n_chunks=7, k_schedule=ks)
     assert sum(alive) >= w.heads // 2
 
 
