@@ -441,6 +441,62 @@ class ChunkDecodeStep:
         torch.cuda.current_stream(self.cache.device).wait_stream(side)
         return graph
 
+    def capture_pipeline(self, q, k, v, o, lse=None):
+        """Capture the step as two graphs for ``run_pipelined``: [blockify(Q) + selection +
+        attend] and [commit blockify(K, V) + memory update] (the own-chunk variant, which needs
+        K, V before the selection, is not split)."""
+        if self.cache.cfg.own_chunk:
+            raise ValueError("the own-chunk variant writes K, V before the selection: use capture()")
+        dev = self.cache.device
+        front, back = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        ca, c = self.cache, self.cache.cfg
+        g, ws, ps = ca.geom, ca.ws, ca.pool_slots
+        with torch.cuda.graph(front, stream=side):
+            ca._select_fused(q, self.q_frames, self.q_reps, self.kv_slot, self.kv_cnt, ca.kv_ld)
+            L.pbsa_attend(g, q, self.q_frames, ca.k_pool, ca.v_pool, ps, self.kv_slot, self.kv_cnt, ca.kv_ld,
+                          o, lse, ws=ws)
+        with torch.cuda.graph(back, stream=side):
+            L.pbsa_blockify(g, k, self.q_frames, ca.k_reps, ps, self.dst, ca.k_pool, ps, ws=ws)
+            L.pbsa_blockify(g, v, self.q_frames, self.vreps, ps, self.dst, ca.v_pool, ps, ws=ws)
+            L.pbsa_memory_update(g, self.q_reps, self.nq, ca.k_reps, ca.k_pool, ca.v_pool, ps, ca.slot_gid,
+                                 ca.slot_ema, c.capacity, c.bpf, self.cs, self.cg, self.ncand, c.gamma,
+                                 ca.p_list, ca.p_cnt, ws=ws)
+        torch.cuda.current_stream(dev).wait_stream(side)
+        self._pipe = {"front": front, "back": back, "bufs": (q, k, v, o),
+                      "h2d": torch.cuda.Stream(device=dev), "d2h": torch.cuda.Stream(device=dev)}
+
+    def run_pipelined(self, qh, kh, vh, oh):
+        """One step from pinned host buffers to a pinned host result, with the transfers
+        overlapped: Q is uploaded first and the front graph (selection + attention) starts as
+        soon as it lands, while K and V upload on a copy stream (only the commit needs them);
+        O downloads on another stream while the commit and memory update run.  All work is
+        ordered on the current stream's timeline when this returns (asynchronously)."""
+        p = self._pipe
+        q, k, v, o = p["bufs"]
+        main = torch.cuda.current_stream(self.cache.device)
+        h2d, d2h = p["h2d"], p["d2h"]
+        h2d.wait_stream(main)                       # previous step done with k, v, q
+        d2h.wait_stream(main)
+        with torch.cuda.stream(h2d):
+            q.copy_(qh, non_blocking=True)
+            q_done = torch.cuda.Event()
+            q_done.record(h2d)
+            k.copy_(kh, non_blocking=True)
+            v.copy_(vh, non_blocking=True)
+        main.wait_event(q_done)
+        p["front"].replay()
+        front_done = torch.cuda.Event()
+        front_done.record(main)
+        with torch.cuda.stream(d2h):
+            d2h.wait_event(front_done)
+            oh.copy_(o, non_blocking=True)
+        main.wait_stream(h2d)                       # K, V uploaded
+        p["back"].replay()
+        main.wait_stream(d2h)                       # O downloaded
+        return oh
+
     def snapshot(self):
         """Copies of everything ``run`` mutates outside the chunk's own ring positions."""
         ca, C = self.cache, self.cache.cfg.capacity

@@ -226,3 +226,34 @@ def test_rollout_5s_layer0_chunk_topk_schedule():
 def test_rollout_1min_layer0_first_chunks():
     w = dataclasses.replace(I.ROLLOUT_1MIN, total_frames=1 + 3 * 12)
     _rollout(w, n_chunks=13, sample_every=4)
+
+
+def test_pipelined_host_step_matches_the_graph_step():
+    """ChunkDecodeStep.run_pipelined (transfers overlapped with the kernels) gives the same O and
+    the same persistent memory as the single-graph step on the same inputs."""
+    w = I.DECODE_5S
+    q, k, v = I.single_step(w)
+    kc = I.tokens(w, w.chunk_frames, I.stream_seed(w.seed, 4))
+    vc = I.tokens(w, w.chunk_frames, I.stream_seed(w.seed, 5))
+    bpf = w.blocks_per_frame
+    cache = P.PBSALayerCache(layer_cfg(w, (w.hist_frames - w.window_frames) * bpf))
+    qd, kcd, vcd = q.to(DEV), kc.to(DEV), vc.to(DEV)
+    cache.prefill(k.to(DEV), v.to(DEV), w.hist_frames, cache.query_reps(qd))
+    step = P.ChunkDecodeStep(cache)
+    snap = step.snapshot()
+    o = torch.empty_like(qd)
+    step.run(qd, kcd, vcd, o)
+    want_o = o.cpu()
+    want_gid = cache.slot_gid.cpu()
+    step.restore(snap)
+    qb, kb, vb, ob = (torch.empty_like(t) for t in (qd, kcd, vcd, o))
+    step.capture_pipeline(qb, kb, vb, ob)
+    qh, kh, vh = (t.pin_memory() for t in (q, kc, vc))
+    oh = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    for _ in range(2):
+        step.restore(snap)
+        step.run_pipelined(qh, kh, vh, oh)
+        torch.cuda.synchronize()
+        assert torch.equal(oh, want_o)
+        assert torch.equal(cache.slot_gid.cpu(), want_gid)
+    assert P.pbsa_get_device_error(cache.ws) == 0
