@@ -26,8 +26,8 @@
 //    pipe), so one warpgroup's exponentials overlap the other's MMAs.
 //  * O_w is rescaled only when its running max grows by more than 2^8; the epilogue
 //    merges the two streams exactly.
-//  * Register split: the producer/issuer warpgroup runs on 56 registers, the softmax
-//    warpgroups on 224 (setmaxnreg), so the softmax holds its row in registers.
+//  * Register split: the producer/issuer warpgroup runs on 64 registers, the softmax
+//    warpgroups on 216 (setmaxnreg), so the softmax holds its row in registers.
 //  * Every wait is bounded; on expiry the kernel records PBSA_ERR_TIMEOUT in the
 //    workspace, drains its own copies and MMAs, frees TMEM and returns.
 #include <math.h>
@@ -44,7 +44,7 @@ constexpr int D = 128;
 constexpr int MAXL = 1024;           // merged list capacity (two lists of <= 512)
 constexpr int NTHREADS = 384;        // warpgroup 0: producer + MMA; 1, 2: softmax
 constexpr int KSTAGES = 3, VSTAGES = 2;
-constexpr uint32_t REG_CTRL = 56, REG_SOFTMAX = 224;   // 128*56 + 256*224 = 384*168
+constexpr uint32_t REG_CTRL = 64, REG_SOFTMAX = 216;   // 128*64 + 256*216 = 384*165
 static_assert(128 * REG_CTRL + 256 * REG_SOFTMAX <= NTHREADS * 168, "register split exceeds launch budget");
 
 // shared memory map (offsets from a 1024-byte aligned base)

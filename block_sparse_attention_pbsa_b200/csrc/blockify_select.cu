@@ -255,6 +255,265 @@ __global__ void __launch_bounds__(BS_THREADS) blockify_select_kernel(
   }
 }
 
+// ---------------------------------------------------------------------------- 8-block form
+// The flat policy with up to 256 candidates: one CTA of 512 threads per (head, 8 query blocks).
+//  1. every thread issues the 16-byte token loads of its four (block, column chunk, row set)
+//     shares -- the blockify split, so each block's mean is summed in blockify's order -- and
+//     the candidate list; then the candidates' representatives are staged in shared memory;
+//  2. warp w scores candidates w, w+16, ... against all 8 pooled queries at once: each lane
+//     holds d/32 elements of the 8 queries and of the candidate, and a transposing butterfly
+//     (9 shuffles for the 8 sums, fixed order) leaves each lane group one query's score;
+//  3. warp b sorts query block b's keys in registers (bitonic, 8 per lane, no block-wide
+//     barrier) and writes the first k.
+constexpr int S8_R = 8, S8_THREADS = 512;
+
+template <typename T, int D>
+__global__ void __launch_bounds__(S8_THREADS) blockify_select8_kernel(
+    const T* __restrict__ x, Geo g, int nq, float* __restrict__ q_reps,
+    const float* __restrict__ k_reps, int pool_slots, const int* __restrict__ cand_slot,
+    const int* __restrict__ cand_gid, int ncand, int k, const int* __restrict__ prefix_slot,
+    const int* __restrict__ prefix_cnt, int prefix_ld, int* __restrict__ out_slot,
+    int* __restrict__ out_cnt, int out_ld, float* __restrict__ out_score,
+    const int* __restrict__ suffix_slot, int suffix_n, void* ws) {
+  constexpr int VEC = 16 / sizeof(T);
+  constexpr int CPR = D / VEC;            // chunks per token row
+  constexpr int RPP = BS_THREADS / CPR;   // rows per pass of a 256-thread blockify share
+  constexpr int PASSES = BT / RPP;
+  constexpr int PL = D / 32;
+  constexpr int NW = S8_THREADS / 32;
+  using V = typename Vec<PL>::type;
+  extern __shared__ __align__(16) float sm8[];
+  float* part = sm8;                                   // [S8_R][RPP][D]
+  float* kb = part + S8_R * RPP * D;                   // [ncand][D]
+  float* qb = kb + (size_t)ncand * D;                  // [S8_R][D]
+  float* sc = qb + S8_R * D;                           // [S8_R][ncand]
+  int* slot = reinterpret_cast<int*>(sc + S8_R * ncand);   // [ncand]
+  int* gid = slot + ncand;                                  // [ncand]
+
+  const int h = blockIdx.y, r0 = blockIdx.x * S8_R;
+  const int nr = min(S8_R, nq - r0);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  // ---- 1. token loads: thread = (virtual blockify thread vt, block parity); blocks bp, bp+2, ..
+  const int vt = tid % BS_THREADS, bp = tid / BS_THREADS;
+  const int c = vt % CPR, rg = vt / CPR;
+  uint4 v[S8_R / 2][PASSES];
+#pragma unroll
+  for (int u = 0; u < S8_R / 2; ++u) {
+    const int b = bp + 2 * u;
+    const int r = r0 + min(b, nr - 1);     // a missing block re-reads the last one (not stored)
+    const int f = r / g.bpf, rem = r - f * g.bpf;
+    const int ty = rem / g.tpr, tx = rem - ty * g.tpr;
+#pragma unroll
+    for (int p = 0; p < PASSES; ++p) {
+      const int row = rg + p * RPP;
+      const int ly = row / g.tw, lx = row - ly * g.tw;
+      const size_t t = (size_t)f * g.tpf + (size_t)(ty * g.th + ly) * g.fw + tx * g.tw + lx;
+      v[u][p] = __ldg(reinterpret_cast<const uint4*>(x + (t * g.H + h) * D) + c);
+    }
+  }
+  for (int j = tid; j < ncand; j += S8_THREADS) {
+    gid[j] = cand_gid[(size_t)h * ncand + j];
+    slot[j] = cand_slot[(size_t)h * ncand + j];
+  }
+#pragma unroll
+  for (int u = 0; u < S8_R / 2; ++u) {
+    float acc[VEC];
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) acc[i] = 0.f;
+#pragma unroll
+    for (int p = 0; p < PASSES; ++p) add_chunk16<T>(acc, v[u][p]);
+    float* pr = part + ((bp + 2 * u) * RPP + rg) * D + c * VEC;
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) pr[i] = acc[i];
+  }
+  __syncthreads();
+  // candidate representatives -> shared memory (all rows' 16-byte loads in flight)
+  {
+    constexpr int F4 = D / 4;
+    for (int base = tid; base < ncand * F4; base += S8_THREADS * 8) {
+      float4 buf[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = base + u * S8_THREADS;
+        buf[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (i < ncand * F4) {
+          const int s = slot[i / F4];
+          if (s >= 0 && s < pool_slots)
+            buf[u] = __ldg(reinterpret_cast<const float4*>(k_reps + ((size_t)h * pool_slots + s) * D) + (i % F4));
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = base + u * S8_THREADS;
+        if (i < ncand * F4) reinterpret_cast<float4*>(kb)[i] = buf[u];
+      }
+    }
+  }
+  // qbar (fixed-order sums, as in the blockify kernel)
+  for (int i = tid; i < S8_R * D; i += S8_THREADS) {
+    const int b = i / D, e = i - b * D;
+    float s = 0.f;
+#pragma unroll 4
+    for (int q = 0; q < RPP; ++q) s += part[(b * RPP + q) * D + e];
+    s *= (1.0f / BT);
+    qb[i] = s;
+    if (b < nr) q_reps[((size_t)h * nq + r0 + b) * D + e] = s;
+  }
+  __syncthreads();
+
+  // ---- 2. scores: warp per candidate, all 8 queries at once
+  float ql[S8_R][PL];
+#pragma unroll
+  for (int b = 0; b < S8_R; ++b)
+#pragma unroll
+    for (int i = 0; i < PL; ++i) ql[b][i] = qb[b * D + lane * PL + i];
+  for (int cc = warp; cc < ncand; cc += NW) {
+    float kv[PL];
+    vec_to(reinterpret_cast<const V*>(kb + (size_t)cc * D)[lane], kv);
+    float a[S8_R];
+#pragma unroll
+    for (int b = 0; b < S8_R; ++b) {
+      a[b] = 0.f;
+#pragma unroll
+      for (int i = 0; i < PL; ++i) a[b] = fmaf(ql[b][i], kv[i], a[b]);
+    }
+    // transposing butterfly: after the xor-16/8/4 exchanges lane l holds query
+    // ((l >> 2) & 7)'s partial over 4 lanes; xor-2/1 finish the sum
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {          // xor 16: keep 4 of 8
+      const bool up = lane & 16;
+      const float send = up ? a[j] : a[j + 4];
+      const float keep = up ? a[j + 4] : a[j];
+      a[j] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+    }
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {          // xor 8: keep 2 of 4
+      const bool up = lane & 8;
+      const float send = up ? a[j] : a[j + 2];
+      const float keep = up ? a[j + 2] : a[j];
+      a[j] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    }
+    {                                      // xor 4: keep 1 of 2
+      const bool up = lane & 4;
+      const float send = up ? a[0] : a[1];
+      const float keep = up ? a[1] : a[0];
+      a[0] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+    }
+    a[0] += __shfl_xor_sync(0xffffffffu, a[0], 2);
+    a[0] += __shfl_xor_sync(0xffffffffu, a[0], 1);
+    if ((lane & 3) == 0) {
+      // lane bits 4, 3, 2 picked halves (upper half = higher index) in that order
+      const int b = ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
+      float val = a[0] * g.scale;
+      const int s = slot[cc];
+      if (s < 0 || s >= pool_slots) {
+        if (b == 0 && r0 == 0) record_error(ws, PBSA_ERR_DEVICE_INDEX, s, K_SCORE);
+        val = -INFINITY;
+      }
+      if (isnan(val)) val = -INFINITY;
+      sc[b * ncand + cc] = val;
+    }
+  }
+  int pc = prefix_cnt ? prefix_cnt[h] : 0;
+  if (pc < 0 || pc > prefix_ld) {
+    if (tid == 0 && r0 == 0) record_error(ws, PBSA_ERR_DEVICE_INDEX, pc, K_SCORE);
+    pc = pc < 0 ? 0 : prefix_ld;
+  }
+  const int kk = min(k, ncand);
+  for (int i = tid; i < nr * (pc + suffix_n); i += S8_THREADS) {
+    const int b = i / (pc + suffix_n), j = i - b * (pc + suffix_n);
+    const size_t o = (size_t)h * nq + r0 + b;
+    out_slot[o * out_ld + (j < pc ? j : kk + j)] = j < pc ? prefix_slot[(size_t)h * prefix_ld + j] : suffix_slot[j - pc];
+  }
+  if (tid < nr) out_cnt[(size_t)h * nq + r0 + tid] = pc + kk + suffix_n;
+  __syncthreads();
+
+  // ---- 3. warp b selects query block b's k best: element e = j*32 + lane (j < 8).  A radix
+  // search finds the k-th largest key (score bits first; the gid bits only on an exact score
+  // tie), so exactly k elements are chosen, then each chosen element's rank among the chosen
+  // is counted and it is written at that rank.
+  if (warp < nr) {
+    const int b = warp;
+    uint64_t kv8[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = j * 32 + lane;
+      kv8[j] = e < ncand ? rank_key(sc[b * ncand + e], gid[e]) : 0ull;
+    }
+    // k-th largest of the high words (score order keys)
+    auto count_hi_ge = [&](uint32_t t) {
+      int n = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) n += (uint32_t)(kv8[j] >> 32) >= t;
+      return __reduce_add_sync(0xffffffffu, n);
+    };
+    uint32_t th = 0;
+    if (kk > 0) {
+#pragma unroll 1
+      for (int bit = 31; bit >= 0; --bit) {
+        const uint32_t t2 = th | (1u << bit);
+        if (count_hi_ge(t2) >= kk) th = t2;
+      }
+    }
+    int n_gt = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) n_gt += (uint32_t)(kv8[j] >> 32) > th;
+    n_gt = __reduce_add_sync(0xffffffffu, n_gt);
+    // among the keys whose high word equals th, the (kk - n_gt)-th largest low word (gid)
+    const int need = kk - n_gt;
+    auto count_lo_ge = [&](uint32_t t) {
+      int n = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) n += ((uint32_t)(kv8[j] >> 32) == th) && ((uint32_t)kv8[j] >= t);
+      return __reduce_add_sync(0xffffffffu, n);
+    };
+    uint32_t tl = 0;
+    if (need > 0 && count_lo_ge(0) > need) {
+#pragma unroll 1
+      for (int bit = 31; bit >= 0; --bit) {
+        const uint32_t t2 = tl | (1u << bit);
+        if (count_lo_ge(t2) >= need) tl = t2;
+      }
+    }
+    const uint64_t tkey = ((uint64_t)th << 32) | tl;
+    int n_above = 0;   // keys strictly above the k-th key
+#pragma unroll
+    for (int j = 0; j < 8; ++j) n_above += kv8[j] > tkey;
+    n_above = __reduce_add_sync(0xffffffffu, n_above);
+    // chosen: every key above tkey, then keys equal to tkey in position order (exact
+    // duplicates of (score, gid) only)
+    int* chosen = reinterpret_cast<int*>(part) + b * 256;    // part is free after the pooling
+    int eq_seen = 0, n_ch = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const bool eq = kk > 0 && kv8[j] == tkey;
+      const unsigned eb = __ballot_sync(0xffffffffu, eq);
+      const bool take_eq = eq && (eq_seen + __popc(eb & ((1u << lane) - 1u)) < kk - n_above);
+      eq_seen += __popc(eb);
+      const bool take = (kk > 0 && kv8[j] > tkey) || take_eq;
+      const unsigned tb = __ballot_sync(0xffffffffu, take);
+      if (take) chosen[n_ch + __popc(tb & ((1u << lane) - 1u))] = j * 32 + lane;
+      n_ch += __popc(tb);
+    }
+    __syncwarp();
+    // rank among the chosen: larger key first, then the lower position
+    const size_t o = (size_t)h * nq + r0 + b;
+    for (int t = lane; t < n_ch; t += 32) {
+      const int e = chosen[t];
+      const uint64_t ke = rank_key(sc[b * ncand + e], gid[e]);
+      int rank = 0;
+      for (int u = 0; u < n_ch; ++u) {
+        const int e2 = chosen[u];
+        const uint64_t k2 = rank_key(sc[b * ncand + e2], gid[e2]);
+        rank += (k2 > ke) | ((k2 == ke) & (e2 < e));
+      }
+      out_slot[o * out_ld + pc + rank] = slot[e];
+      if (out_score) out_score[o * k + rank] = sc[b * ncand + e];
+    }
+  }
+}
+
 template <typename T, int D, bool HSA>
 cudaError_t launch_t(const Geo& g, const void* x, int q_frames, float* q_reps, const float* k_reps,
                      int pool_slots, const int* cand_slot, const int* cand_gid, int ncand, int k,
@@ -262,6 +521,18 @@ cudaError_t launch_t(const Geo& g, const void* x, int q_frames, float* q_reps, c
                      int* out_cnt, int out_ld, float* out_score, int top_frames, int n_recent,
                      const int* suffix_slot, int suffix_n, void* ws, cudaStream_t st) {
   const int nq = q_frames * g.bpf;
+  if (!HSA && ncand <= 256) {
+    constexpr int RPP = BS_THREADS / (D / (16 / (int)sizeof(T)));
+    const size_t smem8 = ((size_t)S8_R * RPP * D + (size_t)ncand * D + (size_t)S8_R * D +
+                          (size_t)S8_R * ncand) * 4 + (size_t)ncand * 8;
+    auto kern8 = blockify_select8_kernel<T, D>;
+    cudaError_t e = set_smem_once((const void*)kern8, (int)smem8);
+    if (e != cudaSuccess) return e;
+    kern8<<<dim3((nq + S8_R - 1) / S8_R, g.H), S8_THREADS, smem8, st>>>(
+        static_cast<const T*>(x), g, nq, q_reps, k_reps, pool_slots, cand_slot, cand_gid, ncand, k,
+        prefix_slot, prefix_cnt, prefix_ld, out_slot, out_cnt, out_ld, out_score, suffix_slot, suffix_n, ws);
+    return cudaGetLastError();
+  }
   const size_t smem = (size_t)ncand * (8 + 4 + 4 + 4);
   auto kern = blockify_select_kernel<T, D, HSA>;
   cudaError_t e = set_smem_once((const void*)kern, (int)(smem > 0 ? smem : 8));
