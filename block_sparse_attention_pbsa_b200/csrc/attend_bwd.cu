@@ -227,7 +227,8 @@ constexpr uint32_t Q_SMEM_BYTES = Q_SM_ONLYB + 512 + 1024;
 enum { QB_QFULL = 0, QB_KFULL = 1, QB_KEMPTY = QB_KFULL + QK_STAGES, QB_VFULL = QB_KEMPTY + QK_STAGES,
        QB_VEMPTY = QB_VFULL + 1, QB_SFULL = QB_VEMPTY + 1 /* [i&1] */,
        QB_PFULL = QB_SFULL + 2 /* [w][i&1], 128 arrivals */, QB_DPFREE = QB_PFULL + 4 /* 256 arrivals */,
-       QB_MMADONE = QB_DPFREE + 1, QB_NUM = QB_MMADONE + 1 };
+       QB_SBFREE = QB_DPFREE + 1 /* [i&1]: dQ(i) has read dS(i) */, QB_MMADONE = QB_SBFREE + 2 /* 2 arrivals */,
+       QB_NUM = QB_MMADONE + 1 };
 
 struct DqParams {
   BwdGeo g;
@@ -264,6 +265,7 @@ __global__ void __launch_bounds__(NT, 1)
     for (int i = 0; i < QB_NUM; ++i) mbar_init(&bars[i], 1);
     for (int i = 0; i < 4; ++i) mbar_init(&bars[QB_PFULL + i], 128);
     mbar_init(&bars[QB_DPFREE], 256);
+    mbar_init(&bars[QB_MMADONE], 2);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -348,20 +350,23 @@ __global__ void __launch_bounds__(NT, 1)
       }
       if (*abort_flag && viss > 0) mbar_wait(&bars[QB_VFULL], (viss - 1) & 1, kWaitLimitNs);
     }
+    // ---- MMA issuers.  TMEM: S[i&1] at 128*(i&1), dP at 256, dQ at 384.
+    // Warp 1 issues S(i) (once dQ(i-2) has read the dS over S[i&1]) and dP(i) (once the
+    // warpgroups hold dP(i-1) in registers), so the tensor pipe computes S(i+1) and dP(i+1)
+    // while the warpgroups form dS(i).  Warp 3 issues dQ += dS(i) K(i) for every step in
+    // order, one thread, so dQ accumulates in a fixed order.
     if (warp == 1 && lane == 0 && nsteps > 0) {
-      // ---- MMA issuer.  TMEM: S[i&1] at 128*(i&1), dP at 256, dQ at 384.
-      // Per step: the next S and, as soon as the warpgroups have read dP(i) into registers,
-      // the next dP; then dQ += dS(i) K(i) once dS(i) is in TMEM.  So the tensor pipe computes
-      // S(i+1) and dP(i+1) while the warpgroups form dS(i).
       const uint64_t dq_ = sw128_desc(smem_u32(sm + Q_SM_Q), 16, 1024);
       const uint64_t ddo = sw128_desc(smem_u32(sm + Q_SM_DO), 16, 1024);
       const uint64_t dk = sw128_desc(smem_u32(sm + Q_SM_K), 16, 1024);
       const uint64_t dv = sw128_desc(smem_u32(sm + Q_SM_V), 16, 1024);
-      const uint64_t dk_mn = sw128_desc(smem_u32(sm + Q_SM_K), 16384, 1024);
-      auto issue_s = [&](int i) {   // S(i) = Q K(i)^T into S[i&1]
+      wait_or_abort(&bars[QB_QFULL], 0, abort_flag, prm.ws, 4, K_BWD_Q);
+      for (int i = 0; i < nsteps && !*abort_flag; ++i) {
         const int sk = i % QK_STAGES;
+        // S(i) = Q K(i)^T into S[i&1]
+        if (i >= 2) wait_or_abort(&bars[QB_SBFREE + (i & 1)], ((i - 2) >> 1) & 1, abort_flag, prm.ws, 10, K_BWD_Q);
         wait_or_abort(&bars[QB_KFULL + sk], (i / QK_STAGES) & 1, abort_flag, prm.ws, 5, K_BWD_Q);
-        if (*abort_flag) return;
+        if (*abort_flag) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
@@ -369,10 +374,10 @@ __global__ void __launch_bounds__(NT, 1)
           mma_bf16_ss(tmem + (i & 1) * 128, dq_ + off, dk + ((sk * 32768) >> 4) + off, IDESC_KMAJ,
                       kk > 0 ? 1u : 0u);
         }
-      };
-      auto issue_dp = [&](int i) {  // dP(i) = dO V(i)^T, then V's stage is free
+        // dP(i) = dO V(i)^T, then V's stage is free
+        if (i >= 1) wait_or_abort(&bars[QB_DPFREE], (i - 1) & 1, abort_flag, prm.ws, 9, K_BWD_Q);
         wait_or_abort(&bars[QB_VFULL], i & 1, abort_flag, prm.ws, 6, K_BWD_Q);
-        if (*abort_flag) return;
+        if (*abort_flag) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
@@ -380,22 +385,18 @@ __global__ void __launch_bounds__(NT, 1)
           mma_bf16_ss(tmem + 256, ddo + off, dv + off, IDESC_KMAJ, kk > 0 ? 1u : 0u);
         }
         mma_commit(&bars[QB_VEMPTY]);
-      };
-      wait_or_abort(&bars[QB_QFULL], 0, abort_flag, prm.ws, 4, K_BWD_Q);
-      issue_s(0);
-      issue_dp(0);
-      mma_commit(&bars[QB_SFULL + 0]);
+        mma_commit(&bars[QB_SFULL + (i & 1)]);
+      }
+      mma_commit(&bars[QB_MMADONE]);
+      mbar_wait(&bars[QB_MMADONE], 0, kWaitLimitNs);
+    }
+    if (warp == 3 && lane == 0 && nsteps > 0) {
+      const uint64_t dk_mn = sw128_desc(smem_u32(sm + Q_SM_K), 16384, 1024);
       for (int i = 0; i < nsteps && !*abort_flag; ++i) {
         const int s = i & 1, sk = i % QK_STAGES;
-        if (i + 1 < nsteps) {
-          issue_s(i + 1);
-          wait_or_abort(&bars[QB_DPFREE], i & 1, abort_flag, prm.ws, 9, K_BWD_Q);
-          issue_dp(i + 1);
-          mma_commit(&bars[QB_SFULL + ((i + 1) & 1)]);
-          if (*abort_flag) break;
-        }
         // dQ += dS(i) K(i): dS(i) (bf16 pairs) sits over S[s], warpgroup w's 64 keys in its
-        // half; K(i) is the B operand (keys x d, d contiguous)
+        // half; K(i) is the B operand (keys x d, d contiguous).  S(i) completed before dS(i)
+        // was formed, so the commits below cover every MMA that read K(i) and S[s].
         for (int w = 0; w < 2; ++w) {
           wait_or_abort(&bars[QB_PFULL + 2 * w + s], (i >> 1) & 1, abort_flag, prm.ws, 3, K_BWD_Q);
           if (*abort_flag) break;
@@ -407,6 +408,7 @@ __global__ void __launch_bounds__(NT, 1)
                         (i > 0 || w > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(&bars[QB_KEMPTY + sk]);
+        mma_commit(&bars[QB_SBFREE + s]);
       }
       mma_commit(&bars[QB_MMADONE]);
       mbar_wait(&bars[QB_MMADONE], 0, kWaitLimitNs);
@@ -517,7 +519,8 @@ constexpr uint32_t KV_SM_ONLYB = KV_SM_LB + 4 * 512;
 constexpr uint32_t KV_SM_TMP = KV_SM_ONLYB + 512;                    // int[512] sort scratch
 constexpr uint32_t KV_SMEM_BYTES = KV_SM_TMP + 4 * 512 + 1024;
 enum { KB_KVFULL = 0, KB_QFULL = 1, KB_QEMPTY = KB_QFULL + KV_QST, KB_SFULL = KB_QEMPTY + KV_QST /* [b] */,
-       KB_PFULL = KB_SFULL + 2 /* [b], 128 arrivals */, KB_MMADONE = KB_PFULL + 2, KB_NUM = KB_MMADONE + 1 };
+       KB_PFULL = KB_SFULL + 2 /* [b], 128 arrivals */, KB_BFREE = KB_PFULL + 2 /* [b] */,
+       KB_MMADONE = KB_BFREE + 2 /* 2 arrivals */, KB_NUM = KB_MMADONE + 1 };
 constexpr uint32_t IDESC_N64 = idesc_bf16_f32(128, 64, 0, 0);   // S^T, dP^T of one query block
 
 struct DkvParams {
@@ -572,6 +575,7 @@ __global__ void __launch_bounds__(NT, 1)
     for (int i = 0; i < KB_NUM; ++i) mbar_init(&bars[i], 1);
     mbar_init(&bars[KB_PFULL + 0], 128);
     mbar_init(&bars[KB_PFULL + 1], 128);
+    mbar_init(&bars[KB_MMADONE], 2);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -648,17 +652,19 @@ __global__ void __launch_bounds__(NT, 1)
           mbar_wait(&bars[KB_QFULL + j % KV_QST], (j / KV_QST) & 1, kWaitLimitNs);
       }
     }
+    // ---- MMA issuers.  TMEM: S^T[b] at 64 b, dP^T[b] at 128 + 64 b (keys on lanes, 64 queries
+    // each), dV at 256, dK at 384; step j uses buffer b = j & 1.  Warp 1 issues S^T/dP^T(j)
+    // as soon as buffer b is free (the dV/dK MMAs of step j-2 done); warp 3 issues the dV/dK
+    // MMAs of every step in order, one thread, so dV and dK accumulate in a fixed order.
     if (warp == 1 && lane == 0 && nsteps > 0) {
-      // ---- MMA issuer (one thread, so dV and dK accumulate in a fixed order).
-      // TMEM: S^T[b] at 64 b, dP^T[b] at 128 + 64 b (keys on lanes, 64 queries each), dV at 256,
-      // dK at 384.  Step j uses buffer b = j & 1; S^T/dP^T(j+2) go into it right behind the
-      // dV/dK MMAs of step j, while the other warpgroup works on step j+1.
       const uint64_t dk = sw128_desc(smem_u32(sm + KV_SM_K), 16, 1024);
       const uint64_t dv = sw128_desc(smem_u32(sm + KV_SM_V), 16, 1024);
-      auto issue_sdp = [&](int j) {   // S^T = K Q_j^T, dP^T = V dO_j^T (M = 128 keys, N = 64)
+      wait_or_abort(&bars[KB_KVFULL], 0, abort_flag, prm.ws, 2, K_BWD_KV);
+      for (int j = 0; j < nsteps && !*abort_flag; ++j) {   // S^T = K Q_j^T, dP^T = V dO_j^T
         const int s = j % KV_QST, b = j & 1;
+        if (j >= 2) wait_or_abort(&bars[KB_BFREE + b], ((j - 2) >> 1) & 1, abort_flag, prm.ws, 8, K_BWD_KV);
         wait_or_abort(&bars[KB_QFULL + s], (j / KV_QST) & 1, abort_flag, prm.ws, 3, K_BWD_KV);
-        if (*abort_flag) return;
+        if (*abort_flag) break;
         tc_fence_after();
         const uint64_t dq_ = sw128_desc(smem_u32(sm + KV_SM_Q + s * KV_STAGE), 16, 1024);
         const uint64_t ddo = sw128_desc(smem_u32(sm + KV_SM_Q + s * KV_STAGE + 16384), 16, 1024);
@@ -670,17 +676,19 @@ __global__ void __launch_bounds__(NT, 1)
           mma_bf16_ss(tmem + 128 + b * 64, dv + ka, ddo + kb, IDESC_N64, kk > 0 ? 1u : 0u);
         }
         mma_commit(&bars[KB_SFULL + b]);
-      };
-      wait_or_abort(&bars[KB_KVFULL], 0, abort_flag, prm.ws, 2, K_BWD_KV);
-      issue_sdp(0);
-      if (nsteps > 1) issue_sdp(1);
+      }
+      mma_commit(&bars[KB_MMADONE]);
+      mbar_wait(&bars[KB_MMADONE], 0, kWaitLimitNs);
+    }
+    if (warp == 3 && lane == 0 && nsteps > 0) {
       for (int j = 0; j < nsteps && !*abort_flag; ++j) {
         const int s = j % KV_QST, b = j & 1;
         wait_or_abort(&bars[KB_PFULL + b], (j >> 1) & 1, abort_flag, prm.ws, 4, K_BWD_KV);
         if (*abort_flag) break;
         tc_fence_after();
         // dV += P^T dO_j, dK += dS^T Q_j: A from TMEM (bf16 pairs over S^T[b] / dP^T[b]), B =
-        // the query block's 64 rows (d contiguous, two 64-column panels 8 KB apart)
+        // the query block's 64 rows (d contiguous, two 64-column panels 8 KB apart).  S^T/dP^T(j)
+        // completed before P(j) was formed, so these commits also cover them.
         const uint32_t q_base = smem_u32(sm + KV_SM_Q + s * KV_STAGE), do_base = q_base + 16384;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
@@ -689,7 +697,7 @@ __global__ void __launch_bounds__(NT, 1)
           mma_bf16_ts(tmem + 384, tmem + 128 + b * 64 + kk * 8, sw128_desc(q_base + kk * 2048, 8192, 1024), IDESC_BMN, acc);
         }
         mma_commit(&bars[KB_QEMPTY + s]);
-        if (j + 2 < nsteps) issue_sdp(j + 2);
+        mma_commit(&bars[KB_BFREE + b]);
       }
       mma_commit(&bars[KB_MMADONE]);
       mbar_wait(&bars[KB_MMADONE], 0, kWaitLimitNs);
