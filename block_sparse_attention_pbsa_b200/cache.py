@@ -254,16 +254,9 @@ class PBSALayerCache:
     def _write_chunk(self, k, v, stream=None):
         n = self.frames_of(k)
         dst = self._frames_dst(self.hist, n)
-        L.pbsa_blockify(self.geom, k, n, self.k_reps, self.pool_slots, dst, self.k_pool,
-                        self.pool_slots, ws=self.ws, stream=stream)
-        L.pbsa_blockify(self.geom, v, n, self._v_reps_sink(), self.pool_slots, dst,
-                        self.v_pool, self.pool_slots, ws=self.ws, stream=stream)
-
-    def _v_reps_sink(self) -> torch.Tensor:
-        # value representatives are not used by the method; blockify still writes them
-        if not hasattr(self, "_vreps"):
-            self._vreps = torch.empty_like(self.k_reps)
-        return self._vreps
+        # K and V blocks in one launch; value representatives are not used by the method
+        L.pbsa_blockify_kv(self.geom, k, v, n, self.k_reps, None, self.pool_slots, dst, self.k_pool,
+                           self.v_pool, self.pool_slots, ws=self.ws, stream=stream)
 
     def commit(self, k, v, q_reps_last=None, stream=None):
         """a4: commit the finished chunk (its last-step K, V) and update the persistent memory.
@@ -316,10 +309,8 @@ class PBSALayerCache:
             for t in range(bpf):
                 dst.append(self.stage_base + staged.index(f) * bpf + t if f in staged else self.ring_slot(f, t))
         dst_t = self._ints(dst)
-        L.pbsa_blockify(self.geom, k_hist, hist_frames, self.k_reps, self.pool_slots, dst_t, self.k_pool,
-                        self.pool_slots, ws=self.ws, stream=stream)
-        L.pbsa_blockify(self.geom, v_hist, hist_frames, self._v_reps_sink(), self.pool_slots, dst_t,
-                        self.v_pool, self.pool_slots, ws=self.ws, stream=stream)
+        L.pbsa_blockify_kv(self.geom, k_hist, v_hist, hist_frames, self.k_reps, None, self.pool_slots, dst_t,
+                           self.k_pool, self.v_pool, self.pool_slots, ws=self.ws, stream=stream)
         cand = [(self.stage_base + i * bpf + t, f * bpf + t) for i, f in enumerate(staged) for t in range(bpf)]
         self._update(q_reps, cand, stream)
         self.hist = hist_frames
@@ -351,8 +342,8 @@ class ChunkDecodeStep:
         self.cache = cache
         self.fused_select = fused_select
         # kernels per run(): [blockify(Q) + select] (1 fused or 2) + attend + blockify K, V (2)
-        # + memory update (2)
-        self.LAUNCHES = (1 if fused_select else 2) + 1 + 2 + 2
+        # + memory update (2); the commit of K and V is one launch
+        self.LAUNCHES = (1 if fused_select else 2) + 1 + 1 + 2
         self.q_frames = q_frames or c.chunk_frames
         if cache._cand is None:
             cache._refresh_window()
@@ -375,7 +366,6 @@ class ChunkDecodeStep:
         self.ncand = len(cand)
         self.cs = cache._ints([[s for s, _ in cand]] * H).view(H, -1) if cand else None
         self.cg = cache._ints([[g for _, g in cand]] * H).view(H, -1) if cand else None
-        self.vreps = cache._v_reps_sink()
 
     def flops(self) -> float:
         """Selected-block attention FLOPs of one run (QK^T and PV, 2 flops per MAC)."""
@@ -398,8 +388,8 @@ class ChunkDecodeStep:
         own = c.own_chunk
         mk(0)
         if own:   # the chunk's K, V go to their ring positions first: every row attends them
-            L.pbsa_blockify(g, k, self.q_frames, ca.k_reps, ps, self.dst, ca.k_pool, ps, ws=ws, stream=stream)
-            L.pbsa_blockify(g, v, self.q_frames, self.vreps, ps, self.dst, ca.v_pool, ps, ws=ws, stream=stream)
+            L.pbsa_blockify_kv(g, k, v, self.q_frames, ca.k_reps, None, ps, self.dst, ca.k_pool, ca.v_pool, ps,
+                               ws=ws, stream=stream)
             mk(1)
         cs, cg, n = ca._cand
         if self.fused_select:
@@ -418,8 +408,8 @@ class ChunkDecodeStep:
                       o, lse, ws=ws, stream=stream)
         mk(3)
         if not own:
-            L.pbsa_blockify(g, k, self.q_frames, ca.k_reps, ps, self.dst, ca.k_pool, ps, ws=ws, stream=stream)
-            L.pbsa_blockify(g, v, self.q_frames, self.vreps, ps, self.dst, ca.v_pool, ps, ws=ws, stream=stream)
+            L.pbsa_blockify_kv(g, k, v, self.q_frames, ca.k_reps, None, ps, self.dst, ca.k_pool, ca.v_pool, ps,
+                               ws=ws, stream=stream)
         mk(4)
         L.pbsa_memory_update(g, self.q_reps, self.nq, ca.k_reps, ca.k_pool, ca.v_pool, ps, ca.slot_gid,
                              ca.slot_ema, c.capacity, c.bpf, self.cs, self.cg, self.ncand, c.gamma,
@@ -458,8 +448,8 @@ class ChunkDecodeStep:
             L.pbsa_attend(g, q, self.q_frames, ca.k_pool, ca.v_pool, ps, self.kv_slot, self.kv_cnt, ca.kv_ld,
                           o, lse, ws=ws)
         with torch.cuda.graph(back, stream=side):
-            L.pbsa_blockify(g, k, self.q_frames, ca.k_reps, ps, self.dst, ca.k_pool, ps, ws=ws)
-            L.pbsa_blockify(g, v, self.q_frames, self.vreps, ps, self.dst, ca.v_pool, ps, ws=ws)
+            L.pbsa_blockify_kv(g, k, v, self.q_frames, ca.k_reps, None, ps, self.dst, ca.k_pool, ca.v_pool, ps,
+                               ws=ws)
             L.pbsa_memory_update(g, self.q_reps, self.nq, ca.k_reps, ca.k_pool, ca.v_pool, ps, ca.slot_gid,
                                  ca.slot_ema, c.capacity, c.bpf, self.cs, self.cg, self.ncand, c.gamma,
                                  ca.p_list, ca.p_cnt, ws=ws)

@@ -93,9 +93,26 @@ pbsa_status pbsa_blockify(const pbsa_geom* gin, const void* x, int n_frames, flo
   if (dst_slot == nullptr && rep_slots < n_frames * g.bpf) return PBSA_ERR_INVALID_ARG;
   if (pool != nullptr && (!pool_ok(g, pool_slots) || !aligned16(pool))) return PBSA_ERR_INVALID_ARG;
   if (pool != nullptr && dst_slot == nullptr && pool_slots < n_frames * g.bpf) return PBSA_ERR_INVALID_ARG;
-  if (!aligned16(x) || (int64_t)n_frames * g.bpf > 65535 * 64) return PBSA_ERR_INVALID_ARG;
+  if (!aligned16(x) || (int64_t)n_frames * g.bpf * g.H > ((int64_t)1 << 30)) return PBSA_ERR_INVALID_ARG;
   return from_cuda(launch_blockify(g, x, n_frames, reps, rep_slots, dst_slot, pool, pool_slots, ws,
                                    static_cast<cudaStream_t>(stream)));
+}
+
+pbsa_status pbsa_blockify_kv(const pbsa_geom* gin, const void* k, const void* v, int n_frames, float* k_reps,
+                             float* v_reps, int rep_slots, const int* dst_slot, void* k_pool, void* v_pool,
+                             int pool_slots, void* ws, void* stream) {
+  Geo g;
+  pbsa_status s = make_geo(gin, &g);
+  if (s != PBSA_OK) return s;
+  if (k == nullptr || v == nullptr || k_reps == nullptr || k_pool == nullptr || v_pool == nullptr)
+    return PBSA_ERR_INVALID_ARG;
+  if (n_frames <= 0 || rep_slots <= 0 || !pool_ok(g, pool_slots)) return PBSA_ERR_INVALID_ARG;
+  if (dst_slot == nullptr && (rep_slots < n_frames * g.bpf || pool_slots < n_frames * g.bpf))
+    return PBSA_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_pool) || !aligned16(v_pool)) return PBSA_ERR_INVALID_ARG;
+  if ((int64_t)n_frames * g.bpf * g.H > ((int64_t)1 << 30)) return PBSA_ERR_INVALID_ARG;
+  return from_cuda(launch_blockify_pair(g, k, v, n_frames, k_reps, v_reps, rep_slots, dst_slot, k_pool,
+                                        v_pool, pool_slots, ws, static_cast<cudaStream_t>(stream)));
 }
 
 pbsa_status pbsa_score_select(const pbsa_geom* gin, const float* q_reps, int nq, const float* k_reps,

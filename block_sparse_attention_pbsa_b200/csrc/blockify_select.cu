@@ -258,14 +258,33 @@ __global__ void __launch_bounds__(BS_THREADS) blockify_select_kernel(
 // ---------------------------------------------------------------------------- 8-block form
 // The flat policy with up to 256 candidates: one CTA of 512 threads per (head, 8 query blocks).
 //  1. every thread issues the 16-byte token loads of its four (block, column chunk, row set)
-//     shares -- the blockify split, so each block's mean is summed in blockify's order -- and
-//     the candidate list; then the candidates' representatives are staged in shared memory;
-//  2. warp w scores candidates w, w+16, ... against all 8 pooled queries at once: each lane
-//     holds d/32 elements of the 8 queries and of the candidate, and a transposing butterfly
-//     (9 shuffles for the 8 sums, fixed order) leaves each lane group one query's score;
-//  3. warp b sorts query block b's keys in registers (bitonic, 8 per lane, no block-wide
-//     barrier) and writes the first k.
+//     shares -- blockify's split, so each block's mean is summed in blockify's order -- and
+//     reads the candidate list; the candidates' representatives are then requested into
+//     shared memory (cp.async, rows padded to d + 4 floats) while the token loads are still
+//     in flight;
+//  2. the 8 pooled queries (rows 0..7 of an m16 tile) times the candidates on the tensor
+//     cores: m16n8k8 TF32 MMAs with each fp32 operand split into a TF32 high part and a TF32
+//     residual (hi*hi + hi*lo + lo*hi, fp32 accumulation: fp32-level accuracy);
+//  3. warp b selects query block b's k best: a radix search on the 64-bit ranking keys finds
+//     the k-th largest key -- it stops as soon as exactly k keys lie at or above the
+//     threshold -- and the chosen keys are put in order by a bitonic sort across the warp
+//     (k <= 32) or by counting (larger k).
 constexpr int S8_R = 8, S8_THREADS = 512;
+
+template <typename T, int D>
+struct S8Layout {
+  static constexpr int VEC = 16 / (int)sizeof(T);
+  static constexpr int CPR = D / VEC;             // chunks per token row
+  static constexpr int RPP = BS_THREADS / CPR;    // rows per pass of a 256-thread blockify share
+  static constexpr int KS = D + 4;                // padded representative row (floats)
+  static __host__ __device__ size_t part_bytes() { return (size_t)S8_R * RPP * D * 4; }
+  static __host__ __device__ int ncs(int ncand) { return ((ncand + 7) / 8) * 8 + 8; }   // score row stride
+  // part | kb [ncand][KS] | qs [16][KS] | ss [S8_R][ncs] | slot, gid [ncand]
+  static __host__ __device__ size_t bytes(int ncand) {
+    return part_bytes() + (size_t)ncand * KS * 4 + (size_t)16 * KS * 4 + (size_t)S8_R * ncs(ncand) * 4 +
+           (size_t)ncand * 8 + 16;
+  }
+};
 
 template <typename T, int D>
 __global__ void __launch_bounds__(S8_THREADS) blockify_select8_kernel(
@@ -275,19 +294,18 @@ __global__ void __launch_bounds__(S8_THREADS) blockify_select8_kernel(
     const int* __restrict__ prefix_cnt, int prefix_ld, int* __restrict__ out_slot,
     int* __restrict__ out_cnt, int out_ld, float* __restrict__ out_score,
     const int* __restrict__ suffix_slot, int suffix_n, void* ws) {
-  constexpr int VEC = 16 / sizeof(T);
-  constexpr int CPR = D / VEC;            // chunks per token row
-  constexpr int RPP = BS_THREADS / CPR;   // rows per pass of a 256-thread blockify share
+  using L = S8Layout<T, D>;
+  constexpr int VEC = L::VEC, CPR = L::CPR, RPP = L::RPP, KS = L::KS;
   constexpr int PASSES = BT / RPP;
-  constexpr int PL = D / 32;
   constexpr int NW = S8_THREADS / 32;
-  using V = typename Vec<PL>::type;
+  constexpr int CH = D / 4;   // 16-byte chunks of a representative row
   extern __shared__ __align__(16) float sm8[];
-  float* part = sm8;                                   // [S8_R][RPP][D]
-  float* kb = part + S8_R * RPP * D;                   // [ncand][D]
-  float* qb = kb + (size_t)ncand * D;                  // [S8_R][D]
-  float* sc = qb + S8_R * D;                           // [S8_R][ncand]
-  int* slot = reinterpret_cast<int*>(sc + S8_R * ncand);   // [ncand]
+  float* part = sm8;                                        // [S8_R][RPP][D]
+  float* kb = part + L::part_bytes() / 4;                   // [ncand][KS]
+  float* qs = kb + (size_t)ncand * KS;                      // [16][KS]
+  float* ss = qs + 16 * KS;                                 // [S8_R][ncs]
+  const int ncs = L::ncs(ncand);
+  int* slot = reinterpret_cast<int*>(ss + S8_R * ncs);      // [ncand]
   int* gid = slot + ncand;                                  // [ncand]
 
   const int h = blockIdx.y, r0 = blockIdx.x * S8_R;
@@ -316,6 +334,17 @@ __global__ void __launch_bounds__(S8_THREADS) blockify_select8_kernel(
     gid[j] = cand_gid[(size_t)h * ncand + j];
     slot[j] = cand_slot[(size_t)h * ncand + j];
   }
+  for (int i = tid; i < 8 * CH; i += S8_THREADS)   // query rows 8..15 of the MMA tile are zero
+    reinterpret_cast<float4*>(qs + (8 + i / CH) * KS)[i % CH] = make_float4(0.f, 0.f, 0.f, 0.f);
+  __syncthreads();
+  {
+    const float* krep_h = k_reps + (size_t)h * pool_slots * D;
+    for (int i = tid; i < ncand * CH; i += S8_THREADS) {
+      const int j = i / CH, e = i - j * CH;
+      const int s = slot[j];
+      if (s >= 0 && s < pool_slots) cp_async16(kb + j * KS + 4 * e, krep_h + (size_t)s * D + 4 * e);
+    }
+  }
 #pragma unroll
   for (int u = 0; u < S8_R / 2; ++u) {
     float acc[VEC];
@@ -328,91 +357,43 @@ __global__ void __launch_bounds__(S8_THREADS) blockify_select8_kernel(
     for (int i = 0; i < VEC; ++i) pr[i] = acc[i];
   }
   __syncthreads();
-  // candidate representatives -> shared memory (all rows' 16-byte loads in flight)
-  {
-    constexpr int F4 = D / 4;
-    for (int base = tid; base < ncand * F4; base += S8_THREADS * 8) {
-      float4 buf[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int i = base + u * S8_THREADS;
-        buf[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (i < ncand * F4) {
-          const int s = slot[i / F4];
-          if (s >= 0 && s < pool_slots)
-            buf[u] = __ldg(reinterpret_cast<const float4*>(k_reps + ((size_t)h * pool_slots + s) * D) + (i % F4));
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int i = base + u * S8_THREADS;
-        if (i < ncand * F4) reinterpret_cast<float4*>(kb)[i] = buf[u];
-      }
-    }
-  }
-  // qbar (fixed-order sums, as in the blockify kernel)
+  // qbar (fixed-order sums, as in the blockify kernel) -> query rows of the MMA tile
   for (int i = tid; i < S8_R * D; i += S8_THREADS) {
     const int b = i / D, e = i - b * D;
     float s = 0.f;
 #pragma unroll 4
     for (int q = 0; q < RPP; ++q) s += part[(b * RPP + q) * D + e];
     s *= (1.0f / BT);
-    qb[i] = s;
+    qs[b * KS + e] = s;
     if (b < nr) q_reps[((size_t)h * nq + r0 + b) * D + e] = s;
   }
+  cp_async_wait_all();
   __syncthreads();
 
-  // ---- 2. scores: warp per candidate, all 8 queries at once
-  float ql[S8_R][PL];
+  // ---- 2. scores on the tensor cores: warp w takes the 8-candidate tiles w, w + NW, ...
+  {
+    const int gq = lane >> 2, t4 = lane & 3;
+    const int ntiles = (ncand + 7) / 8;
+    for (int nt = warp; nt < ntiles; nt += NW) {
+      float acc[6][4] = {};
+      const float* brow = kb + (nt * 8 + gq) * KS;   // candidate nt*8 + gq (past ncand: unused)
+      const uint32_t zero[1] = {0u};
 #pragma unroll
-  for (int b = 0; b < S8_R; ++b)
-#pragma unroll
-    for (int i = 0; i < PL; ++i) ql[b][i] = qb[b * D + lane * PL + i];
-  for (int cc = warp; cc < ncand; cc += NW) {
-    float kv[PL];
-    vec_to(reinterpret_cast<const V*>(kb + (size_t)cc * D)[lane], kv);
-    float a[S8_R];
-#pragma unroll
-    for (int b = 0; b < S8_R; ++b) {
-      a[b] = 0.f;
-#pragma unroll
-      for (int i = 0; i < PL; ++i) a[b] = fmaf(ql[b][i], kv[i], a[b]);
-    }
-    // transposing butterfly: after the xor-16/8/4 exchanges lane l holds query
-    // ((l >> 2) & 7)'s partial over 4 lanes; xor-2/1 finish the sum
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {          // xor 16: keep 4 of 8
-      const bool up = lane & 16;
-      const float send = up ? a[j] : a[j + 4];
-      const float keep = up ? a[j + 4] : a[j];
-      a[j] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
-    }
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {          // xor 8: keep 2 of 4
-      const bool up = lane & 8;
-      const float send = up ? a[j] : a[j + 2];
-      const float keep = up ? a[j + 2] : a[j];
-      a[j] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
-    }
-    {                                      // xor 4: keep 1 of 2
-      const bool up = lane & 4;
-      const float send = up ? a[0] : a[1];
-      const float keep = up ? a[1] : a[0];
-      a[0] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-    }
-    a[0] += __shfl_xor_sync(0xffffffffu, a[0], 2);
-    a[0] += __shfl_xor_sync(0xffffffffu, a[0], 1);
-    if ((lane & 3) == 0) {
-      // lane bits 4, 3, 2 picked halves (upper half = higher index) in that order
-      const int b = ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
-      float val = a[0] * g.scale;
-      const int s = slot[cc];
-      if (s < 0 || s >= pool_slots) {
-        if (b == 0 && r0 == 0) record_error(ws, PBSA_ERR_DEVICE_INDEX, s, K_SCORE);
-        val = -INFINITY;
+      for (int k0 = 0; k0 < D; k0 += 8) {
+        const int par = (k0 >> 3) & 1;
+        uint32_t ah[4], al[4], bh0, bl0, bh1, bl1;
+        tf32_split(qs[gq * KS + k0 + t4], ah[0], al[0]);
+        tf32_split(qs[gq * KS + k0 + t4 + 4], ah[2], al[2]);
+        ah[1] = ah[3] = al[1] = al[3] = zero[0];   // rows 8..15: zero queries
+        tf32_split(brow[k0 + t4], bh0, bl0);
+        tf32_split(brow[k0 + t4 + 4], bh1, bl1);
+        mma_tf32(acc[3 * par + 0], al, bh0, bh1);
+        mma_tf32(acc[3 * par + 1], ah, bl0, bl1);
+        mma_tf32(acc[3 * par + 2], ah, bh0, bh1);
       }
-      if (isnan(val)) val = -INFINITY;
-      sc[b * ncand + cc] = val;
+      float r0v = ((acc[0][0] + acc[3][0]) + (acc[1][0] + acc[4][0])) + (acc[2][0] + acc[5][0]);
+      float r1v = ((acc[0][1] + acc[3][1]) + (acc[1][1] + acc[4][1])) + (acc[2][1] + acc[5][1]);
+      *reinterpret_cast<float2*>(ss + gq * ncs + nt * 8 + 2 * t4) = make_float2(r0v, r1v);
     }
   }
   int pc = prefix_cnt ? prefix_cnt[h] : 0;
@@ -429,87 +410,135 @@ __global__ void __launch_bounds__(S8_THREADS) blockify_select8_kernel(
   if (tid < nr) out_cnt[(size_t)h * nq + r0 + tid] = pc + kk + suffix_n;
   __syncthreads();
 
-  // ---- 3. warp b selects query block b's k best: element e = j*32 + lane (j < 8).  A radix
-  // search finds the k-th largest key (score bits first; the gid bits only on an exact score
-  // tie), so exactly k elements are chosen, then each chosen element's rank among the chosen
-  // is counted and it is written at that rank.
+  // ---- 3. warp b selects query block b's k best: element e = j*32 + lane (j < 8)
   if (warp < nr) {
     const int b = warp;
+    auto score_of = [&](int e) {   // masked, scaled score of candidate e
+      const int s = slot[e];
+      float val = ss[b * ncs + e] * g.scale;
+      if (s < 0 || s >= pool_slots) {
+        if (b == 0 && r0 == 0) record_error(ws, PBSA_ERR_DEVICE_INDEX, s, K_SCORE);
+        val = -INFINITY;
+      }
+      return isnan(val) ? -INFINITY : val;
+    };
     uint64_t kv8[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int e = j * 32 + lane;
-      kv8[j] = e < ncand ? rank_key(sc[b * ncand + e], gid[e]) : 0ull;
+      kv8[j] = e < ncand ? rank_key(score_of(e), gid[e]) : 0ull;
     }
-    // k-th largest of the high words (score order keys)
     auto count_hi_ge = [&](uint32_t t) {
       int n = 0;
 #pragma unroll
       for (int j = 0; j < 8; ++j) n += (uint32_t)(kv8[j] >> 32) >= t;
       return __reduce_add_sync(0xffffffffu, n);
     };
+    // k-th largest high word (score order); stop early once exactly kk keys are at or above
     uint32_t th = 0;
+    bool exact = false;
     if (kk > 0) {
 #pragma unroll 1
       for (int bit = 31; bit >= 0; --bit) {
         const uint32_t t2 = th | (1u << bit);
-        if (count_hi_ge(t2) >= kk) th = t2;
+        const int cnt = count_hi_ge(t2);
+        if (cnt >= kk) {
+          th = t2;
+          if (cnt == kk) {
+            exact = true;
+            break;
+          }
+        }
       }
     }
-    int n_gt = 0;
+    // the chosen set: exact -> every key whose high word is >= th; otherwise the keys above the
+    // k-th key (high word, then the gid word), then keys equal to it in position order
+    uint64_t tkey = 0;
+    int n_above = 0;
+    if (!exact && kk > 0) {
+      int n_gt = 0;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) n_gt += (uint32_t)(kv8[j] >> 32) > th;
-    n_gt = __reduce_add_sync(0xffffffffu, n_gt);
-    // among the keys whose high word equals th, the (kk - n_gt)-th largest low word (gid)
-    const int need = kk - n_gt;
-    auto count_lo_ge = [&](uint32_t t) {
-      int n = 0;
+      for (int j = 0; j < 8; ++j) n_gt += (uint32_t)(kv8[j] >> 32) > th;
+      n_gt = __reduce_add_sync(0xffffffffu, n_gt);
+      const int need = kk - n_gt;
+      auto count_lo_ge = [&](uint32_t t) {
+        int n = 0;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) n += ((uint32_t)(kv8[j] >> 32) == th) && ((uint32_t)kv8[j] >= t);
-      return __reduce_add_sync(0xffffffffu, n);
-    };
-    uint32_t tl = 0;
-    if (need > 0 && count_lo_ge(0) > need) {
+        for (int j = 0; j < 8; ++j) n += ((uint32_t)(kv8[j] >> 32) == th) && ((uint32_t)kv8[j] >= t);
+        return __reduce_add_sync(0xffffffffu, n);
+      };
+      uint32_t tl = 0;
+      if (need > 0 && count_lo_ge(0) > need) {
 #pragma unroll 1
-      for (int bit = 31; bit >= 0; --bit) {
-        const uint32_t t2 = tl | (1u << bit);
-        if (count_lo_ge(t2) >= need) tl = t2;
+        for (int bit = 31; bit >= 0; --bit) {
+          const uint32_t t2 = tl | (1u << bit);
+          if (count_lo_ge(t2) >= need) tl = t2;
+        }
       }
-    }
-    const uint64_t tkey = ((uint64_t)th << 32) | tl;
-    int n_above = 0;   // keys strictly above the k-th key
+      tkey = ((uint64_t)th << 32) | tl;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) n_above += kv8[j] > tkey;
-    n_above = __reduce_add_sync(0xffffffffu, n_above);
-    // chosen: every key above tkey, then keys equal to tkey in position order (exact
-    // duplicates of (score, gid) only)
+      for (int j = 0; j < 8; ++j) n_above += kv8[j] > tkey;
+      n_above = __reduce_add_sync(0xffffffffu, n_above);
+    }
     int* chosen = reinterpret_cast<int*>(part) + b * 256;    // part is free after the pooling
     int eq_seen = 0, n_ch = 0;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      const bool eq = kk > 0 && kv8[j] == tkey;
-      const unsigned eb = __ballot_sync(0xffffffffu, eq);
-      const bool take_eq = eq && (eq_seen + __popc(eb & ((1u << lane) - 1u)) < kk - n_above);
-      eq_seen += __popc(eb);
-      const bool take = (kk > 0 && kv8[j] > tkey) || take_eq;
+      bool take;
+      if (exact) {
+        take = kv8[j] != 0ull && (uint32_t)(kv8[j] >> 32) >= th;
+      } else {
+        const bool eq = kk > 0 && kv8[j] == tkey;
+        const unsigned eb = __ballot_sync(0xffffffffu, eq);
+        const bool take_eq = eq && (eq_seen + __popc(eb & ((1u << lane) - 1u)) < kk - n_above);
+        eq_seen += __popc(eb);
+        take = (kk > 0 && kv8[j] > tkey) || take_eq;
+      }
       const unsigned tb = __ballot_sync(0xffffffffu, take);
       if (take) chosen[n_ch + __popc(tb & ((1u << lane) - 1u))] = j * 32 + lane;
       n_ch += __popc(tb);
     }
     __syncwarp();
-    // rank among the chosen: larger key first, then the lower position
     const size_t o = (size_t)h * nq + r0 + b;
-    for (int t = lane; t < n_ch; t += 32) {
-      const int e = chosen[t];
-      const uint64_t ke = rank_key(sc[b * ncand + e], gid[e]);
-      int rank = 0;
-      for (int u = 0; u < n_ch; ++u) {
-        const int e2 = chosen[u];
-        const uint64_t k2 = rank_key(sc[b * ncand + e2], gid[e2]);
-        rank += (k2 > ke) | ((k2 == ke) & (e2 < e));
+    if (n_ch <= 32) {
+      // order the chosen: larger key first, then the lower position (bitonic across lanes)
+      int e = lane < n_ch ? chosen[lane] : 0x7FFFFFFF;
+      float val = lane < n_ch ? score_of(e) : -INFINITY;
+      uint64_t key = lane < n_ch ? rank_key(val, gid[e]) : 0ull;
+#pragma unroll
+      for (int k2 = 2; k2 <= 32; k2 <<= 1) {
+#pragma unroll
+        for (int j = k2 >> 1; j > 0; j >>= 1) {
+          const uint64_t ok = __shfl_xor_sync(0xffffffffu, key, j);
+          const int oe = __shfl_xor_sync(0xffffffffu, e, j);
+          const float ov = __shfl_xor_sync(0xffffffffu, val, j);
+          const bool other_first = ok > key || (ok == key && oe < e);
+          const bool lower = (lane & j) == 0, desc = (lane & k2) == 0;
+          if ((lower == desc) ? other_first : !other_first) {
+            key = ok;
+            e = oe;
+            val = ov;
+          }
+        }
       }
-      out_slot[o * out_ld + pc + rank] = slot[e];
-      if (out_score) out_score[o * k + rank] = sc[b * ncand + e];
+      if (lane < n_ch) {
+        out_slot[o * out_ld + pc + lane] = slot[e];
+        if (out_score) out_score[o * k + lane] = val;
+      }
+    } else {
+      // rank among the chosen: larger key first, then the lower position
+      for (int t = lane; t < n_ch; t += 32) {
+        const int e = chosen[t];
+        const uint64_t ke = rank_key(score_of(e), gid[e]);
+        int rank = 0;
+        for (int u = 0; u < n_ch; ++u) {
+          const int e2 = chosen[u];
+          const uint64_t k2 = rank_key(score_of(e2), gid[e2]);
+          rank += (k2 > ke) | ((k2 == ke) & (e2 < e));
+        }
+        out_slot[o * out_ld + pc + rank] = slot[e];
+        if (out_score) out_score[o * k + rank] = score_of(e);
+      }
     }
   }
 }
@@ -522,9 +551,7 @@ cudaError_t launch_t(const Geo& g, const void* x, int q_frames, float* q_reps, c
                      const int* suffix_slot, int suffix_n, void* ws, cudaStream_t st) {
   const int nq = q_frames * g.bpf;
   if (!HSA && ncand <= 256) {
-    constexpr int RPP = BS_THREADS / (D / (16 / (int)sizeof(T)));
-    const size_t smem8 = ((size_t)S8_R * RPP * D + (size_t)ncand * D + (size_t)S8_R * D +
-                          (size_t)S8_R * ncand) * 4 + (size_t)ncand * 8;
+    const size_t smem8 = S8Layout<T, D>::bytes(ncand);
     auto kern8 = blockify_select8_kernel<T, D>;
     cudaError_t e = set_smem_once((const void*)kern8, (int)smem8);
     if (e != cudaSuccess) return e;

@@ -92,6 +92,22 @@ PBSA_API pbsa_status pbsa_blockify(const pbsa_geom* g, const void* x, int n_fram
                           float* reps, int rep_slots, const int* dst_slot,
                           void* pool, int pool_slots, void* ws, void* stream);
 
+/* a1 for a committed chunk -- pbsa_blockify of K and of V in one launch, with the same
+ * destination slots (the chunk's K and V blocks enter the cache together; English 2.E
+ * "blockifying the latent space").  Equivalent to
+ *   pbsa_blockify(k, n_frames, k_reps, rep_slots, dst_slot, k_pool, pool_slots) and
+ *   pbsa_blockify(v, n_frames, v_reps, rep_slots, dst_slot, v_pool, pool_slots).
+ *  k, v           [n_frames*frame_h*frame_w][H][d] raster, geometry dtype (16-byte aligned).
+ *  k_reps         out [H][rep_slots][d] fp32 (required).
+ *  v_reps         nullable out [H][rep_slots][d] fp32; NULL skips the V representatives
+ *                 (the method only scores K).
+ *  k_pool, v_pool out [H][pool_slots][64][d] (both required).
+ *  dst_slot       nullable [n_frames*bpf], as for pbsa_blockify.
+ * Errors as for pbsa_blockify. */
+PBSA_API pbsa_status pbsa_blockify_kv(const pbsa_geom* g, const void* k, const void* v, int n_frames,
+                          float* k_reps, float* v_reps, int rep_slots, const int* dst_slot,
+                          void* k_pool, void* v_pool, int pool_slots, void* ws, void* stream);
+
 /* a2 -- coarse score + top-k: for each head h and query block r,
  *   score(r, c) = scale * <q_reps[h][r], k_reps[h][cand_slot[h][c]]>  (fp32)
  * and the k best candidates (score descending, ties to the lower cand_gid, then the lower

@@ -55,6 +55,47 @@ def test_blockify_reps_and_pool(w):
         assert torch.equal(pool[:, s].cpu(), x[rows].permute(1, 0, 2))
 
 
+@pytest.mark.parametrize("w,n_frames,with_v_reps", [(I.TINY, 3, True), (I.DECODE_5S, 7, False),
+                                                     (I.DECODE_5S, 1, True),
+                                                     (dataclasses.replace(I.DECODE_5S, tile_h=4, tile_w=16), 2, True)])
+def test_blockify_kv_one_launch(w, n_frames, with_v_reps):
+    """pbsa_blockify_kv: K and V of several frames in one launch (many units per CTA of the
+    persistent grid), against the oracle's means and the raster rows of every block."""
+    g = geom_for(w)
+    k, v = I.tokens(w, n_frames, 21), I.tokens(w, n_frames, 22)
+    nb = n_frames * w.blocks_per_frame
+    slots = nb + 7
+    dst = torch.randperm(slots, generator=torch.Generator().manual_seed(5))[:nb].to(torch.int32)
+    k_reps = torch.zeros((w.heads, slots, w.head_dim), device=DEV)
+    v_reps = torch.zeros((w.heads, slots, w.head_dim), device=DEV) if with_v_reps else None
+    k_pool = torch.zeros((w.heads, slots, 64, w.head_dim), dtype=k.dtype, device=DEV)
+    v_pool = torch.zeros_like(k_pool)
+    ws = ws_for(g)
+    P.pbsa_blockify_kv(g, k.to(DEV), v.to(DEV), n_frames, k_reps, v_reps, slots, dst.to(DEV), k_pool, v_pool,
+                       slots, ws)
+    check_no_device_error(ws)
+    want_k = O.block_reps(f64(k), geom_dict(w), n_frames)
+    want_v = O.block_reps(f64(v), geom_dict(w), n_frames)
+    got_k = f64(k_reps)
+    got_v = f64(v_reps) if with_v_reps else None
+    kp, vp = k_pool.cpu(), v_pool.cpu()
+    for b in range(nb):
+        s = int(dst[b])
+        np.testing.assert_allclose(got_k[:, s], want_k[:, b], rtol=0, atol=2e-6)
+        if with_v_reps:
+            np.testing.assert_allclose(got_v[:, s], want_v[:, b], rtol=0, atol=2e-6)
+        rows = O.block_token_rows(w.frame_h, w.frame_w, w.tile_h, w.tile_w, b)
+        assert torch.equal(kp[:, s], k[rows].permute(1, 0, 2))
+        assert torch.equal(vp[:, s], v[rows].permute(1, 0, 2))
+    # slots that no block maps to stay untouched
+    unused = sorted(set(range(slots)) - set(dst.tolist()))
+    assert not kp[:, unused].any() and not vp[:, unused].any() and not k_reps[:, unused].any()
+    # the K representatives equal pbsa_blockify's bit for bit (one summation order)
+    k_reps1 = torch.zeros_like(k_reps)
+    P.pbsa_blockify(g, k.to(DEV), n_frames, k_reps1, slots, dst.to(DEV), None, 0, ws)
+    assert torch.equal(k_reps1, k_reps)
+
+
 # ----------------------------------------------------------------------------- score + select
 def _selection_case(seed, H=3, nq=9, pool=200, ncand=144, d=128, k=32, prefix=20, dup=False):
     gen = torch.Generator().manual_seed(seed)
