@@ -52,7 +52,7 @@ _I = ctypes.c_int
 _SIGS = {
     "pbsa_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(Geom), _I, _I]),
     "pbsa_blockify": (_I, [ctypes.POINTER(Geom), _P, _I, _P, _I, _P, _P, _I, _P, _P]),
-    "pbsa_blockify_kv": (_I, [ctypes.POINTER(Geom), _P, _P, _I, _P, _P, _I, _P, _P, _P, _I, _P, _P]),
+    "pbsa_blockify_kv": (_I, [ctypes.POINTER(Geom), _P, _P, _I, _P, _P, _I, _P, _P, _P, _I, _I, _P, _P]),
     "pbsa_score_select": (_I, [ctypes.POINTER(Geom), _P, _I, _P, _I, _P, _P, _I, _I, _P, _P, _I,
                                _P, _P, _I, _P, _P, _P]),
     "pbsa_blockify_score_select": (_I, [ctypes.POINTER(Geom), _P, _I, _P, _P, _I, _P, _P, _I, _I, _P,
@@ -134,13 +134,16 @@ def pbsa_blockify(g: Geom, x, n_frames, reps, rep_slots, dst_slot=None, pool=Non
         pool_slots, _ptr(ws, None, "ws"), _stream(stream)))
 
 
+PBSA_OVERLAP_PREVIOUS = 1
+
+
 def pbsa_blockify_kv(g: Geom, k, v, n_frames, k_reps, v_reps, rep_slots, dst_slot, k_pool, v_pool,
-                     pool_slots, ws=None, stream=None):
+                     pool_slots, flags=0, ws=None, stream=None):
     _check("pbsa_blockify_kv", load().pbsa_blockify_kv(
         ctypes.byref(g), _ptr(k, _tok_dtype(g), "k"), _ptr(v, _tok_dtype(g), "v"), n_frames,
         _ptr(k_reps, torch.float32, "k_reps"), _ptr(v_reps, torch.float32, "v_reps"), rep_slots,
         _ptr(dst_slot, torch.int32, "dst_slot"), _ptr(k_pool, _tok_dtype(g), "k_pool"),
-        _ptr(v_pool, _tok_dtype(g), "v_pool"), pool_slots, _ptr(ws, None, "ws"), _stream(stream)))
+        _ptr(v_pool, _tok_dtype(g), "v_pool"), pool_slots, flags, _ptr(ws, None, "ws"), _stream(stream)))
 
 
 def pbsa_score_select(g: Geom, q_reps, nq, k_reps, pool_slots, cand_slot, cand_gid, ncand, k,

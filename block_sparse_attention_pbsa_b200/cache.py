@@ -408,8 +408,11 @@ class ChunkDecodeStep:
                       o, lse, ws=ws, stream=stream)
         mk(3)
         if not own:
+            # the commit writes only free ring slots, which the attend lists never name: without
+            # timing events in between it may start on SMs that attend's last wave leaves idle
+            flags = L.PBSA_OVERLAP_PREVIOUS if marks is None else 0
             L.pbsa_blockify_kv(g, k, v, self.q_frames, ca.k_reps, None, ps, self.dst, ca.k_pool, ca.v_pool, ps,
-                               ws=ws, stream=stream)
+                               flags=flags, ws=ws, stream=stream)
         mk(4)
         L.pbsa_memory_update(g, self.q_reps, self.nq, ca.k_reps, ca.k_pool, ca.v_pool, ps, ca.slot_gid,
                              ca.slot_ema, c.capacity, c.bpf, self.cs, self.cg, self.ncand, c.gamma,
@@ -417,17 +420,23 @@ class ChunkDecodeStep:
         mk(5)
         return o
 
-    def capture(self, q, k, v, o, lse=None, marks=None) -> torch.cuda.CUDAGraph:
+    def capture(self, q, k, v, o, lse=None, marks=None, ends=None) -> torch.cuda.CUDAGraph:
         """Capture ``run`` in a CUDA graph (one launch replays all kernels of the step).
 
         Call ``run`` once before capturing (kernel attributes are set on first use).  With
-        ``marks``, pass events created with ``external=True`` so they time inside the graph.
+        ``marks`` (6 events between the kernel groups) or ``ends`` (2 events around the whole
+        step, which leave the commit free to overlap attend), pass events created with
+        ``external=True`` so they time inside the graph.
         """
         graph = torch.cuda.CUDAGraph()
         side = torch.cuda.Stream(device=self.cache.device)
         side.wait_stream(torch.cuda.current_stream(self.cache.device))
         with torch.cuda.graph(graph, stream=side):
+            if ends is not None:
+                ends[0].record(side)
             self.run(q, k, v, o, lse, stream=None, marks=marks)
+            if ends is not None:
+                ends[1].record(side)
         torch.cuda.current_stream(self.cache.device).wait_stream(side)
         return graph
 

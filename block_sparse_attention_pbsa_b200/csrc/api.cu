@@ -100,7 +100,7 @@ pbsa_status pbsa_blockify(const pbsa_geom* gin, const void* x, int n_frames, flo
 
 pbsa_status pbsa_blockify_kv(const pbsa_geom* gin, const void* k, const void* v, int n_frames, float* k_reps,
                              float* v_reps, int rep_slots, const int* dst_slot, void* k_pool, void* v_pool,
-                             int pool_slots, void* ws, void* stream) {
+                             int pool_slots, int flags, void* ws, void* stream) {
   Geo g;
   pbsa_status s = make_geo(gin, &g);
   if (s != PBSA_OK) return s;
@@ -111,8 +111,10 @@ pbsa_status pbsa_blockify_kv(const pbsa_geom* gin, const void* k, const void* v,
     return PBSA_ERR_INVALID_ARG;
   if (!aligned16(k) || !aligned16(v) || !aligned16(k_pool) || !aligned16(v_pool)) return PBSA_ERR_INVALID_ARG;
   if ((int64_t)n_frames * g.bpf * g.H > ((int64_t)1 << 30)) return PBSA_ERR_INVALID_ARG;
+  if ((flags & ~PBSA_OVERLAP_PREVIOUS) != 0) return PBSA_ERR_INVALID_ARG;
   return from_cuda(launch_blockify_pair(g, k, v, n_frames, k_reps, v_reps, rep_slots, dst_slot, k_pool,
-                                        v_pool, pool_slots, ws, static_cast<cudaStream_t>(stream)));
+                                        v_pool, pool_slots, (flags & PBSA_OVERLAP_PREVIOUS) != 0, ws,
+                                        static_cast<cudaStream_t>(stream)));
 }
 
 pbsa_status pbsa_score_select(const pbsa_geom* gin, const float* q_reps, int nq, const float* k_reps,

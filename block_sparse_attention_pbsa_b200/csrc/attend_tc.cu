@@ -28,6 +28,7 @@
 //    merges the two streams exactly.
 //  * Register split: the producer/issuer warpgroup runs on 64 registers, the softmax
 //    warpgroups on 216 (setmaxnreg), so the softmax holds its row in registers.
+//  * Each CTA signals programmatic dependents at its start (griddepcontrol.launch_dependents).
 //  * Every wait is bounded; on expiry the kernel records PBSA_ERR_TIMEOUT in the
 //    workspace, drains its own copies and MMAs, frees TMEM and returns.
 #include <math.h>
@@ -136,6 +137,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     tx * prm.tw, ty * prm.th, f);
     }
   }
+  // A kernel launched after this one as a programmatic dependent (pbsa_blockify_kv with
+  // PBSA_OVERLAP_PREVIOUS) may start once every CTA of this grid has started: it then only
+  // takes SMs this grid leaves idle in its last wave.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (warp == 1) {
     tmem_alloc(tmem_holder, 512);
     tmem_relinquish();

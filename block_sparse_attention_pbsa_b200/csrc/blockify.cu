@@ -19,7 +19,9 @@
 //    blockify + select kernel's query representative);
 //  * a stage is refilled one unit later, once its bulk copy has read it and every thread is
 //    past it (NST - 1 loads stay in flight while a store drains).
-// K and V of a chunk go through one launch (two tensor maps, units of both tensors).
+// K and V of a chunk go through one launch (two tensor maps, units of both tensors).  On request
+// the launch is a programmatic dependent of the previous kernel on the stream: it may start on
+// SMs that kernel leaves idle and waits for it (griddepcontrol.wait) before completing.
 #include <mutex>
 
 #include "common.cuh"
@@ -130,6 +132,7 @@ __global__ void __launch_bounds__(BY_THREADS) blockify_kernel(const __grid_const
           mbar_wait(&full[j % BY_STAGES], (j / BY_STAGES) & 1, kWaitLimitNs);
         bulk_wait_all();
       }
+      asm volatile("griddepcontrol.wait;" ::: "memory");
       return;
     }
     const uint8_t* tile = sm + s * TL::BYTES;
@@ -170,6 +173,10 @@ __global__ void __launch_bounds__(BY_THREADS) blockify_kernel(const __grid_const
     // the next iteration's barrier orders these reads of `part` before it is rewritten
   }
   if (tid == 0) bulk_wait_all();
+  // Launched as a programmatic dependent, this grid must not complete before the grid it
+  // overlaps: what follows on the stream then still runs after both.  (Returns at once for an
+  // ordinary launch.)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -216,7 +223,7 @@ int persistent_grid(const void* kernel, int smem) {
 
 template <typename T, int D>
 cudaError_t launch_t(const Geo& g, const void* x0, const void* x1, int n_frames, const BlockifyParams& p,
-                     cudaStream_t st) {
+                     bool overlap_previous, cudaStream_t st) {
   CUtensorMap m0, m1;
   if (!encode_raster(&m0, g, x0, n_frames)) return cudaErrorNotSupported;
   if (x1 != nullptr) {
@@ -230,15 +237,24 @@ cudaError_t launch_t(const Geo& g, const void* x0, const void* x1, int n_frames,
   if (e != cudaSuccess) return e;
   const long units = (long)p.nz * p.nblk * p.H;
   const int grid = (int)(units < persistent_grid((const void*)kern, smem) ? units : persistent_grid((const void*)kern, smem));
-  kern<<<grid, BY_THREADS, smem, st>>>(m0, m1, p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(BY_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = overlap_previous ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, m0, m1, p);
 }
 
 }  // namespace
 
 cudaError_t launch_blockify_pair(const Geo& g, const void* x0, const void* x1, int n_frames, float* reps0,
                                  float* reps1, int rep_slots, const int* dst_slot, void* pool0, void* pool1,
-                                 int pool_slots, void* ws, cudaStream_t st) {
+                                 int pool_slots, bool overlap_previous, void* ws, cudaStream_t st) {
   BlockifyParams p;
   p.nz = x1 != nullptr ? 2 : 1;
   p.nblk = n_frames * g.bpf;
@@ -256,12 +272,12 @@ cudaError_t launch_blockify_pair(const Geo& g, const void* x0, const void* x1, i
   p.dst_slot = dst_slot;
   p.ws = ws;
   if (g.dtype == PBSA_BF16) {
-    if (g.d == 128) return launch_t<__nv_bfloat16, 128>(g, x0, x1, n_frames, p, st);
-    if (g.d == 64) return launch_t<__nv_bfloat16, 64>(g, x0, x1, n_frames, p, st);
+    if (g.d == 128) return launch_t<__nv_bfloat16, 128>(g, x0, x1, n_frames, p, overlap_previous, st);
+    if (g.d == 64) return launch_t<__nv_bfloat16, 64>(g, x0, x1, n_frames, p, overlap_previous, st);
   } else {
-    if (g.d == 128) return launch_t<float, 128>(g, x0, x1, n_frames, p, st);
-    if (g.d == 64) return launch_t<float, 64>(g, x0, x1, n_frames, p, st);
-    if (g.d == 32) return launch_t<float, 32>(g, x0, x1, n_frames, p, st);
+    if (g.d == 128) return launch_t<float, 128>(g, x0, x1, n_frames, p, overlap_previous, st);
+    if (g.d == 64) return launch_t<float, 64>(g, x0, x1, n_frames, p, overlap_previous, st);
+    if (g.d == 32) return launch_t<float, 32>(g, x0, x1, n_frames, p, overlap_previous, st);
   }
   return cudaErrorNotSupported;
 }
@@ -270,7 +286,7 @@ cudaError_t launch_blockify(const Geo& g, const void* x, int n_frames, float* re
                             const int* dst_slot, void* pool, int pool_slots, void* ws,
                             cudaStream_t st) {
   return launch_blockify_pair(g, x, nullptr, n_frames, reps, nullptr, rep_slots, dst_slot, pool, nullptr,
-                              pool_slots, ws, st);
+                              pool_slots, false, ws, st);
 }
 
 }  // namespace pbsa

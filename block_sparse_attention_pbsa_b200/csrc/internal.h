@@ -32,10 +32,11 @@ cudaError_t launch_blockify(const Geo& g, const void* x, int n_frames, float* re
                             cudaStream_t st);
 
 // K and V (x1, reps1, pool1 nullable: one tensor only; reps0/reps1 nullable: no reps of that
-// tensor) in one launch, with the same destination slots.
+// tensor) in one launch, with the same destination slots; overlap_previous: programmatic
+// dependent launch after the previous kernel on the stream.
 cudaError_t launch_blockify_pair(const Geo& g, const void* x0, const void* x1, int n_frames, float* reps0,
                                  float* reps1, int rep_slots, const int* dst_slot, void* pool0, void* pool1,
-                                 int pool_slots, void* ws, cudaStream_t st);
+                                 int pool_slots, bool overlap_previous, void* ws, cudaStream_t st);
 
 cudaError_t launch_score_select(const Geo& g, const float* q_reps, int nq, const float* k_reps,
                                 int pool_slots, const int* cand_slot, const int* cand_gid,

@@ -103,10 +103,18 @@ PBSA_API pbsa_status pbsa_blockify(const pbsa_geom* g, const void* x, int n_fram
  *                 (the method only scores K).
  *  k_pool, v_pool out [H][pool_slots][64][d] (both required).
  *  dst_slot       nullable [n_frames*bpf], as for pbsa_blockify.
- * Errors as for pbsa_blockify. */
+ *  flags          0, or PBSA_OVERLAP_PREVIOUS: launch as a programmatic dependent of the
+ *                 previous kernel on `stream`.  The commit may then start on SMs that kernel
+ *                 leaves idle (pbsa_attend signals this once all of its CTAs have started), and
+ *                 it still completes only after that kernel, so later work on the stream sees
+ *                 both.  Only valid when the previous kernel neither writes k or v nor reads
+ *                 or writes the destination slots and k_reps rows (true of pbsa_attend before
+ *                 the commit of the chunk it attended: its lists never name free ring slots).
+ * Errors as for pbsa_blockify (an unknown flag bit is PBSA_ERR_INVALID_ARG). */
+#define PBSA_OVERLAP_PREVIOUS 1
 PBSA_API pbsa_status pbsa_blockify_kv(const pbsa_geom* g, const void* k, const void* v, int n_frames,
                           float* k_reps, float* v_reps, int rep_slots, const int* dst_slot,
-                          void* k_pool, void* v_pool, int pool_slots, void* ws, void* stream);
+                          void* k_pool, void* v_pool, int pool_slots, int flags, void* ws, void* stream);
 
 /* a2 -- coarse score + top-k: for each head h and query block r,
  *   score(r, c) = scale * <q_reps[h][r], k_reps[h][cand_slot[h][c]]>  (fp32)

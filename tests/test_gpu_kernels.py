@@ -72,7 +72,7 @@ def test_blockify_kv_one_launch(w, n_frames, with_v_reps):
     v_pool = torch.zeros_like(k_pool)
     ws = ws_for(g)
     P.pbsa_blockify_kv(g, k.to(DEV), v.to(DEV), n_frames, k_reps, v_reps, slots, dst.to(DEV), k_pool, v_pool,
-                       slots, ws)
+                       slots, ws=ws)
     check_no_device_error(ws)
     want_k = O.block_reps(f64(k), geom_dict(w), n_frames)
     want_v = O.block_reps(f64(v), geom_dict(w), n_frames)
