@@ -193,9 +193,11 @@ def algorithmic_bytes(w, ncopy: int):
         "blockify_score_select": tok + reps_q + H * nwin * d * 4 + H * nq * (w.capacity + w.topk) * 4
         + H * w.capacity * 4,
         "commit_blockify_kv": 2 * (tok + tok) + 2 * reps_q,
-        # scores/softmax: q reps + pool reps + p matrix (write, read); copies: K+V+reps per promotion
-        "memory_update": reps_q + H * (w.capacity + w.chunk_frames * bpf) * d * 4
-        + 2 * H * nq * (w.capacity + w.chunk_frames * bpf) * 4 + ncopy * 2 * (2 * 64 * d * 2 + d * 4),
+        # plan: q reps + pool reps read, slot tables and lists (the score matrix stays on chip)
+        "memory_update_plan": reps_q + H * (w.capacity + w.chunk_frames * bpf) * d * 4
+        + H * w.capacity * 4 * 4,
+        # apply: K, V blocks and k_reps rows of every promoted block, read and written
+        "memory_update_apply": ncopy * 2 * (2 * 64 * d * 2 + d * 4),
     }
 
 
@@ -379,28 +381,33 @@ def run_variant(P, I, dev, w, steps: int, **cfg_changes):
         step.restore(snap)
         step.run(qd, kcd, vcd, o)
     torch.cuda.synchronize(dev)
-    marks = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(6)]
-    graph = step.capture(qd, kcd, vcd, o, marks=marks)
+    ends = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+    graph = step.capture(qd, kcd, vcd, o, ends=ends)
+    marks = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(7)]
+    graph_parts = step.capture(qd, kcd, vcd, o, marks=marks)
     if cfg.own_chunk:   # the chunk's K, V are written before the selection
-        spans = {"commit_blockify_kv": (0, 1), "blockify_select": (1, 2), "attend": (2, 3), "memory_update": (4, 5)}
+        spans = {"commit_blockify_kv": (0, 1), "blockify_select": (1, 2), "attend": (2, 3),
+                 "memory_update_plan": (4, 5), "memory_update_apply": (5, 6)}
     else:
-        spans = {"blockify_select": (0, 2), "attend": (2, 3), "commit_blockify_kv": (3, 4), "memory_update": (4, 5)}
+        spans = {"blockify_select": (0, 2), "attend": (2, 3), "commit_blockify_kv": (3, 4),
+                 "memory_update_plan": (4, 5), "memory_update_apply": (5, 6)}
     runs = {g: [] for g in spans}
     total = []
     for s in range(steps + 3):
-        step.restore(snap)
-        flush.fill_(1)
-        graph.replay()
-        torch.cuda.synchronize(dev)
+        for gr in (graph, graph_parts):
+            step.restore(snap)
+            flush.fill_(1)
+            gr.replay()
+            torch.cuda.synchronize(dev)
         if s >= 3:
             for g, (a, b) in spans.items():
                 runs[g].append(marks[a].elapsed_time(marks[b]))
-            total.append(marks[0].elapsed_time(marks[5]))
+            total.append(ends[0].elapsed_time(ends[1]))
     _check_device(P, cache.ws, "in a variant run")
     flops = step.flops()
     per = {g: statistics.mean(x) for g, x in runs.items()}
     ms = statistics.mean(total)
-    del graph
+    del graph, graph_parts
     return {"policy": cfg_changes, "ms_per_chunk_decode": ms, "kernels_ms": per,
             "selected_flops": flops, "value_tflops": flops / (ms * 1e-3) / 1e12,
             "attend_tflops": flops / (per["attend"] * 1e-3) / 1e12}
@@ -463,7 +470,7 @@ def run_pbsa(args, w, rank, world, local_rank):
     # the kernel groups gives the per-kernel breakdown
     ends = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
     graph = step.capture(qd, kcd, vcd, o, ends=ends)
-    marks = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(6)]
+    marks = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(7)]
     graph_parts = step.capture(qd, kcd, vcd, o, marks=marks)
     torch.cuda.synchronize(dev)
 
@@ -492,7 +499,7 @@ def run_pbsa(args, w, rank, world, local_rank):
     # kernel groups by the in-graph marks they lie between (marks 1 and 2 are adjacent: the
     # fused blockify + select is one kernel); outside the timed region
     spans = {"blockify_score_select": (0, 2), "attend": (2, 3), "commit_blockify_kv": (3, 4),
-             "memory_update": (4, 5)}
+             "memory_update_plan": (4, 5), "memory_update_apply": (5, 6)}
     groups = list(spans)
     per_runs = {g: [] for g in groups}
     parts_total = []
@@ -501,7 +508,7 @@ def run_pbsa(args, w, rank, world, local_rank):
         torch.cuda.synchronize(dev)
         for g, (a, b) in spans.items():
             per_runs[g].append(marks[a].elapsed_time(marks[b]))
-        parts_total.append(marks[0].elapsed_time(marks[5]))
+        parts_total.append(marks[0].elapsed_time(marks[6]))
     per = {g: statistics.mean(v) for g, v in per_runs.items()}
     step_ms = statistics.mean(step_runs)
     step_ms_max = max_over_ranks(step_ms, dev, world)

@@ -64,6 +64,9 @@ _SIGS = {
     "pbsa_attend": (_I, [ctypes.POINTER(Geom), _P, _I, _P, _P, _I, _P, _P, _I, _P, _P, _P, _P]),
     "pbsa_memory_update": (_I, [ctypes.POINTER(Geom), _P, _I, _P, _P, _P, _I, _P, _P, _I, _I, _P,
                                 _P, _I, ctypes.c_float, _P, _P, _P, _P]),
+    "pbsa_memory_update_plan": (_I, [ctypes.POINTER(Geom), _P, _I, _P, _I, _P, _P, _I, _I, _P, _P, _I,
+                                     ctypes.c_float, _P, _P, _I, _P, _P]),
+    "pbsa_memory_update_apply": (_I, [ctypes.POINTER(Geom), _P, _P, _P, _I, _I, _I, _P, _P]),
     "pbsa_memory_update_noalloc": (_I, [ctypes.POINTER(Geom), _P, _I, _P, _P, _P, _I, _P, _P, _I, _I,
                                         _P, _P, _I, ctypes.c_float, _P, _P, _P]),
     "pbsa_get_device_error": (_I, [_P, _P]),
@@ -217,6 +220,23 @@ def pbsa_memory_update(g: Geom, q_reps, nq, k_reps, k_pool, v_pool, pool_slots, 
         n_sink_gid, _ptr(cand_slot, torch.int32, "cand_slot"), _ptr(cand_gid, torch.int32, "cand_gid"),
         ncand, float(gamma), _ptr(p_list, torch.int32, "p_list"), _ptr(p_cnt, torch.int32, "p_cnt"),
         _ptr(ws, None, "ws"), _stream(stream)))
+
+
+def pbsa_memory_update_plan(g: Geom, q_reps, nq, k_reps, pool_slots, slot_gid, slot_ema, capacity, n_sink_gid,
+                            cand_slot, cand_gid, ncand, gamma, p_list=None, p_cnt=None, flags=0, ws=None,
+                            stream=None):
+    _check("pbsa_memory_update_plan", load().pbsa_memory_update_plan(
+        ctypes.byref(g), _ptr(q_reps, torch.float32, "q_reps"), nq, _ptr(k_reps, torch.float32, "k_reps"),
+        pool_slots, _ptr(slot_gid, torch.int32, "slot_gid"), _ptr(slot_ema, torch.float32, "slot_ema"),
+        capacity, n_sink_gid, _ptr(cand_slot, torch.int32, "cand_slot"), _ptr(cand_gid, torch.int32, "cand_gid"),
+        ncand, float(gamma), _ptr(p_list, torch.int32, "p_list"), _ptr(p_cnt, torch.int32, "p_cnt"), flags,
+        _ptr(ws, None, "ws"), _stream(stream)))
+
+
+def pbsa_memory_update_apply(g: Geom, k_reps, k_pool, v_pool, pool_slots, capacity, ncand, ws=None, stream=None):
+    _check("pbsa_memory_update_apply", load().pbsa_memory_update_apply(
+        ctypes.byref(g), _ptr(k_reps, torch.float32, "k_reps"), _ptr(k_pool, _tok_dtype(g), "k_pool"),
+        _ptr(v_pool, _tok_dtype(g), "v_pool"), pool_slots, capacity, ncand, _ptr(ws, None, "ws"), _stream(stream)))
 
 
 def pbsa_memory_update_noalloc(g: Geom, q_reps, nq, k_reps, k_pool, v_pool, pool_slots, slot_gid,

@@ -341,8 +341,8 @@ class ChunkDecodeStep:
         c = cache.cfg
         self.cache = cache
         self.fused_select = fused_select
-        # kernels per run(): [blockify(Q) + select] (1 fused or 2) + attend + blockify K, V (2)
-        # + memory update (2); the commit of K and V is one launch
+        # kernels per run(): [blockify(Q) + select] (1 fused or 2) + attend + commit of K and V (1)
+        # + memory update (plan + apply)
         self.LAUNCHES = (1 if fused_select else 2) + 1 + 1 + 2
         self.q_frames = q_frames or c.chunk_frames
         if cache._cand is None:
@@ -374,10 +374,11 @@ class ChunkDecodeStep:
         return 4.0 * 64 * 64 * c.head_dim * cnt
 
     def run(self, q, k, v, o, lse=None, stream=None, marks=None):
-        """``marks``: optional list of 6 torch.cuda.Event recorded around the kernel groups:
+        """``marks``: optional list of 7 torch.cuda.Event recorded around the kernel groups:
         0 | blockify Q (+ select) | 1 | select | 2 | attend | 3 | commit blockify K+V | 4 | memory
-        update | 5.  For the own-chunk variant the chunk's blockify K+V runs first (between
-        marks 0 and 1), the fused selection between 1 and 2, and nothing between 3 and 4."""
+        update plan | 5 | memory update apply (copies) | 6.  For the own-chunk variant the chunk's
+        blockify K+V runs first (between marks 0 and 1), the fused selection between 1 and 2, and
+        nothing between 3 and 4.  Without marks the plan and the commit overlap attend."""
         ca, c = self.cache, self.cache.cfg
         g, ws, ps = ca.geom, ca.ws, ca.pool_slots
         if marks is not None:
@@ -407,24 +408,39 @@ class ChunkDecodeStep:
         L.pbsa_attend(g, q, self.q_frames, ca.k_pool, ca.v_pool, ps, self.kv_slot, self.kv_cnt, ca.kv_ld,
                       o, lse, ws=ws, stream=stream)
         mk(3)
-        if not own:
-            # the commit writes only free ring slots, which the attend lists never name: without
-            # timing events in between it may start on SMs that attend's last wave leaves idle
-            flags = L.PBSA_OVERLAP_PREVIOUS if marks is None else 0
-            L.pbsa_blockify_kv(g, k, v, self.q_frames, ca.k_reps, None, ps, self.dst, ca.k_pool, ca.v_pool, ps,
-                               flags=flags, ws=ws, stream=stream)
-        mk(4)
-        L.pbsa_memory_update(g, self.q_reps, self.nq, ca.k_reps, ca.k_pool, ca.v_pool, ps, ca.slot_gid,
-                             ca.slot_ema, c.capacity, c.bpf, self.cs, self.cg, self.ncand, c.gamma,
-                             ca.p_list, ca.p_cnt, ws=ws, stream=stream)
-        mk(5)
+        if marks is None:
+            # Programmatic dependents of attend: the memory update's plan (scores, ranking, slot
+            # table; no pool access) and the commit of K, V (free ring slots, which the attend
+            # lists never name) run on the SMs that attend's last wave leaves idle; the copies
+            # of promoted blocks into persistent slots wait until attend has finished.
+            L.pbsa_memory_update_plan(g, self.q_reps, self.nq, ca.k_reps, ps, ca.slot_gid, ca.slot_ema, c.capacity,
+                                      c.bpf, self.cs, self.cg, self.ncand, c.gamma, ca.p_list, ca.p_cnt,
+                                      flags=L.PBSA_OVERLAP_PREVIOUS, ws=ws, stream=stream)
+            if not own:
+                L.pbsa_blockify_kv(g, k, v, self.q_frames, ca.k_reps, None, ps, self.dst, ca.k_pool, ca.v_pool, ps,
+                                   flags=L.PBSA_OVERLAP_PREVIOUS, ws=ws, stream=stream)
+            L.pbsa_memory_update_apply(g, ca.k_reps, ca.k_pool, ca.v_pool, ps, c.capacity, self.ncand, ws=ws,
+                                       stream=stream)
+        else:
+            # the same kernels, serialised between the timing events
+            if not own:
+                L.pbsa_blockify_kv(g, k, v, self.q_frames, ca.k_reps, None, ps, self.dst, ca.k_pool, ca.v_pool, ps,
+                                   ws=ws, stream=stream)
+            mk(4)
+            L.pbsa_memory_update_plan(g, self.q_reps, self.nq, ca.k_reps, ps, ca.slot_gid, ca.slot_ema, c.capacity,
+                                      c.bpf, self.cs, self.cg, self.ncand, c.gamma, ca.p_list, ca.p_cnt, ws=ws,
+                                      stream=stream)
+            mk(5)
+            L.pbsa_memory_update_apply(g, ca.k_reps, ca.k_pool, ca.v_pool, ps, c.capacity, self.ncand, ws=ws,
+                                       stream=stream)
+        mk(6)
         return o
 
     def capture(self, q, k, v, o, lse=None, marks=None, ends=None) -> torch.cuda.CUDAGraph:
         """Capture ``run`` in a CUDA graph (one launch replays all kernels of the step).
 
         Call ``run`` once before capturing (kernel attributes are set on first use).  With
-        ``marks`` (6 events between the kernel groups) or ``ends`` (2 events around the whole
+        ``marks`` (7 events between the kernel groups) or ``ends`` (2 events around the whole
         step, which leave the commit free to overlap attend), pass events created with
         ``external=True`` so they time inside the graph.
         """

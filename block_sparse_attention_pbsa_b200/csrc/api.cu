@@ -243,6 +243,41 @@ pbsa_status pbsa_memory_update(const pbsa_geom* gin, const float* q_reps, int nq
                                         gamma, p_list, p_cnt, ws, static_cast<cudaStream_t>(stream)));
 }
 
+pbsa_status pbsa_memory_update_plan(const pbsa_geom* gin, const float* q_reps, int nq, const float* k_reps,
+                                    int pool_slots, int* slot_gid, float* slot_ema, int capacity, int n_sink_gid,
+                                    const int* cand_slot, const int* cand_gid, int ncand, float gamma, int* p_list,
+                                    int* p_cnt, int flags, void* ws, void* stream) {
+  Geo g;
+  pbsa_status s = make_geo(gin, &g);
+  if (s != PBSA_OK) return s;
+  if (q_reps == nullptr || k_reps == nullptr || slot_gid == nullptr || slot_ema == nullptr || ws == nullptr)
+    return PBSA_ERR_INVALID_ARG;
+  if (nq <= 0 || capacity <= 0 || ncand < 0 || n_sink_gid < 0) return PBSA_ERR_INVALID_ARG;
+  if (ncand > 0 && (cand_slot == nullptr || cand_gid == nullptr)) return PBSA_ERR_INVALID_ARG;
+  if (!(gamma >= 0.f && gamma <= 1.f)) return PBSA_ERR_INVALID_ARG;
+  if (!pool_ok(g, pool_slots) || capacity > pool_slots) return PBSA_ERR_INVALID_ARG;
+  if (!aligned16(k_reps) || !aligned16(q_reps)) return PBSA_ERR_INVALID_ARG;
+  if ((flags & ~PBSA_OVERLAP_PREVIOUS) != 0) return PBSA_ERR_INVALID_ARG;
+  if (capacity + ncand > 2048 || nq > 65535) return PBSA_ERR_UNSUPPORTED;
+  return from_cuda(launch_memory_update_plan(g, q_reps, nq, k_reps, pool_slots, slot_gid, slot_ema, capacity,
+                                             n_sink_gid, cand_slot, cand_gid, ncand, gamma, p_list, p_cnt,
+                                             (flags & PBSA_OVERLAP_PREVIOUS) != 0, ws,
+                                             static_cast<cudaStream_t>(stream)));
+}
+
+pbsa_status pbsa_memory_update_apply(const pbsa_geom* gin, float* k_reps, void* k_pool, void* v_pool,
+                                     int pool_slots, int capacity, int ncand, void* ws, void* stream) {
+  Geo g;
+  pbsa_status s = make_geo(gin, &g);
+  if (s != PBSA_OK) return s;
+  if (k_reps == nullptr || k_pool == nullptr || v_pool == nullptr || ws == nullptr) return PBSA_ERR_INVALID_ARG;
+  if (capacity <= 0 || ncand < 0 || !pool_ok(g, pool_slots) || capacity > pool_slots) return PBSA_ERR_INVALID_ARG;
+  if (!aligned16(k_pool) || !aligned16(v_pool) || !aligned16(k_reps)) return PBSA_ERR_INVALID_ARG;
+  if (capacity + ncand > 2048) return PBSA_ERR_UNSUPPORTED;
+  return from_cuda(launch_memory_update_apply(g, k_reps, k_pool, v_pool, pool_slots, capacity, ncand, ws,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
 size_t pbsa_bwd_workspace_bytes(const pbsa_geom* gin, int q_frames, int pool_slots, int kv_ld) {
   Geo g;
   if (make_geo(gin, &g) != PBSA_OK || q_frames <= 0 || pool_slots <= 0 || kv_ld <= 0) return 0;

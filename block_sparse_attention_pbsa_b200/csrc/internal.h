@@ -70,6 +70,15 @@ cudaError_t launch_memory_update(const Geo& g, const float* q_reps, int nq, floa
                                  const int* cand_gid, int ncand, float gamma, int* p_list,
                                  int* p_cnt, void* ws, cudaStream_t st);
 
+// The update in two launches: plan (scores, ranking, slot table, copy list in ws; no pool
+// access) and apply (the copies).  overlap_previous: programmatic dependent launch of the plan.
+cudaError_t launch_memory_update_plan(const Geo& g, const float* q_reps, int nq, const float* k_reps,
+                                      int pool_slots, int* slot_gid, float* slot_ema, int C, int n_sink_gid,
+                                      const int* cand_slot, const int* cand_gid, int ncand, float gamma,
+                                      int* p_list, int* p_cnt, bool overlap_previous, void* ws, cudaStream_t st);
+cudaError_t launch_memory_update_apply(const Geo& g, float* k_reps, void* k_pool, void* v_pool, int pool_slots,
+                                       int C, int ncand, void* ws, cudaStream_t st);
+
 size_t attend_bwd_ws_bytes(const Geo& g, int q_frames, int pool_slots, int kv_ld);
 cudaError_t launch_attend_bwd(const Geo& g, const void* q, int q_frames, const void* k_pool,
                               const void* v_pool, int pool_slots, const int* kv_slot,

@@ -36,17 +36,20 @@ constexpr int MU_BATCH = 12;   // pool entries per warp in flight
 struct MuLayout {
   size_t part_off, copy_off, ncopy_off, count_off, end;
 };
-// part [H][ceil(nq / MU_RQ)][nb] column partial sums; copy list [H][2][nb] (sources, then
-// destinations); ncopy [H];
-// count [H] finished score CTAs per head (zero between calls)
+constexpr int MU_MAX_HEADS = 4096;   // the geometry's limit on heads
+// count [MU_MAX_HEADS] finished score CTAs per head, at a fixed offset for every shape (zero
+// between calls; no other data ever lands there, whatever shapes share the workspace); copy
+// list [H][2][nb] (sources, then destinations); ncopy [H]; part [H][ceil(nq / MU_RQ)][nb] column
+// partial sums.  The copy list's offset depends on H and nb only (the apply step finds it
+// without nq).
 __host__ __device__ inline MuLayout mu_layout(int H, int nq, int nb) {
   MuLayout L;
   const size_t nqb = (size_t)(nq + MU_RQ - 1) / MU_RQ;
-  L.part_off = WS_HEADER_BYTES;
-  L.copy_off = L.part_off + align256((size_t)H * nqb * nb * sizeof(float));
+  L.count_off = WS_HEADER_BYTES;
+  L.copy_off = L.count_off + align256((size_t)MU_MAX_HEADS * sizeof(int));
   L.ncopy_off = L.copy_off + align256((size_t)H * nb * 2 * sizeof(int));
-  L.count_off = L.ncopy_off + align256((size_t)H * sizeof(int));
-  L.end = L.count_off + align256((size_t)H * sizeof(int));
+  L.part_off = L.ncopy_off + align256((size_t)H * sizeof(int));
+  L.end = L.part_off + align256((size_t)H * nqb * nb * sizeof(float));
   return L;
 }
 
@@ -633,6 +636,197 @@ __global__ void __cluster_dims__(MF_NC, 1, 1) __launch_bounds__(MF_THREADS, 1) m
   if (tid < mine && !copy_ok(tid)) record_error(ws, PBSA_ERR_DEVICE_INDEX, my_src[tid], K_MU_COPY);
 }
 
+// ---------------------------------------------------------------------------- plan / apply
+// The update split in two: mu_plan_kernel scores, ranks and assigns (slot table, persistent
+// list, copy list in the workspace) without touching the K/V pools, so it may run while the
+// attention of the same chunk still reads them; mu_copy_kernel then applies the copy list.
+// One CTA per head (up to MF_MAX_NB pool entries, any number of query blocks): the pool
+// representatives are staged once; query rows go through the MMA tile 16 at a time (scores by
+// split-TF32 MMAs, softmax per row by one warp, column sums in row order).  Launched as a
+// programmatic dependent, the grid signals its own dependents at once and waits for the grid
+// it overlaps before completing.
+template <int D>
+__global__ void __launch_bounds__(MF_THREADS, 1) mu_plan_kernel(
+    const float* __restrict__ q_reps, int nq, const float* __restrict__ k_reps, int pool_slots,
+    int* __restrict__ slot_gid, float* __restrict__ slot_ema, int C, int n_sink_gid,
+    const int* __restrict__ cand_slot, const int* __restrict__ cand_gid, int ncand, float gamma, float scale,
+    int* __restrict__ copy_list, int* __restrict__ ncopy, int* __restrict__ p_list, int* __restrict__ p_cnt,
+    void* ws) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  using L = MfLayout<float, D>;
+  constexpr int KS = L::KS, CH = D / 4;
+  extern __shared__ uint8_t mp_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(mp_raw) + 127) & ~(uintptr_t)127);
+  float* kb = reinterpret_cast<float*>(sm);
+  float* qs = reinterpret_cast<float*>(sm + L::OFF_Q);
+  float* ss = reinterpret_cast<float*>(sm + L::OFF_S);
+  int* gid = reinterpret_cast<int*>(sm + L::OFF_GID);
+  int* eslot = reinterpret_cast<int*>(sm + L::OFF_ESLOT);
+  float* col = reinterpret_cast<float*>(sm + L::OFF_COL);
+  float* prev = reinterpret_cast<float*>(sm + L::OFF_PREV);
+  const int h = blockIdx.x, nb = C + ncand;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const float* krep_h = k_reps + (size_t)h * pool_slots * D;
+
+  // ---- entries and representatives (a persistent entry's slot is its index)
+  for (int i = tid; i < C * CH; i += MF_THREADS) {
+    const int j = i / CH, e = i - j * CH;
+    cp_async16(kb + j * KS + 4 * e, krep_h + (size_t)j * D + 4 * e);
+  }
+  if (tid < MF_MAX_NB) {
+    int sl = 0;
+    gid[tid] = tid < nb ? entry_of(tid, h, C, ncand, pool_slots, slot_gid, cand_slot, cand_gid, &sl, ws, true) : -1;
+    eslot[tid] = sl;
+    col[tid] = 0.f;
+    if (tid < C) prev[tid] = slot_ema[(size_t)h * C + tid];
+  }
+  __syncthreads();
+  for (int i = tid; i < ncand * CH; i += MF_THREADS) {
+    const int j = C + i / CH, e = i % CH;
+    if (gid[j] >= 0) cp_async16(kb + j * KS + 4 * e, krep_h + (size_t)eslot[j] * D + 4 * e);
+  }
+
+  // ---- query rows 16 at a time: scores, softmax, column sums (rows in order)
+  const int gq = lane >> 2, t4 = lane & 3;
+  const int ntiles = (nb + 7) / 8;
+  for (int r0 = 0; r0 < nq; r0 += MF_MAX_R) {
+    const int nr = min(MF_MAX_R, nq - r0);
+    for (int i = tid; i < MF_MAX_R * CH; i += MF_THREADS) {
+      const int r = i / CH, e = i - r * CH;
+      if (r < nr) cp_async16(qs + r * KS + 4 * e, q_reps + ((size_t)h * nq + r0 + r) * D + 4 * e);
+      else reinterpret_cast<float4*>(qs + r * KS)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    cp_async_wait_all();
+    __syncthreads();
+    for (int nt = warp; nt < ntiles; nt += MF_THREADS / 32) {
+      float acc[6][4] = {};
+      const float* brow = kb + (nt * 8 + gq) * KS;
+#pragma unroll
+      for (int k0 = 0; k0 < D; k0 += 8) {
+        const int par = (k0 >> 3) & 1;
+        uint32_t ah[4], al[4], bh0, bl0, bh1, bl1;
+        tf32_split(qs[gq * KS + k0 + t4], ah[0], al[0]);
+        tf32_split(qs[(gq + 8) * KS + k0 + t4], ah[1], al[1]);
+        tf32_split(qs[gq * KS + k0 + t4 + 4], ah[2], al[2]);
+        tf32_split(qs[(gq + 8) * KS + k0 + t4 + 4], ah[3], al[3]);
+        tf32_split(brow[k0 + t4], bh0, bl0);
+        tf32_split(brow[k0 + t4 + 4], bh1, bl1);
+        mma_tf32(acc[3 * par + 0], al, bh0, bh1);
+        mma_tf32(acc[3 * par + 1], ah, bl0, bl1);
+        mma_tf32(acc[3 * par + 2], ah, bh0, bh1);
+      }
+      float r4[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        r4[e] = ((acc[0][e] + acc[3][e]) + (acc[1][e] + acc[4][e])) + (acc[2][e] + acc[5][e]);
+      *reinterpret_cast<float2*>(ss + gq * MF_SCS + nt * 8 + 2 * t4) = make_float2(r4[0], r4[1]);
+      *reinterpret_cast<float2*>(ss + (gq + 8) * MF_SCS + nt * 8 + 2 * t4) = make_float2(r4[2], r4[3]);
+    }
+    __syncthreads();
+    for (int r = warp; r < nr; r += MF_THREADS / 32) {
+      float* row = ss + r * MF_SCS;
+      float m = -INFINITY;
+      for (int j = lane; j < nb; j += 32) m = fmaxf(m, gid[j] >= 0 ? row[j] * scale : -INFINITY);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      float sum = 0.f;
+      for (int j = lane; j < nb; j += 32) sum += gid[j] >= 0 ? expf(row[j] * scale - m) : 0.f;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      const float inv = sum > 0.f ? 1.0f / sum : 0.f;
+      for (int j = lane; j < nb; j += 32) row[j] = gid[j] >= 0 ? expf(row[j] * scale - m) * inv : 0.f;
+    }
+    __syncthreads();
+    if (tid < nb) {
+      float a = col[tid];
+      for (int r = 0; r < nr; ++r) a += ss[r * MF_SCS + tid];
+      col[tid] = a;
+    }
+    __syncthreads();   // qs and ss are rewritten by the next tile
+  }
+
+  // ---- a_b = mean over the rows, EMA, ranking, slot assignment
+  {
+    float* ema = reinterpret_cast<float*>(sm + L::OFF_SEL);
+    uint64_t* key = reinterpret_cast<uint64_t*>(ema + MF_MAX_NB);
+    int* rank = reinterpret_cast<int*>(key + MF_MAX_NB);
+    int* by_rank = rank + MF_MAX_NB;
+    int* filled = by_rank + MF_MAX_NB;
+    int* flist = filled + MF_MAX_NB;
+    int* plist2 = flist + MF_MAX_NB;
+    if (tid < nb) ema[tid] = col[tid] * (1.0f / (float)nq);
+    __syncthreads();
+    mu_select_head(h, nb, pool_slots, slot_gid, slot_ema, prev, C, n_sink_gid, gamma, gid, eslot, ema, key, rank,
+                   by_rank, filled, flist, plist2, copy_list + (size_t)h * nb * 2,
+                   copy_list + (size_t)h * nb * 2 + nb, ncopy + h, p_list, p_cnt, ws);
+  }
+  // a programmatic dependent of another grid completes only after it (no-op otherwise)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+template <int D>
+cudaError_t launch_plan(const Geo& g, const float* q_reps, int nq, const float* k_reps, int pool_slots,
+                        int* slot_gid, float* slot_ema, int C, int n_sink_gid, const int* cand_slot,
+                        const int* cand_gid, int ncand, float gamma, int* p_list, int* p_cnt, bool overlap_previous,
+                        void* ws, cudaStream_t st) {
+  const int nb = C + ncand;
+  const MuLayout L = mu_layout(g.H, nq, nb);
+  char* base = static_cast<char*>(ws);
+  int* copy_list = reinterpret_cast<int*>(base + L.copy_off);
+  int* ncopy = reinterpret_cast<int*>(base + L.ncopy_off);
+  cudaError_t e;
+  if (nb <= MF_MAX_NB) {
+    auto kern = mu_plan_kernel<D>;
+    constexpr int smem = MfLayout<float, D>::BYTES;
+    if ((e = set_smem_once((const void*)kern, smem)) != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(g.H);
+    cfg.blockDim = dim3(MF_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = overlap_previous ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, q_reps, nq, k_reps, pool_slots, slot_gid, slot_ema, C, n_sink_gid,
+                              cand_slot, cand_gid, ncand, gamma, g.scale, copy_list, ncopy, p_list, p_cnt, ws);
+  }
+  // larger pools: the score kernel of the two-launch path (an ordinary launch: it does not
+  // wait for a grid it would overlap)
+  float* part = reinterpret_cast<float*>(base + L.part_off);
+  int* count = reinterpret_cast<int*>(base + L.count_off);
+  const size_t sel = (size_t)14 * nb * 4 + 16, sco = (size_t)MU_RQ * nb * 4;
+  const size_t smem = (size_t)2 * nb * 4 + (size_t)MU_RQ * D * 4 + (sel > sco ? sel : sco);
+  if ((e = set_smem_once((const void*)mu_score_select_kernel<D>, (int)smem)) != cudaSuccess) return e;
+  mu_score_select_kernel<D><<<dim3((nq + MU_RQ - 1) / MU_RQ, g.H), MU_THREADS, smem, st>>>(
+      const_cast<float*>(q_reps), nq, const_cast<float*>(k_reps), pool_slots, slot_gid, slot_ema, C, n_sink_gid,
+      cand_slot, cand_gid, ncand, gamma, g.scale, part, copy_list, ncopy, count, p_list, p_cnt, ws);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_apply(const Geo& g, float* k_reps, void* k_pool, void* v_pool, int pool_slots, int C, int ncand,
+                         void* ws, cudaStream_t st) {
+  const int nb = C + ncand;
+  const MuLayout L = mu_layout(g.H, 1, nb);
+  char* base = static_cast<char*>(ws);
+  const int* copy_list = reinterpret_cast<const int*>(base + L.copy_off);
+  const int* ncopy = reinterpret_cast<const int*>(base + L.ncopy_off);
+  const int max_copies = C < nb ? C : nb;
+  if (max_copies <= 0) return cudaSuccess;
+  dim3 grid(max_copies, g.H, 2);
+  if (g.dtype == PBSA_BF16)
+    mu_copy_kernel<__nv_bfloat16, D><<<grid, MU_THREADS, 0, st>>>(copy_list, ncopy, nb, C, k_reps,
+                                                                  static_cast<__nv_bfloat16*>(k_pool),
+                                                                  static_cast<__nv_bfloat16*>(v_pool), pool_slots, ws);
+  else
+    mu_copy_kernel<float, D><<<grid, MU_THREADS, 0, st>>>(copy_list, ncopy, nb, C, k_reps,
+                                                          static_cast<float*>(k_pool), static_cast<float*>(v_pool),
+                                                          pool_slots, ws);
+  return cudaGetLastError();
+}
+
 template <int D>
 cudaError_t launch_mu(const Geo& g, const float* q_reps, int nq, float* k_reps, void* k_pool,
                       void* v_pool, int pool_slots, int* slot_gid, float* slot_ema, int C,
@@ -705,6 +899,32 @@ cudaError_t launch_memory_update(const Geo& g, const float* q_reps, int nq, floa
   if (g.d == 64) { PBSA_MU(64) }
   if (g.d == 32) { PBSA_MU(32) }
 #undef PBSA_MU
+  return cudaErrorNotSupported;
+}
+
+}  // namespace pbsa
+
+namespace pbsa {
+
+cudaError_t launch_memory_update_plan(const Geo& g, const float* q_reps, int nq, const float* k_reps,
+                                      int pool_slots, int* slot_gid, float* slot_ema, int C, int n_sink_gid,
+                                      const int* cand_slot, const int* cand_gid, int ncand, float gamma,
+                                      int* p_list, int* p_cnt, bool overlap_previous, void* ws, cudaStream_t st) {
+#define PBSA_MP(DD)                                                                                          \
+  return launch_plan<DD>(g, q_reps, nq, k_reps, pool_slots, slot_gid, slot_ema, C, n_sink_gid, cand_slot,   \
+                         cand_gid, ncand, gamma, p_list, p_cnt, overlap_previous, ws, st);
+  if (g.d == 128) { PBSA_MP(128) }
+  if (g.d == 64) { PBSA_MP(64) }
+  if (g.d == 32) { PBSA_MP(32) }
+#undef PBSA_MP
+  return cudaErrorNotSupported;
+}
+
+cudaError_t launch_memory_update_apply(const Geo& g, float* k_reps, void* k_pool, void* v_pool, int pool_slots,
+                                       int C, int ncand, void* ws, cudaStream_t st) {
+  if (g.d == 128) return launch_apply<128>(g, k_reps, k_pool, v_pool, pool_slots, C, ncand, ws, st);
+  if (g.d == 64) return launch_apply<64>(g, k_reps, k_pool, v_pool, pool_slots, C, ncand, ws, st);
+  if (g.d == 32) return launch_apply<32>(g, k_reps, k_pool, v_pool, pool_slots, C, ncand, ws, st);
   return cudaErrorNotSupported;
 }
 

@@ -250,6 +250,30 @@ PBSA_API pbsa_status pbsa_memory_update(const pbsa_geom* g, const float* q_reps,
                                const int* cand_slot, const int* cand_gid, int ncand,
                                float gamma, int* p_list, int* p_cnt, void* ws, void* stream);
 
+/* a4 in two launches, so that the scoring can overlap other work.  Together,
+ *   pbsa_memory_update_plan(...) ; pbsa_memory_update_apply(...)
+ * compute what pbsa_memory_update computes (the same rule; the column sums of the softmax may
+ * be added in another order, so EMA values may differ in the last bits).
+ * plan: everything but the block copies -- scores, softmax, EMA, ranking, the new slot_gid /
+ *   slot_ema, p_list / p_cnt, and the copy list, which it leaves in `ws`.  It reads q_reps,
+ *   k_reps, the slot table and the candidate lists; it never touches k_pool / v_pool.
+ *   flags: 0, or PBSA_OVERLAP_PREVIOUS (pools of up to 256 entries): launch as a programmatic
+ *   dependent of the previous kernel on `stream`, which may still be running (e.g. pbsa_attend
+ *   of the same chunk, which reads the pools but nothing plan writes); plan completes only
+ *   after that kernel.  Larger pools ignore the flag.
+ * apply: copies the promoted blocks (K, V and k_reps rows) as listed in `ws`; `ws`, capacity
+ *   and ncand must be those of the plan call, with nothing else using `ws` in between.
+ * Arguments otherwise as for pbsa_memory_update; workspace pbsa_workspace_bytes(g, nq,
+ * capacity + ncand). */
+PBSA_API pbsa_status pbsa_memory_update_plan(const pbsa_geom* g, const float* q_reps, int nq,
+                               const float* k_reps, int pool_slots, int* slot_gid, float* slot_ema,
+                               int capacity, int n_sink_gid, const int* cand_slot, const int* cand_gid,
+                               int ncand, float gamma, int* p_list, int* p_cnt, int flags, void* ws,
+                               void* stream);
+PBSA_API pbsa_status pbsa_memory_update_apply(const pbsa_geom* g, float* k_reps, void* k_pool,
+                               void* v_pool, int pool_slots, int capacity, int ncand, void* ws,
+                               void* stream);
+
 /* pbsa_memory_update without a caller-provided workspace.  The paper has no counterpart;
  * this is a library convenience for callers that cannot allocate device memory (for
  * example a plug-in whose host application owns every device allocation, or a runtime

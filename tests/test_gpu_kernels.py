@@ -390,8 +390,12 @@ def test_invalid_arguments_are_rejected_on_host():
 
 
 # ----------------------------------------------------------------------------- memory update
+@pytest.mark.parametrize("split", [False, True])
 @pytest.mark.parametrize("n_pers,ncand,C", [(70, 72, 96), (24, 48, 96), (96, 72, 96), (0, 264, 96), (3, 5, 8)])
-def test_memory_update(n_pers, ncand, C):
+def test_memory_update(n_pers, ncand, C, split):
+    """pbsa_memory_update, or (split) pbsa_memory_update_plan + pbsa_memory_update_apply --
+    one CTA per head for pools of up to 256 entries, the two-launch score kernel above -- against
+    the oracle: kept sets (outside EMA near-ties), EMA values, promoted copies, persistent list."""
     H, d, nq, S = 3, 128, 72, min(24, C // 2)
     w = dataclasses.replace(I.DECODE_5S, heads=H)
     g = geom_for(w)
@@ -421,8 +425,13 @@ def test_memory_update(n_pers, ncand, C):
     plist = torch.full((H, C), -5, dtype=torch.int32, device=DEV)
     pcnt = torch.zeros((H,), dtype=torch.int32, device=DEV)
     ws = torch.zeros(P.pbsa_workspace_bytes(g, nq, C + ncand), dtype=torch.uint8, device=DEV)
-    P.pbsa_memory_update(g, qr.to(DEV), nq, kr_d, kp_d, vp_d, pool, sgid_d, sema_d, C, S, cs.to(DEV),
-                         cg.to(DEV), ncand, 0.9, plist, pcnt, ws)
+    if split:
+        P.pbsa_memory_update_plan(g, qr.to(DEV), nq, kr_d, pool, sgid_d, sema_d, C, S, cs.to(DEV), cg.to(DEV), ncand,
+                                  0.9, plist, pcnt, ws=ws)
+        P.pbsa_memory_update_apply(g, kr_d, kp_d, vp_d, pool, C, ncand, ws=ws)
+    else:
+        P.pbsa_memory_update(g, qr.to(DEV), nq, kr_d, kp_d, vp_d, pool, sgid_d, sema_d, C, S, cs.to(DEV),
+                             cg.to(DEV), ncand, 0.9, plist, pcnt, ws)
     check_no_device_error(ws)
     new_gid, new_ema = sgid_d.cpu(), sema_d.cpu()
     for h in range(H):
