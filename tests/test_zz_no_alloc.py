@@ -39,8 +39,12 @@ def _cands(seed, H, C, pool, ncand, first_gid):
     return cs.to(DEV), cg.to(DEV)
 
 
-def test_noalloc_matches_workspace_update_twice():
-    H, d, nq, C, S, ncand = 12, 128, 72, 96, 24, 72
+@pytest.mark.parametrize("ncand", [72, 264])
+def test_noalloc_matches_workspace_update_twice(ncand):
+    # 72 candidates: the one-launch update (its scratch holds the error word); 264: the pool of
+    # 360 entries takes the two-launch path, whose column partial sums, per-head completion
+    # counts and copy list all live in the scratch
+    H, d, nq, C, S = 12, 128, 72, 96, 24
     pool = C + 3 * ncand
     w = dataclasses.replace(I.DECODE_5S, heads=H)
     g = P.make_geom(H, d, w.frame_h, w.frame_w, w.tile_h, w.tile_w, w.scale, "bf16")
