@@ -251,25 +251,31 @@ class PBSALayerCache:
         kv_cnt = torch.full((self.cfg.heads, nq), nq, dtype=torch.int32, device=self.device)
         return self.attend(q, kv_slot, kv_cnt, nq, o, lse, stream)
 
-    def _write_chunk(self, k, v, stream=None):
+    def _write_chunk(self, k, v, stream=None, flags=0):
         n = self.frames_of(k)
         dst = self._frames_dst(self.hist, n)
         # K and V blocks in one launch; value representatives are not used by the method
         L.pbsa_blockify_kv(self.geom, k, v, n, self.k_reps, None, self.pool_slots, dst, self.k_pool,
-                           self.v_pool, self.pool_slots, ws=self.ws, stream=stream)
+                           self.v_pool, self.pool_slots, flags=flags, ws=self.ws, stream=stream)
 
-    def commit(self, k, v, q_reps_last=None, stream=None):
+    def commit(self, k, v, q_reps_last=None, stream=None, overlap=False, split=False):
         """a4: commit the finished chunk (its last-step K, V) and update the persistent memory.
 
         The chunk's blocks enter the ring; the frames that leave the window, and frame 0's
         sink blocks when frame 0 is in the chunk, are the candidates of the memory update,
         scored by the chunk's last-step query representatives.
+
+        ``overlap``: the call directly follows this cache's last ``decode_step`` on the stream,
+        with nothing launched in between.  The memory update's plan and the write of the chunk
+        then run as programmatic dependents of that attend, on the SMs its last wave leaves idle,
+        and the copies of promoted blocks follow it.  (A chunk whose own blocks were attended --
+        the first chunk, the own-chunk variant -- takes the serial order: the write would
+        overlap their reads.)  ``split``: the memory update as plan + apply without the overlap.
         """
         c = self.cfg
         bpf, H = c.bpf, c.heads
         q_reps_last = self.q_reps if q_reps_last is None else q_reps_last
         first, n = self.hist, self.frames_of(k)
-        self._write_chunk(k, v, stream)
         old_win = set(self.window_frames(first))
         new_hist = first + n
         new_win = set(self.window_frames(new_hist))
@@ -278,17 +284,33 @@ class PBSALayerCache:
         cand = [(self.ring_slot(f, t), f * bpf + t) for f in evicted for t in range(bpf)]
         if first == 0:
             cand = [(self.ring_slot(0, t), t) for t in range(bpf)] + cand
-        self._update(q_reps_last, cand, stream)
+        if overlap and not (first == 0 or c.own_chunk):
+            # the candidates are the frames leaving the window, never the chunk's own slots
+            self._update(q_reps_last, cand, stream, split=True, plan_flags=L.PBSA_OVERLAP_PREVIOUS, apply=False)
+            self._write_chunk(k, v, stream, flags=L.PBSA_OVERLAP_PREVIOUS)
+            L.pbsa_memory_update_apply(self.geom, self.k_reps, self.k_pool, self.v_pool, self.pool_slots,
+                                       c.capacity, len(cand), ws=self.ws, stream=stream)
+        else:
+            self._write_chunk(k, v, stream)
+            self._update(q_reps_last, cand, stream, split=split or overlap)
         self.hist = new_hist
         self._refresh_window()
 
-    def _update(self, q_reps, cand, stream=None):
+    def _update(self, q_reps, cand, stream=None, split=False, plan_flags=0, apply=True):
         c, H = self.cfg, self.cfg.heads
         ncand = len(cand)
         cs, cg = self._list_pair(cand) if ncand else (None, None)
-        L.pbsa_memory_update(self.geom, q_reps, q_reps.shape[1], self.k_reps, self.k_pool, self.v_pool,
-                             self.pool_slots, self.slot_gid, self.slot_ema, c.capacity, c.bpf, cs, cg,
-                             ncand, c.gamma, self.p_list, self.p_cnt, ws=self.ws, stream=stream)
+        if not split:
+            L.pbsa_memory_update(self.geom, q_reps, q_reps.shape[1], self.k_reps, self.k_pool, self.v_pool,
+                                 self.pool_slots, self.slot_gid, self.slot_ema, c.capacity, c.bpf, cs, cg,
+                                 ncand, c.gamma, self.p_list, self.p_cnt, ws=self.ws, stream=stream)
+            return
+        L.pbsa_memory_update_plan(self.geom, q_reps, q_reps.shape[1], self.k_reps, self.pool_slots, self.slot_gid,
+                                  self.slot_ema, c.capacity, c.bpf, cs, cg, ncand, c.gamma, self.p_list, self.p_cnt,
+                                  flags=plan_flags, ws=self.ws, stream=stream)
+        if apply:
+            L.pbsa_memory_update_apply(self.geom, self.k_reps, self.k_pool, self.v_pool, self.pool_slots,
+                                       c.capacity, ncand, ws=self.ws, stream=stream)
 
     def prefill(self, k_hist, v_hist, hist_frames: int, q_reps, stream=None):
         """Load a history of ``hist_frames`` frames at once (single-step decode workloads).

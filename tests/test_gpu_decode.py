@@ -205,6 +205,30 @@ def _rollout(w, n_chunks, sample_every=3, k_schedule=None):
     return alive
 
 
+def test_rollout_overlapped_commit_matches_serial():
+    """Each chunk committed right after its last-step attention with the overlap (the write of
+    the chunk and the memory update's plan as programmatic dependents of attend) gives the same
+    outputs and the same cache, bit for bit, as the same kernels run in series."""
+    w = I.ROLLOUT_5S
+    caches = [P.PBSALayerCache(layer_cfg(w)) for _ in range(2)]   # [serial, overlapped]
+    for c, (f0, nf) in enumerate(I.rollout_chunks(w)):
+        wc = dataclasses.replace(w, chunk_frames=nf)
+        for s in range(w.steps):
+            q, k, v = (I.tokens(wc, nf, I.stream_seed(w.seed, c, s, t)).to(DEV) for t in range(3))
+            outs = []
+            for i, ca in enumerate(caches):
+                outs.append(ca.decode_step(q, k, v))
+                if s == w.steps - 1:
+                    ca.commit(k, v, overlap=i == 1, split=i == 0)
+            torch.cuda.synchronize()
+            assert torch.equal(outs[0], outs[1]), (c, s)
+        a, b = caches
+        for name in ("slot_gid", "slot_ema", "k_pool", "v_pool", "k_reps", "p_list", "p_cnt"):
+            assert torch.equal(getattr(a, name), getattr(b, name)), (c, name)
+        for ca in caches:
+            assert P.pbsa_get_device_error(ca.ws) == 0
+
+
 def test_rollout_5s_layer0():
     w = I.ROLLOUT_5S
     alive = _rollout(w, n_chunks=7)
