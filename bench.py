@@ -418,6 +418,83 @@ def run_variant(P, I, dev, w, steps: int, **cfg_changes):
             "attend_tflops": flops / (per["attend"] * 1e-3) / 1e12}
 
 
+def run_hbm_at_scale(P, I, dev, peaks, reps: int = 10):
+    """The HBM-bound kernels at sizes where bandwidth, not launch and first-byte latency, decides:
+    the commit of K and V over an 18-frame history (the prefill's size, 340 MB moved), and the
+    memory update's copies for 30 layers x 12 heads folded into 360 heads, 72 promotions each
+    (1.7 GB moved).  CUDA events around a graph of the one kernel, L2 flushed before each replay."""
+    w = I.DECODE_5S
+    H, d, bpf = w.heads, w.head_dim, w.blocks_per_frame
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    out = {}
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize(dev)
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.graph(graph, stream=side):
+            fn()
+        torch.cuda.current_stream(dev).wait_stream(side)
+        ts = []
+        for i in range(reps + 2):
+            flush.fill_(i & 255)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            graph.replay()
+            e1.record()
+            e1.synchronize()
+            if i >= 2:
+                ts.append(e0.elapsed_time(e1))
+        del graph
+        return statistics.median(ts)
+
+    # commit of K and V, 18 frames
+    g = P.make_geom(H, d, w.frame_h, w.frame_w, w.tile_h, w.tile_w, w.scale, w.dtype)
+    nf = 18
+    kx = torch.randn((nf * w.tokens_per_frame, H, d), device=dev).to(torch.bfloat16)
+    vx = torch.randn_like(kx)
+    slots = nf * bpf
+    k_pool = torch.empty((H, slots, 64, d), dtype=torch.bfloat16, device=dev)
+    v_pool = torch.empty_like(k_pool)
+    k_reps = torch.empty((H, slots, d), device=dev)
+    ws = torch.zeros(P.pbsa_workspace_bytes(g, 72, 168), dtype=torch.uint8, device=dev)
+    ms = timed(lambda: P.pbsa_blockify_kv(g, kx, vx, nf, k_reps, None, slots, None, k_pool, v_pool, slots, ws=ws))
+    nbytes = 2 * (2 * kx.numel() * 2) + k_reps.numel() * 4
+    out["commit_blockify_kv_18_frames"] = {"ms": ms, "algorithmic_bytes": nbytes,
+                                           "achieved_gbs": nbytes / (ms * 1e-3) / 1e9,
+                                           "frac_hbm": nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+    del kx, vx, k_pool, v_pool, k_reps
+
+    # the memory update's copies, 360 heads x 72 promotions
+    Hs, C, S, nc = 30 * H, w.capacity, bpf, 72
+    gs = P.make_geom(Hs, d, w.frame_h, w.frame_w, w.tile_h, w.tile_w, w.scale, w.dtype)
+    pool = C + nc
+    k_pool = torch.randn((Hs, pool, 64, d), device=dev).to(torch.bfloat16)
+    v_pool = torch.randn_like(k_pool)
+    k_reps = torch.randn((Hs, pool, d), device=dev) * 0.35
+    q_reps = torch.randn((Hs, 72, d), device=dev) * 0.3
+    slot_gid = torch.full((Hs, C), -1, dtype=torch.int32, device=dev)
+    slot_gid[:, :S] = torch.arange(S, dtype=torch.int32, device=dev)      # sinks only: every
+    slot_ema = torch.zeros((Hs, C), device=dev)                            # candidate is promoted
+    cs = (torch.arange(nc, dtype=torch.int32, device=dev) + C).repeat(Hs, 1).contiguous()
+    cg = (torch.arange(nc, dtype=torch.int32, device=dev) + 1000).repeat(Hs, 1).contiguous()
+    wss = torch.zeros(P.pbsa_workspace_bytes(gs, 72, C + nc), dtype=torch.uint8, device=dev)
+    P.pbsa_memory_update_plan(gs, q_reps, 72, k_reps, pool, slot_gid, slot_ema, C, S, cs, cg, nc, w.gamma, ws=wss)
+    torch.cuda.synchronize(dev)
+    promoted = int((slot_gid >= 1000).sum().item())
+    ms = timed(lambda: P.pbsa_memory_update_apply(gs, k_reps, k_pool, v_pool, pool, C, nc, ws=wss))
+    nbytes = promoted * 2 * (2 * 64 * d * 2 + d * 4)
+    out["memory_update_apply_360_heads"] = {"ms": ms, "promoted_blocks": promoted, "algorithmic_bytes": nbytes,
+                                            "achieved_gbs": nbytes / (ms * 1e-3) / 1e9,
+                                            "frac_hbm": nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+    _check_device(P, wss, "in the memory update at scale")
+    _check_device(P, ws, "in the commit at scale")
+    del k_pool, v_pool
+    return out
+
+
 def rank_workload(w, rank: int):
     """Weak scaling: every rank decodes its own independent layer (same shapes, its own seed)."""
     import dataclasses
@@ -582,6 +659,7 @@ def run_pbsa(args, w, rank, world, local_rank):
     }
     if not args.no_train:
         line["train"] = run_train(P, I, dev, 5, peaks)
+    line["kernels_at_scale"] = run_hbm_at_scale(P, I, dev, peaks)
     line["variants"] = [run_variant(P, I, dev, w, max(5, args.steps // 2), hsa_top_frames=3, hsa_recent=1),
                         run_variant(P, I, dev, w, max(5, args.steps // 2), own_chunk=True)]
     if not args.no_rollout:
