@@ -96,6 +96,33 @@ def test_blockify_kv_one_launch(w, n_frames, with_v_reps):
     assert torch.equal(k_reps1, k_reps)
 
 
+def test_blockify_kv_bad_slot_is_reported_and_skipped():
+    """A destination slot outside the pool is recorded in the workspace's error word (index error,
+    the bad slot) and that block is skipped; every other block is written as usual."""
+    w = I.DECODE_5S
+    g = geom_for(w)
+    k, v = I.tokens(w, 1, 31), I.tokens(w, 1, 32)
+    nb = w.blocks_per_frame
+    slots = nb + 2
+    dst = torch.arange(nb, dtype=torch.int32)
+    dst[5] = slots + 100                               # outside the pool
+    k_reps = torch.zeros((w.heads, slots, w.head_dim), device=DEV)
+    k_pool = torch.zeros((w.heads, slots, 64, w.head_dim), dtype=k.dtype, device=DEV)
+    v_pool = torch.zeros_like(k_pool)
+    ws = ws_for(g)
+    P.pbsa_blockify_kv(g, k.to(DEV), v.to(DEV), 1, k_reps, None, slots, dst.to(DEV), k_pool, v_pool, slots, ws=ws)
+    torch.cuda.synchronize()
+    word = ws[:16].view(torch.int32).tolist()
+    assert word[0] == 5 and word[1] == slots + 100
+    kp = k_pool.cpu()
+    for b in range(nb):
+        if b == 5:
+            continue
+        rows = O.block_token_rows(w.frame_h, w.frame_w, w.tile_h, w.tile_w, b)
+        assert torch.equal(kp[:, b], k[rows].permute(1, 0, 2))
+    assert not kp[:, 5].any() and not kp[:, nb:].any()   # nothing landed in unlisted slots
+
+
 # ----------------------------------------------------------------------------- score + select
 def _selection_case(seed, H=3, nq=9, pool=200, ncand=144, d=128, k=32, prefix=20, dup=False):
     gen = torch.Generator().manual_seed(seed)
