@@ -70,6 +70,7 @@ _SIGS = {
     "pbsa_memory_update_noalloc": (_I, [ctypes.POINTER(Geom), _P, _I, _P, _P, _P, _I, _P, _P, _I, _I,
                                         _P, _P, _I, ctypes.c_float, _P, _P, _P]),
     "pbsa_get_device_error": (_I, [_P, _P]),
+    "pbsa_selftest_wait_timeout": (_I, [_P, ctypes.c_uint, _P]),
     "pbsa_status_string": (ctypes.c_char_p, [_I]),
     "pbsa_bwd_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(Geom), _I, _I, _I]),
     "pbsa_attend_bwd": (_I, [ctypes.POINTER(Geom), _P, _I, _P, _P, _I, _P, _P, _I, _P, _P, _P,
@@ -265,6 +266,11 @@ def pbsa_attend_bwd(g: Geom, q, q_frames, k_pool, v_pool, pool_slots, kv_slot, k
         pool_slots, _ptr(kv_slot, torch.int32, "kv_slot"), _ptr(kv_cnt, torch.int32, "kv_cnt"), kv_ld,
         _ptr(o, dt, "o"), _ptr(d_o, dt, "d_o"), _ptr(lse, torch.float32, "lse"), _ptr(dq, dt, "dq"),
         _ptr(dk_pool, dt, "dk_pool"), _ptr(dv_pool, dt, "dv_pool"), _ptr(ws, None, "ws"), _stream(stream)))
+
+
+def pbsa_selftest_wait_timeout(ws, limit_us: int, stream=None):
+    _check("pbsa_selftest_wait_timeout", load().pbsa_selftest_wait_timeout(_ptr(ws, None, "ws"), int(limit_us),
+                                                                           _stream(stream)))
 
 
 def pbsa_get_device_error(ws, stream=None) -> int:

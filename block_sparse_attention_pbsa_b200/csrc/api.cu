@@ -52,6 +52,17 @@ bool pool_ok(const Geo& g, int pool_slots) {
   return pool_slots > 0 && (int64_t)g.H * pool_slots * BT < ((int64_t)1 << 31);
 }
 
+// The bounded-wait path every kernel relies on, on its own: one thread waits on an mbarrier
+// that nothing ever arrives on, gives up after limit_ns, records PBSA_ERR_TIMEOUT and returns.
+__global__ void selftest_wait_kernel(void* ws, unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+    if (!mbar_wait(&bar, 0, limit_ns)) record_error(ws, PBSA_ERR_TIMEOUT, 0, K_SELFTEST);
+  }
+}
+
 }  // namespace
 
 cudaError_t set_smem_once(const void* kernel, int bytes) {
@@ -304,6 +315,12 @@ pbsa_status pbsa_attend_bwd(const pbsa_geom* gin, const void* q, int q_frames, c
   if (nq > 512 || (int64_t)q_frames * g.tpf * g.H > ((int64_t)1 << 31)) return PBSA_ERR_UNSUPPORTED;
   return from_cuda(launch_attend_bwd(g, q, q_frames, k_pool, v_pool, pool_slots, kv_slot, kv_cnt, kv_ld,
                                      o, d_o, lse, dq, dk_pool, dv_pool, ws, static_cast<cudaStream_t>(stream)));
+}
+
+pbsa_status pbsa_selftest_wait_timeout(void* ws, unsigned int limit_us, void* stream) {
+  if (ws == nullptr || limit_us == 0 || limit_us > 1000000) return PBSA_ERR_INVALID_ARG;
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(ws, (unsigned long long)limit_us * 1000ull);
+  return from_cuda(cudaGetLastError());
 }
 
 pbsa_status pbsa_get_device_error(void* ws, void* stream) {

@@ -23,7 +23,8 @@ struct Geo {
 
 // Kernel ids recorded with device errors.
 enum KernelId { K_BLOCKIFY = 1, K_SCORE = 2, K_ATTEND_F32 = 3, K_ATTEND_TC = 4, K_MU_SCORE = 5,
-                K_MU_SELECT = 6, K_MU_COPY = 7, K_BWD_PREP = 8, K_BWD_KV = 9, K_BWD_Q = 10 };
+                K_MU_SELECT = 6, K_MU_COPY = 7, K_BWD_PREP = 8, K_BWD_KV = 9, K_BWD_Q = 10,
+                K_SELFTEST = 11 };
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bound of every in-kernel wait
 

@@ -298,6 +298,14 @@ PBSA_API pbsa_status pbsa_memory_update_noalloc(const pbsa_geom* g, const float*
 
 /* Synchronises `stream`, reads and clears the workspace's device error word, and returns
  * it (PBSA_OK when clean). */
+/* Self-test of the bounded waits (the paper has no counterpart).  Every kernel that waits on an
+ * mbarrier gives up after a time limit, records PBSA_ERR_TIMEOUT in the workspace's error word
+ * and returns instead of hanging.  This launches one thread that waits, with that same code, on
+ * an mbarrier nothing ever arrives on, for limit_us microseconds (1 .. 1000000): afterwards
+ * pbsa_get_device_error(ws) reports PBSA_ERR_TIMEOUT and the context remains usable.
+ *  ws: a workspace whose first 256 bytes are the error word. */
+PBSA_API pbsa_status pbsa_selftest_wait_timeout(void* ws, unsigned int limit_us, void* stream);
+
 PBSA_API pbsa_status pbsa_get_device_error(void* ws, void* stream);
 
 /* Static description of a status code. */

@@ -205,6 +205,32 @@ def _rollout(w, n_chunks, sample_every=3, k_schedule=None):
     return alive
 
 
+def test_decode_step_is_deterministic():
+    """The 5 s chunk decode (fused selection, attention, overlapped memory-update plan and commit,
+    copies) run twice from the same state gives bit-identical lists, O and cache."""
+    w = I.DECODE_5S
+    q, k, v = I.single_step(w)
+    kc = I.tokens(w, w.chunk_frames, I.stream_seed(w.seed, 4))
+    vc = I.tokens(w, w.chunk_frames, I.stream_seed(w.seed, 5))
+    bpf = w.blocks_per_frame
+    cache = P.PBSALayerCache(layer_cfg(w, (w.hist_frames - w.window_frames) * bpf))
+    qd, kcd, vcd = q.to(DEV), kc.to(DEV), vc.to(DEV)
+    cache.prefill(k.to(DEV), v.to(DEV), w.hist_frames, cache.query_reps(qd))
+    step = P.ChunkDecodeStep(cache)
+    snap = step.snapshot()
+    runs = []
+    for _ in range(2):
+        step.restore(snap)
+        o = torch.empty_like(qd)
+        step.run(qd, kcd, vcd, o)
+        torch.cuda.synchronize()
+        runs.append([o.clone(), step.kv_slot.clone(), step.kv_cnt.clone()] +
+                    [getattr(cache, n).clone() for n in ("slot_gid", "slot_ema", "k_pool", "v_pool", "k_reps")])
+    for a, b in zip(*runs):
+        assert torch.equal(a, b)
+    assert P.pbsa_get_device_error(cache.ws) == 0
+
+
 def test_rollout_overlapped_commit_matches_serial():
     """Each chunk committed right after its last-step attention with the overlap (the write of
     the chunk and the memory update's plan as programmatic dependents of attend) gives the same

@@ -123,6 +123,26 @@ def test_blockify_kv_bad_slot_is_reported_and_skipped():
     assert not kp[:, 5].any() and not kp[:, nb:].any()   # nothing landed in unlisted slots
 
 
+def test_bounded_wait_expires_is_reported_and_the_context_stays_usable():
+    """The bounded mbarrier wait every kernel uses gives up after its limit: a wait on a barrier
+    nothing arrives on (20 ms limit) returns, the error word reads PBSA_ERR_TIMEOUT, and the
+    next kernel on the same context runs correctly."""
+    import time
+    w = I.TINY
+    g = geom_for(w)
+    ws = ws_for(g)
+    t0 = time.perf_counter()
+    P.pbsa_selftest_wait_timeout(ws, 20000)
+    assert P.pbsa_get_device_error(ws) == 4            # PBSA_ERR_TIMEOUT (and the word is cleared)
+    assert time.perf_counter() - t0 >= 0.019
+    assert P.pbsa_get_device_error(ws) == 0
+    x = I.tokens(w, 1, 41)
+    reps = torch.zeros((w.heads, w.blocks_per_frame, w.head_dim), device=DEV)
+    P.pbsa_blockify(g, x.to(DEV), 1, reps, w.blocks_per_frame, None, None, 0, ws)
+    check_no_device_error(ws)
+    np.testing.assert_allclose(f64(reps), O.block_reps(f64(x), geom_dict(w), 1), rtol=0, atol=2e-6)
+
+
 # ----------------------------------------------------------------------------- score + select
 def _selection_case(seed, H=3, nq=9, pool=200, ncand=144, d=128, k=32, prefix=20, dup=False):
     gen = torch.Generator().manual_seed(seed)
