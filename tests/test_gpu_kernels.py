@@ -200,7 +200,9 @@ def test_score_select(ncand, k, dup):
 @pytest.mark.parametrize("wname,ncand,k,dup", [("decode", 144, 32, False), ("decode", 48, 32, False),
                                                ("decode", 300, 16, False), ("decode", 144, 32, True),
                                                ("decode", 0, 8, False), ("tiny", 8, 4, False),
-                                               ("tile4x16", 20, 32, False)])
+                                               ("tile4x16", 20, 32, False),
+                                               # either side of the 8-block kernel's 256-candidate limit
+                                               ("decode", 256, 32, False), ("decode", 257, 32, False)])
 def test_blockify_score_select(wname, ncand, k, dup):
     """pbsa_blockify_score_select: q reps = the oracle's block means (and bit-identical to
     pbsa_blockify), selection = the oracle's top-k of its own coarse scores outside near ties."""
@@ -438,12 +440,16 @@ def test_invalid_arguments_are_rejected_on_host():
 
 # ----------------------------------------------------------------------------- memory update
 @pytest.mark.parametrize("split", [False, True])
-@pytest.mark.parametrize("n_pers,ncand,C", [(70, 72, 96), (24, 48, 96), (96, 72, 96), (0, 264, 96), (3, 5, 8)])
-def test_memory_update(n_pers, ncand, C, split):
+@pytest.mark.parametrize("n_pers,ncand,C,nq", [(70, 72, 96, 72), (24, 48, 96, 72), (96, 72, 96, 72), (0, 264, 96, 72),
+                                               (3, 5, 8, 72),
+                                               # either side of the one-launch limits: 256 pool entries, 128 query blocks
+                                               (96, 160, 96, 72), (96, 161, 96, 72), (70, 72, 96, 128),
+                                               (70, 72, 96, 129)])
+def test_memory_update(n_pers, ncand, C, nq, split):
     """pbsa_memory_update, or (split) pbsa_memory_update_plan + pbsa_memory_update_apply --
     one CTA per head for pools of up to 256 entries, the two-launch score kernel above -- against
     the oracle: kept sets (outside EMA near-ties), EMA values, promoted copies, persistent list."""
-    H, d, nq, S = 3, 128, 72, min(24, C // 2)
+    H, d, S = 3, 128, min(24, C // 2)
     w = dataclasses.replace(I.DECODE_5S, heads=H)
     g = geom_for(w)
     gen = torch.Generator().manual_seed(n_pers * 1000 + ncand)
