@@ -410,6 +410,33 @@ def test_attend_bf16(fh, fw, q_frames, shared, local, empty):
                 assert np.isneginf(f64(lse[h, rows])).all()
 
 
+def test_attend_bf16_running_max_grows():
+    """Key magnitudes grow geometrically along every (sorted) list, so each row's running
+    maximum jumps by more than 2^8 at many steps of both softmax streams and both S buffers:
+    the path that rescales the O accumulator, against the oracle."""
+    w = dataclasses.replace(I.DECODE_5S, heads=2, frame_h=16, frame_w=16)
+    q_frames, slots = 2, 48
+    nq = q_frames * w.blocks_per_frame
+    rng = np.random.default_rng(7)
+    lists = [[sorted(rng.choice(slots, size=int(rng.integers(9, 41)), replace=False).tolist()) for _ in range(nq)]
+             for _ in range(w.heads)]
+    q, kp, vp, kv, cnt, ld = _attend_case(w, q_frames, slots, lists, 11)
+    kp = (kp.float() * (1.12 ** torch.arange(slots, dtype=torch.float32)).view(1, slots, 1, 1)).to(kp.dtype)
+    o, lse = _run_attend(w, q, q_frames, kp, vp, kv, cnt, ld)
+    jumps = 0
+    for h in range(w.heads):
+        for r in range(nq):
+            rows, (want, wlse) = _oracle_unit(w, q, kp, vp, h, r, lists[h][r])
+            assert_bf16_close(f64(o[rows, h]), want, f"h{h} r{r}")
+            np.testing.assert_allclose(f64(lse[h, rows]), wlse, rtol=1e-5, atol=2e-3)
+            # how often the running maximum (log2 units) grew by more than 8 along the list
+            lg = w.scale / np.log(2.0) * f64(q[rows, h]) @ f64(kp[h][lists[h][r]]).reshape(-1, w.head_dim).T
+            bm = lg.reshape(len(rows), len(lists[h][r]), 64).max(axis=2)
+            run = np.maximum.accumulate(bm, axis=1)
+            jumps += int((bm[:, 1:] > run[:, :-1] + 8).sum())
+    assert jumps > 100
+
+
 def test_attend_bf16_bad_slot_is_reported():
     w = dataclasses.replace(I.DECODE_5S, heads=1, frame_h=8, frame_w=16)
     lists = [[[0, 1, 999], [2, 3]]]
