@@ -437,6 +437,29 @@ def test_attend_bf16_running_max_grows():
     assert jumps > 100
 
 
+@pytest.mark.parametrize("case", ["pool_above_bitmap", "merged_list_at_capacity"])
+def test_attend_bf16_list_merge_limits(case):
+    """The pair's list merge at its limits: a pool of more slots than the membership bitmaps
+    cover (the quadratic merge, slots above 8192 in the lists), and two disjoint lists of the
+    maximum length 512 (a merged list of 1024 entries)."""
+    w = dataclasses.replace(I.DECODE_5S, heads=1, frame_h=8, frame_w=16)   # 2 query blocks
+    rng = np.random.default_rng(3)
+    if case == "pool_above_bitmap":
+        slots = 8300
+        shared = rng.choice(np.arange(8100, slots), size=12, replace=False).tolist()
+        lists = [[shared + rng.choice(slots, size=n, replace=False).tolist() for n in (20, 9)]]
+    else:
+        slots = 1024
+        perm = rng.permutation(slots).tolist()
+        lists = [[perm[:512], perm[512:]]]
+    q, kp, vp, kv, cnt, ld = _attend_case(w, 1, slots, lists, 17)
+    o, lse = _run_attend(w, q, 1, kp, vp, kv, cnt, ld)
+    for r in range(2):
+        rows, (want, wlse) = _oracle_unit(w, q, kp, vp, 0, r, lists[0][r])
+        assert_bf16_close(f64(o[rows, 0]), want, f"r{r}")
+        np.testing.assert_allclose(f64(lse[0, rows]), wlse, rtol=0, atol=2e-3)
+
+
 def test_attend_bf16_bad_slot_is_reported():
     w = dataclasses.replace(I.DECODE_5S, heads=1, frame_h=8, frame_w=16)
     lists = [[[0, 1, 999], [2, 3]]]
