@@ -496,6 +496,10 @@ def test_invalid_arguments_are_rejected_on_host():
                                                (96, 160, 96, 72), (96, 161, 96, 72), (70, 72, 96, 128),
                                                (70, 72, 96, 129)])
 def test_memory_update(n_pers, ncand, C, nq, split):
+    _check_memory_update(n_pers, ncand, C, nq, split)
+
+
+def _check_memory_update(n_pers, ncand, C, nq, split, gamma=0.9):
     """pbsa_memory_update, or (split) pbsa_memory_update_plan + pbsa_memory_update_apply --
     one CTA per head for pools of up to 256 entries, the two-launch score kernel above -- against
     the oracle: kept sets (outside EMA near-ties), EMA values, promoted copies, persistent list."""
@@ -524,17 +528,18 @@ def test_memory_update(n_pers, ncand, C, nq, split):
         if n_pers == 0 and ncand >= S:
             cg[h, :S] = torch.arange(S, dtype=torch.int32)   # sinks arriving as candidates
     kr_d, kp_d, vp_d = kr.to(DEV), kp.to(DEV), vp.to(DEV)
+    cs_d, cg_d = (cs.to(DEV), cg.to(DEV)) if ncand else (None, None)
     sgid_d, sema_d = sgid.to(DEV), sema.to(DEV)
     plist = torch.full((H, C), -5, dtype=torch.int32, device=DEV)
     pcnt = torch.zeros((H,), dtype=torch.int32, device=DEV)
     ws = torch.zeros(P.pbsa_workspace_bytes(g, nq, C + ncand), dtype=torch.uint8, device=DEV)
     if split:
-        P.pbsa_memory_update_plan(g, qr.to(DEV), nq, kr_d, pool, sgid_d, sema_d, C, S, cs.to(DEV), cg.to(DEV), ncand,
-                                  0.9, plist, pcnt, ws=ws)
+        P.pbsa_memory_update_plan(g, qr.to(DEV), nq, kr_d, pool, sgid_d, sema_d, C, S, cs_d, cg_d, ncand,
+                                  gamma, plist, pcnt, ws=ws)
         P.pbsa_memory_update_apply(g, kr_d, kp_d, vp_d, pool, C, ncand, ws=ws)
     else:
-        P.pbsa_memory_update(g, qr.to(DEV), nq, kr_d, kp_d, vp_d, pool, sgid_d, sema_d, C, S, cs.to(DEV),
-                             cg.to(DEV), ncand, 0.9, plist, pcnt, ws)
+        P.pbsa_memory_update(g, qr.to(DEV), nq, kr_d, kp_d, vp_d, pool, sgid_d, sema_d, C, S, cs_d,
+                             cg_d, ncand, gamma, plist, pcnt, ws)
     check_no_device_error(ws)
     new_gid, new_ema = sgid_d.cpu(), sema_d.cpu()
     for h in range(H):
@@ -542,7 +547,7 @@ def test_memory_update(n_pers, ncand, C, nq, split):
         ent += [(int(cs[h, i]), int(cg[h, i]), np.nan) for i in range(ncand)]
         slots_, gids_, prev = zip(*ent)
         sink = [gg < S for gg in gids_]
-        ema, keep, a = O.memory_update(f64(qr[h]), f64(kr[h][list(slots_)]), gids_, prev, sink, w.scale, 0.9, C)
+        ema, keep, a = O.memory_update(f64(qr[h]), f64(kr[h][list(slots_)]), gids_, prev, sink, w.scale, gamma, C)
         want = {gg for gg, kp_ in zip(gids_, keep) if kp_}
         got = {int(x) for x in new_gid[h] if x >= 0}
         assert len(got) <= C and {gg for gg in gids_ if gg < S} <= got
@@ -562,3 +567,65 @@ def test_memory_update(n_pers, ncand, C, nq, split):
                 assert torch.equal(kr_d[h, s].cpu(), kr[h, src])
         valid = [s for s in range(C) if new_gid[h, s] >= 0]
         assert int(pcnt[h]) == len(valid) and plist[h, :len(valid)].cpu().tolist() == valid
+
+
+@pytest.mark.parametrize("split", [False, True])
+@pytest.mark.parametrize("n_pers,ncand,C,gamma", [
+    (70, 72, 96, 0.0),     # the EMA is the chunk's attention alone
+    (70, 72, 96, 1.0),     # the EMA of a block seen before never moves
+    (20, 30, 96, 0.9),     # capacity above the entries: everything is kept, no eviction
+    (70, 0, 96, 0.9),      # no candidates: re-scoring and EMA only
+])
+def test_memory_update_degenerate(n_pers, ncand, C, gamma, split):
+    """The update at its degenerate points, against the oracle (same checks as above)."""
+    _check_memory_update(n_pers, ncand, C, 72, split, gamma)
+
+
+@pytest.mark.parametrize("split", [False, True])
+def test_memory_update_bad_candidate_slot_is_reported_and_dropped(split):
+    """A candidate whose slot lies outside the staging range is reported (PBSA_ERR_DEVICE_INDEX)
+    and left out of the softmax and the ranking: the result is the oracle's over the others."""
+    H, d, nq, C, S, ncand = 1, 128, 24, 16, 4, 12
+    w = dataclasses.replace(I.DECODE_5S, heads=H)
+    g = geom_for(w)
+    gen = torch.Generator().manual_seed(99)
+    pool = C + ncand + 4
+    qr = torch.randn((H, nq, d), generator=gen) * 0.3
+    kr = torch.randn((H, pool, d), generator=gen) * 0.35
+    kp = torch.randn((H, pool, 64, d), generator=gen).to(torch.bfloat16)
+    vp = torch.randn((H, pool, 64, d), generator=gen).to(torch.bfloat16)
+    sgid = torch.full((H, C), -1, dtype=torch.int32)
+    sema = torch.zeros((H, C))
+    for s_ in range(10):                       # 4 sinks + 6 earlier blocks
+        sgid[0, s_] = s_ if s_ < S else 100 + s_
+        sema[0, s_] = 0.01 * (s_ % 3)
+    cs = (torch.arange(ncand, dtype=torch.int32) + C).view(H, ncand).clone()
+    cg = (torch.arange(ncand, dtype=torch.int32) + 500).view(H, ncand).clone()
+    cs[0, 3] = pool + 7                        # out of range
+    kr_d, kp_d, vp_d, sgid_d, sema_d = (t.to(DEV) for t in (kr, kp, vp, sgid, sema))
+    plist = torch.full((H, C), -5, dtype=torch.int32, device=DEV)
+    pcnt = torch.zeros((H,), dtype=torch.int32, device=DEV)
+    ws = torch.zeros(P.pbsa_workspace_bytes(g, nq, C + ncand), dtype=torch.uint8, device=DEV)
+    if split:
+        P.pbsa_memory_update_plan(g, qr.to(DEV), nq, kr_d, pool, sgid_d, sema_d, C, S, cs.to(DEV), cg.to(DEV),
+                                  ncand, 0.9, plist, pcnt, ws=ws)
+        P.pbsa_memory_update_apply(g, kr_d, kp_d, vp_d, pool, C, ncand, ws=ws)
+    else:
+        P.pbsa_memory_update(g, qr.to(DEV), nq, kr_d, kp_d, vp_d, pool, sgid_d, sema_d, C, S, cs.to(DEV),
+                             cg.to(DEV), ncand, 0.9, plist, pcnt, ws)
+    assert P.pbsa_get_device_error(ws) == 5
+    ent = [(s_, int(sgid[0, s_]), float(sema[0, s_])) for s_ in range(C) if sgid[0, s_] >= 0]
+    ent += [(int(cs[0, i]), int(cg[0, i]), np.nan) for i in range(ncand) if i != 3]
+    slots_, gids_, prev = zip(*ent)
+    sink = [gg < S for gg in gids_]
+    ema, keep, _ = O.memory_update(f64(qr[0]), f64(kr[0][list(slots_)]), gids_, prev, sink, w.scale, 0.9, C)
+    got = {int(x) for x in sgid_d.cpu()[0] if x >= 0}
+    assert int(cg[0, 3]) not in got
+    if O.ema_boundary_gap(ema, gids_, sink, C) > EMA_NEAR_TIE_REL:
+        assert got == {gg for gg, k_ in zip(gids_, keep) if k_}
+    ema_of = dict(zip(gids_, ema))
+    new_ema = sema_d.cpu()
+    for s_ in range(C):
+        gg = int(sgid_d[0, s_])
+        if gg >= 0:
+            np.testing.assert_allclose(float(new_ema[0, s_]), ema_of[gg], rtol=2e-5, atol=1e-9)
