@@ -361,6 +361,10 @@ class ChunkDecodeStep:
 
     def __init__(self, cache: PBSALayerCache, q_frames: int | None = None, fused_select: bool = True):
         c = cache.cfg
+        if cache.hist == 0:
+            # the first chunk attends its own blocks, and frame 0's blocks are candidates of its
+            # update, which must then follow their commit: decode_step + commit cover that case
+            raise ValueError("a chunk decode step needs a history: use decode_step for the first chunk")
         self.cache = cache
         self.fused_select = fused_select
         # kernels per run(): [blockify(Q) + select] (1 fused or 2) + attend + commit of K and V (1)
@@ -479,13 +483,15 @@ class ChunkDecodeStep:
         return graph
 
     def capture_pipeline(self, q, k, v, o, lse=None):
-        """Capture the step as two graphs for ``run_pipelined``: [blockify(Q) + selection +
-        attend] and [commit blockify(K, V) + memory update] (the own-chunk variant, which needs
-        K, V before the selection, is not split)."""
+        """Capture the step as three graphs for ``run_pipelined``: [blockify(Q) + selection +
+        attend], [memory update] and [commit blockify(K, V)].  The update reads neither K nor V
+        of the chunk (its candidates are blocks leaving the window, never the chunk's ring
+        positions), so it runs while they upload; only the commit waits for them.  (The
+        own-chunk variant, which needs K, V before the selection, is not split.)"""
         if self.cache.cfg.own_chunk:
             raise ValueError("the own-chunk variant writes K, V before the selection: use capture()")
         dev = self.cache.device
-        front, back = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        front, mid, back = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
         side = torch.cuda.Stream(device=dev)
         side.wait_stream(torch.cuda.current_stream(dev))
         ca, c = self.cache, self.cache.cfg
@@ -494,22 +500,23 @@ class ChunkDecodeStep:
             ca._select_fused(q, self.q_frames, self.q_reps, self.kv_slot, self.kv_cnt, ca.kv_ld)
             L.pbsa_attend(g, q, self.q_frames, ca.k_pool, ca.v_pool, ps, self.kv_slot, self.kv_cnt, ca.kv_ld,
                           o, lse, ws=ws)
+        with torch.cuda.graph(mid, stream=side):   # the kernels of run(): the same results, bit for bit
+            L.pbsa_memory_update_plan(g, self.q_reps, self.nq, ca.k_reps, ps, ca.slot_gid, ca.slot_ema, c.capacity,
+                                      c.bpf, self.cs, self.cg, self.ncand, c.gamma, ca.p_list, ca.p_cnt, ws=ws)
+            L.pbsa_memory_update_apply(g, ca.k_reps, ca.k_pool, ca.v_pool, ps, c.capacity, self.ncand, ws=ws)
         with torch.cuda.graph(back, stream=side):
             L.pbsa_blockify_kv(g, k, v, self.q_frames, ca.k_reps, None, ps, self.dst, ca.k_pool, ca.v_pool, ps,
                                ws=ws)
-            L.pbsa_memory_update(g, self.q_reps, self.nq, ca.k_reps, ca.k_pool, ca.v_pool, ps, ca.slot_gid,
-                                 ca.slot_ema, c.capacity, c.bpf, self.cs, self.cg, self.ncand, c.gamma,
-                                 ca.p_list, ca.p_cnt, ws=ws)
         torch.cuda.current_stream(dev).wait_stream(side)
-        self._pipe = {"front": front, "back": back, "bufs": (q, k, v, o),
+        self._pipe = {"front": front, "mid": mid, "back": back, "bufs": (q, k, v, o),
                       "h2d": torch.cuda.Stream(device=dev), "d2h": torch.cuda.Stream(device=dev)}
 
     def run_pipelined(self, qh, kh, vh, oh):
         """One step from pinned host buffers to a pinned host result, with the transfers
         overlapped: Q is uploaded first and the front graph (selection + attention) starts as
-        soon as it lands, while K and V upload on a copy stream (only the commit needs them);
-        O downloads on another stream while the commit and memory update run.  All work is
-        ordered on the current stream's timeline when this returns (asynchronously)."""
+        soon as it lands, while K and V upload on a copy stream; O downloads on another stream
+        while the memory update runs, and the commit of K and V follows their upload.  All
+        work is ordered on the current stream's timeline when this returns (asynchronously)."""
         p = self._pipe
         q, k, v, o = p["bufs"]
         main = torch.cuda.current_stream(self.cache.device)
@@ -529,6 +536,7 @@ class ChunkDecodeStep:
         with torch.cuda.stream(d2h):
             d2h.wait_event(front_done)
             oh.copy_(o, non_blocking=True)
+        p["mid"].replay()                           # memory update (needs no K, V)
         main.wait_stream(h2d)                       # K, V uploaded
         p["back"].replay()
         main.wait_stream(d2h)                       # O downloaded

@@ -278,9 +278,18 @@ def test_rollout_1min_layer0_first_chunks():
     _rollout(w, n_chunks=13, sample_every=4)
 
 
+def test_chunk_decode_step_needs_a_history():
+    """The first chunk attends its own blocks (decode_step + commit); a step object refuses it."""
+    w = I.ROLLOUT_5S
+    cache = P.PBSALayerCache(layer_cfg(w))
+    with pytest.raises(ValueError):
+        P.ChunkDecodeStep(cache)
+
+
 def test_pipelined_host_step_matches_the_graph_step():
-    """ChunkDecodeStep.run_pipelined (transfers overlapped with the kernels) gives the same O and
-    the same persistent memory as the single-graph step on the same inputs."""
+    """ChunkDecodeStep.run_pipelined (transfers overlapped with the kernels, the memory update
+    ahead of the commit of K and V) gives the same O and the same cache, bit for bit, as the
+    single-graph step on the same inputs."""
     w = I.DECODE_5S
     q, k, v = I.single_step(w)
     kc = I.tokens(w, w.chunk_frames, I.stream_seed(w.seed, 4))
@@ -294,7 +303,8 @@ def test_pipelined_host_step_matches_the_graph_step():
     o = torch.empty_like(qd)
     step.run(qd, kcd, vcd, o)
     want_o = o.cpu()
-    want_gid = cache.slot_gid.cpu()
+    names = ("slot_gid", "slot_ema", "k_pool", "v_pool", "k_reps", "p_list", "p_cnt")
+    want = [getattr(cache, n).cpu() for n in names]
     step.restore(snap)
     qb, kb, vb, ob = (torch.empty_like(t) for t in (qd, kcd, vcd, o))
     step.capture_pipeline(qb, kb, vb, ob)
@@ -305,5 +315,6 @@ def test_pipelined_host_step_matches_the_graph_step():
         step.run_pipelined(qh, kh, vh, oh)
         torch.cuda.synchronize()
         assert torch.equal(oh, want_o)
-        assert torch.equal(cache.slot_gid.cpu(), want_gid)
+        for n, t in zip(names, want):
+            assert torch.equal(getattr(cache, n).cpu(), t), n
     assert P.pbsa_get_device_error(cache.ws) == 0
