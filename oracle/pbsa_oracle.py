@@ -29,8 +29,11 @@ reading, not a quotation):
 Parity pins (tests/test_oracle.py): closed-form block means, brute-force and
 permutation checks of the selection, reduction of the attention to dense
 softmax attention (a library routine) when every block is selected, softmax
-row sums, closed-form memory-update values, invariants of the persistent set,
-and central finite differences for the backward pass.
+row sums, closed-form memory-update values (with scale 1 and with the scale
+1/sqrt(d)), invariants of the persistent set, the EMA carried between a
+rollout's updates, and central finite differences for the backward pass.
+tests/test_oracle_mutants.py plants one plausible mistake at a time in a copy of
+this module and checks that some pin fails for each.
 """
 from __future__ import annotations
 

@@ -162,6 +162,19 @@ def test_memory_update_closed_form():
     assert keep.tolist() == fx["expected_keep"]
 
 
+def test_memory_update_closed_form_with_the_attention_scale():
+    """d = 4: the scale 1/2 enters the softmax (the d = 1 fixture above cannot see it)."""
+    fx = json.load(open(os.path.join(GOLDEN, "memory_update_closed_form_scaled.json")))
+    d = len(fx["q_reps"][0])
+    assert fx["scale"] == 1.0 / math.sqrt(d)
+    prev = [np.nan if p is None else p for p in fx["prev_ema"]]
+    ema, keep, a = O.memory_update(np.array(fx["q_reps"]), np.array(fx["pool_reps"]), fx["pool_gids"],
+                                   prev, fx["is_sink"], fx["scale"], fx["gamma"], fx["capacity"])
+    np.testing.assert_allclose(a, fx["expected_a"], atol=1e-15)
+    np.testing.assert_allclose(ema, fx["expected_ema"], atol=1e-15)
+    assert keep.tolist() == fx["expected_keep"]
+
+
 def test_memory_update_invariants():
     rng = np.random.default_rng(4)
     for trial in range(30):
@@ -218,6 +231,28 @@ def test_rollout_windows_and_capacity_5s():
     assert local_sizes == [0, 48, 120, 144, 144, 144, 144]
     assert evicted == [[], [], [1, 2], [3, 4, 5], [6, 7, 8], [9, 10, 11], [12, 13, 14]]
     assert p_sizes[:3] == [24, 24, 72] and all(p == 96 for p in p_sizes[3:])
+
+
+def test_rollout_carries_the_ema_between_updates():
+    """A block kept by two consecutive updates ends with EMA gamma * (its EMA before) + (1 - gamma)
+    * a, a its attention share in the second update (that update's value with no history)."""
+    g = geom(32, 48, 8, 8, d=4)
+    ro = O.RolloutOracle(g, heads=1, capacity=96, window=6, topk=32, gamma=0.9)
+    rng = np.random.default_rng(9)
+    for c in range(4):
+        ro.commit(3 * c, 3, rng.standard_normal((1, 72, 4)), rng.standard_normal((1, 72, 4)))
+    before = dict(ro.P[0])
+    q = rng.standard_normal((1, 72, 4))
+    evicted = ro.commit(12, 3, rng.standard_normal((1, 72, 4)), q)
+    pool = sorted(before) + evicted
+    reps = np.stack([ro.kreps[gg][0] for gg in pool])
+    _, _, a = O.memory_update(q[0], reps, pool, [np.nan] * len(pool), [gg < 24 for gg in pool],
+                              g["scale"], 0.9, 96)
+    carried = [gg for gg in before if gg in ro.P[0]]
+    assert len(carried) >= 24
+    for gg in carried:
+        want = 0.9 * before[gg] + 0.1 * a[pool.index(gg)]
+        assert abs(ro.P[0][gg] - want) <= 1e-12 * max(1.0, abs(want))
 
 
 def test_single_step_partition_5s():
