@@ -31,7 +31,9 @@ permutation checks of the selection, reduction of the attention to dense
 softmax attention (a library routine) when every block is selected, softmax
 row sums, closed-form memory-update values (with scale 1 and with the scale
 1/sqrt(d)), invariants of the persistent set, the EMA carried between a
-rollout's updates, and central finite differences for the backward pass.
+rollout's updates, central finite differences for the backward pass, a hand-built
+trainable-path case whose top-k is known by construction, and hand values of the two
+near-tie gaps (``kth_gap``, ``ema_boundary_gap``).
 tests/test_oracle_mutants.py plants one plausible mistake at a time in a copy of
 this module and checks that some pin fails for each.
 """

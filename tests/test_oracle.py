@@ -282,6 +282,89 @@ def test_train_masks_shape():
     assert set(m[30][4:6]) <= set(range(4, 24))
 
 
+def _const_block_tokens(reps, fh, fw, th, tw, n_frames):
+    """Raster tokens [n_frames*fh*fw, H, d] in which every token of block b equals reps[:, b]
+    (so each block's mean is exactly reps[:, b]); block of token (f, y, x) = f*bpf +
+    (y // th)*(fw // tw) + x // tw, written out here independently of the oracle."""
+    H, _, d = reps.shape
+    x = np.zeros((n_frames * fh * fw, H, d))
+    bpf = (fh // th) * (fw // tw)
+    for f in range(n_frames):
+        for y in range(fh):
+            for xx in range(fw):
+                x[f * fh * fw + y * fw + xx] = reps[:, f * bpf + (y // th) * (fw // tw) + xx // tw]
+    return x
+
+
+def test_train_masks_selection_hand_built():
+    """Trainable-path masks on a case whose top-2 is known by construction (4 blocks per frame,
+    9 frames, 3-frame chunks, batch 2).  Every block's tokens are one constant vector, so the
+    representatives are exact.  Query block r scores with e_(r mod 2) * 2 (even rows rank the
+    keys by their first coordinate a, odd rows by their second b; scale 1/2 undoes the 2).
+    Batch 0: a = 100 on the sinks, 50 on chunk 1's blocks 12..23, 200 on chunk 2's blocks
+    24..35 (each would win if sinks, the own chunk or a later chunk were candidates), and
+    a[4..11] = 1, 7, 3, 7, -2, 5, 0, 7 (a three-way tie at 7 on blocks 5, 7, 11);
+    b = 100 on the sinks, 300 on chunk 2, b[4] = 9, b[8] = 8, b[20] = 10, else 0.
+    Batch 1 swaps a and b (its even rows see batch 0's odd-row ranking)."""
+    fh, fw, th, tw, d, F, cf, bpf = 16, 16, 8, 8, 4, 9, 3, 4
+    g = {"frame_h": fh, "frame_w": fw, "tile_h": th, "tile_w": tw, "scale": 0.5}
+    a = np.zeros(36)
+    a[0:4], a[12:24], a[24:36] = 100, 50, 200
+    a[4:12] = [1, 7, 3, 7, -2, 5, 0, 7]
+    b = np.zeros(36)
+    b[0:4], b[24:36] = 100, 300
+    b[4], b[8], b[20] = 9, 8, 10
+    kreps = np.zeros((2, 1, 36, d))
+    kreps[0, 0, :, 0], kreps[0, 0, :, 1] = a, b
+    kreps[1, 0, :, 0], kreps[1, 0, :, 1] = b, a
+    qreps = np.zeros((2, 1, 36, d))
+    for r in range(36):
+        qreps[:, 0, r, r % 2] = 2.0
+    q = np.stack([_const_block_tokens(qreps[i], fh, fw, th, tw, F) for i in range(2)])
+    k = np.stack([_const_block_tokens(kreps[i], fh, fw, th, tw, F) for i in range(2)])
+    masks, gaps = O.train_masks(q, k, g, F, cf, topk=2)
+    sinks = [0, 1, 2, 3]
+    own = {c: list(range(12 * c, 12 * c + 12)) for c in range(3)}
+    # chosen local blocks by (batch, chunk, row parity), worked out from the tables above
+    want = {(0, 1, 0): [5, 7], (0, 1, 1): [4, 8], (0, 2, 0): [12, 13], (0, 2, 1): [20, 4],
+            (1, 1, 0): [4, 8], (1, 1, 1): [5, 7], (1, 2, 0): [20, 4], (1, 2, 1): [12, 13]}
+    # |2nd best - 3rd best|: 7 - 7; 8 - 0; 50 - 50; 9 - 8
+    want_gap = {(0, 1, 0): 0.0, (0, 1, 1): 8.0, (0, 2, 0): 0.0, (0, 2, 1): 1.0,
+                (1, 1, 0): 8.0, (1, 1, 1): 0.0, (1, 2, 0): 1.0, (1, 2, 1): 0.0}
+    for bb in range(2):
+        for r in range(36):
+            c = r // 12
+            m = masks[bb][0][r]
+            if c == 0:
+                assert m == own[0] and gaps[bb][0][r] == float("inf")
+                continue
+            key = (bb, c, r % 2)
+            assert m[:4] == sinks and m[-12:] == own[c]
+            assert sorted(m[4:-12]) == sorted(want[key]), (bb, r, m)
+            assert gaps[bb][0][r] == pytest.approx(want_gap[key]), (bb, r)
+
+
+def test_kth_gap_hand_values():
+    """Scores 3, 1, 2.5, 2.5, -1 (gids 10..14) in ranking order: 3 | 2.5 (gid 12) | 2.5 (gid 13)
+    | 1 | -1.  The gap at k is |k-th - (k+1)-th|; none when k is 0 or takes every candidate."""
+    sc = np.array([3.0, 1.0, 2.5, 2.5, -1.0], np.float32)
+    gids = [10, 11, 12, 13, 14]
+    assert [O.kth_gap(sc, gids, k) for k in range(6)] == [float("inf"), 0.5, 0.0, 1.5, 2.0, float("inf")]
+
+
+def test_ema_boundary_gap_hand_values():
+    """EMA 0.5 (sink), 0.30, 0.12, 0.20, 0.03: the non-sink values ranked are 0.30, 0.20, 0.12,
+    0.03 and C - 1 of them are kept; the gap is (last kept - first dropped) / last kept."""
+    ema = np.array([0.5, 0.30, 0.12, 0.20, 0.03])
+    gids = [0, 11, 12, 13, 14]
+    sink = [True, False, False, False, False]
+    got = {C: O.ema_boundary_gap(ema, gids, sink, C) for C in range(1, 6)}
+    assert got[1] == float("inf") and got[5] == float("inf")
+    assert got[2] == pytest.approx(0.1 / 0.3, rel=1e-12)
+    assert got[3] == pytest.approx(0.08 / 0.20, rel=1e-12)
+    assert got[4] == pytest.approx(0.09 / 0.12, rel=1e-12)
+
+
 # ------------------------------------------------------------------ hierarchical (frame -> block) selection
 def test_hsa_frames_ranked_by_mean_not_by_best_block():
     """Hand-built case: frame 0 holds the single best block but the lowest mean, frame 1 the

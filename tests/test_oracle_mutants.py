@@ -30,6 +30,9 @@ PINS = {
     "rollout_ema": T.test_rollout_carries_the_ema_between_updates,
     "single_step": T.test_single_step_partition_5s,
     "train_masks": T.test_train_masks_shape,
+    "train_select": T.test_train_masks_selection_hand_built,
+    "kth_gap": T.test_kth_gap_hand_values,
+    "ema_gap": T.test_ema_boundary_gap_hand_values,
     "hsa_mean": T.test_hsa_frames_ranked_by_mean_not_by_best_block,
     "hsa_flat": lambda: [T.test_hsa_reduces_to_flat_topk(s) for s in (0, 1, 2)],
     "hsa_brute": T.test_hsa_brute_force_small,
@@ -95,6 +98,26 @@ MUTANTS = [
      "own = frame_blocks(range(c * chunk, c * chunk + 1), bpf)", ["train_masks"]),
     ("training masks: sinks missing from later chunks", "mh.append(frame_blocks([0], bpf) + sorted(earlier[i] for i in pos) + own)",
      "mh.append(sorted(earlier[i] for i in pos) + own)", ["train_masks"]),
+    ("training masks: every row scored with the chunk's first query block",
+     "sc = coarse_scores(qr[h][r:r + 1], kr[h][earlier]", "sc = coarse_scores(qr[h][c * chunk * bpf:c * chunk * bpf + 1], kr[h][earlier]",
+     ["train_select"]),
+    ("training masks: keys of the other batch item", "kr = block_reps(k[b], geom, batch_frames)",
+     "kr = block_reps(k[B - 1 - b], geom, batch_frames)", ["train_select"]),
+    ("training masks: own chunk among the candidates", "earlier = frame_blocks(range(1, c * chunk), bpf)",
+     "earlier = frame_blocks(range(1, (c + 1) * chunk), bpf)", ["train_select"]),
+    ("training masks: sinks among the candidates", "earlier = frame_blocks(range(1, c * chunk), bpf)",
+     "earlier = frame_blocks(range(0, c * chunk), bpf)", ["train_select"]),
+    ("k-th gap taken one place early", "return abs(float(scores[order[k - 1]]) - float(scores[order[k]]))",
+     "return abs(float(scores[order[k - 2]]) - float(scores[order[k - 1]]))", ["kth_gap"]),
+    ("k-th gap of zero when nothing is cut", "    if k <= 0 or k >= len(order):\n        return float(\"inf\")",
+     "    if k <= 0 or k >= len(order):\n        return 0.0", ["kth_gap"]),
+    ("EMA boundary gap absolute instead of relative",
+     "return abs(vals[free - 1] - vals[free]) / max(abs(vals[free - 1]), 1e-30)",
+     "return abs(vals[free - 1] - vals[free])", ["ema_gap"]),
+    ("EMA boundary gap ranks the sinks too", "vals = sorted((float(ema[i]) for i in range(len(pool_gids)) if not sink[i]), reverse=True)",
+     "vals = sorted((float(ema[i]) for i in range(len(pool_gids))), reverse=True)", ["ema_gap"]),
+    ("EMA boundary gap one place late", "return abs(vals[free - 1] - vals[free]) / max(abs(vals[free - 1]), 1e-30)",
+     "return abs(vals[free] - vals[min(free + 1, len(vals) - 1)]) / max(abs(vals[free]), 1e-30)", ["ema_gap"]),
 ]
 
 
