@@ -405,7 +405,8 @@ def train_masks(q, k, geom: dict, batch_frames: int, chunk: int, topk: int):
     """Fixed block masks of the trainable path, per (batch, head, query block): global ids.
 
     Chunk 0 attends its own blocks.  A later chunk attends the sinks (frame 0), its top-k
-    blocks among the earlier non-sink blocks, and its own chunk's blocks.  ``q``/``k``
+    blocks among the earlier non-sink blocks, and its own chunk's blocks (a sequence whose
+    length is not a whole number of chunks ends with a shorter chunk).  ``q``/``k``
     are ``[B, T, H, d]``.  Returns masks[b][h][r] (r over all query blocks of the sequence)
     and the k-th gaps.
     """
@@ -420,7 +421,7 @@ def train_masks(q, k, geom: dict, batch_frames: int, chunk: int, topk: int):
             mh, gh = [], []
             for r in range(batch_frames * bpf):
                 c = (r // bpf) // chunk
-                own = frame_blocks(range(c * chunk, (c + 1) * chunk), bpf)
+                own = frame_blocks(range(c * chunk, min((c + 1) * chunk, batch_frames)), bpf)
                 if c == 0:
                     mh.append(own)
                     gh.append(float("inf"))

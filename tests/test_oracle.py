@@ -280,6 +280,10 @@ def test_train_masks_shape():
     assert len(m[12]) == 4 + 2 + 12 and set(m[12][:4]) == set(range(4))
     assert set(m[12][4:6]) <= set(range(4, 12))
     assert set(m[30][4:6]) <= set(range(4, 24))
+    # 8 frames: the last chunk holds frames 6 and 7 only
+    masks, _ = O.train_masks(q[:, :8 * 256], k[:, :8 * 256], g, 8, 3, topk=2)
+    m = masks[0][0]
+    assert len(m) == 32 and m[31][-8:] == list(range(24, 32)) and len(m[31]) == 4 + 2 + 8
 
 
 def _const_block_tokens(reps, fh, fw, th, tw, n_frames):

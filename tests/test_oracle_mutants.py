@@ -94,8 +94,11 @@ MUTANTS = [
     ("attended query block indexed as if the chunk began at frame 0",
      "qb = block_tokens(q, geom, q_first_frame * bpf + r, q_first_frame)",
      "qb = block_tokens(q, geom, q_first_frame * bpf + r, 0)", ["dense"]),
-    ("training masks: own chunk is one frame", "own = frame_blocks(range(c * chunk, (c + 1) * chunk), bpf)",
+    ("training masks: own chunk is one frame", "own = frame_blocks(range(c * chunk, min((c + 1) * chunk, batch_frames)), bpf)",
      "own = frame_blocks(range(c * chunk, c * chunk + 1), bpf)", ["train_masks"]),
+    ("training masks: a short last chunk runs past the sequence",
+     "own = frame_blocks(range(c * chunk, min((c + 1) * chunk, batch_frames)), bpf)",
+     "own = frame_blocks(range(c * chunk, (c + 1) * chunk), bpf)", ["train_masks"]),
     ("training masks: sinks missing from later chunks", "mh.append(frame_blocks([0], bpf) + sorted(earlier[i] for i in pos) + own)",
      "mh.append(sorted(earlier[i] for i in pos) + own)", ["train_masks"]),
     ("training masks: every row scored with the chunk's first query block",
