@@ -97,21 +97,20 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def profiled_traffic(profile: str, source: str):
-    """DRAM bytes per launch from a committed ncu summary, or None when the kernel source has
-    changed since the counters were taken (the summary records the source's sha256 prefix)."""
+def profiled_traffic(record: str, source: str):
+    """DRAM bytes per launch from the ncu counters recorded beside the profile summaries
+    (``profiles/<record>``: a small JSON with the kernel source's sha256 prefix), or None when
+    the kernel source has changed since the counters were taken."""
     import hashlib
-    import re
     try:
-        text = open(os.path.join(ROOT, "profiles", profile)).read()
+        with open(os.path.join(ROOT, "profiles", record)) as f:
+            rec = json.load(f)
         sha = hashlib.sha256(open(os.path.join(ROOT, source), "rb").read()).hexdigest()[:16]
-    except OSError:
+    except (OSError, ValueError):
         return None
-    m_sha = re.search(r"kernel_source_sha256:\s*([0-9a-f]+)", text)
-    m_tr = re.search(r"traffic_bytes_per_launch:\s*(\d+)", text)
-    if not m_sha or not m_tr or m_sha.group(1) != sha:
+    if rec.get("kernel_source_sha256") != sha:
         return None
-    return int(m_tr.group(1))
+    return int(rec["dram_bytes_per_launch"])
 
 
 def workload_config(w):
@@ -125,31 +124,30 @@ def workload_config(w):
 
 # ----------------------------------------------------------------------------- CPU oracle arm
 def oracle_sample(w, q, k, v, units: int, seed: int = 0):
-    """Time the oracle on a bounded sample of one chunk decode; returns (seconds extrapolated
-    to the full step, description, threads)."""
+    """Time the oracle, single-threaded (BLAS pools limited to one thread), on a bounded sample of
+    one chunk decode; returns (seconds extrapolated to the full step, description, threads)."""
+    from threadpoolctl import threadpool_info, threadpool_limits
     from oracle import pbsa_oracle as O
-    try:
-        from threadpoolctl import threadpool_info
-        threads = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
-    except Exception:  # pragma: no cover - informational only
-        threads = 1
     gd = {"frame_h": w.frame_h, "frame_w": w.frame_w, "tile_h": w.tile_h, "tile_w": w.tile_w, "scale": w.scale}
     q64, k64, v64 = (t.double().numpy() for t in (q, k, v))
-    t0 = time.perf_counter()
-    plan = O.single_step_plan(q64, k64, gd, w.hist_frames, w.chunk_frames, w.capacity, w.window_frames,
-                              w.topk, w.gamma)
-    t_plan = time.perf_counter() - t0
     nq = w.chunk_frames * w.blocks_per_frame
-    rng = np.random.default_rng(seed)
-    pick = rng.choice(w.heads * nq, size=units, replace=False)
-    t0 = time.perf_counter()
-    for u in pick:
-        h, r = divmod(int(u), nq)
-        O.attend_gids(q64, k64, v64, gd, h, r, plan["P"][h] + plan["sel"][h][r], q_first_frame=w.hist_frames)
-    t_att = (time.perf_counter() - t0) / units
+    with threadpool_limits(limits=1):
+        threads = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+        t0 = time.perf_counter()
+        plan = O.single_step_plan(q64, k64, gd, w.hist_frames, w.chunk_frames, w.capacity, w.window_frames,
+                                  w.topk, w.gamma)
+        t_plan = time.perf_counter() - t0
+        rng = np.random.default_rng(seed)
+        pick = rng.choice(w.heads * nq, size=units, replace=False)
+        t0 = time.perf_counter()
+        for u in pick:
+            h, r = divmod(int(u), nq)
+            O.attend_gids(q64, k64, v64, gd, h, r, plan["P"][h] + plan["sel"][h][r], q_first_frame=w.hist_frames)
+        t_att = (time.perf_counter() - t0) / units
     full = t_plan + t_att * w.heads * nq
-    desc = (f"oracle selection/update plan for all {w.heads} heads (timed whole, {t_plan:.2f}s) + "
-            f"fine attention of {units} of {w.heads * nq} (head, query block) units, extrapolated")
+    desc = (f"single-threaded oracle: selection/update plan for all {w.heads} heads (timed whole, {t_plan:.2f}s) + "
+            f"fine attention of {units} of {w.heads * nq} (head, query block) units timed and extrapolated "
+            f"to all of them ({t_att * 1e3:.1f} ms per unit)")
     return full, desc, threads
 
 
@@ -202,63 +200,70 @@ def algorithmic_bytes(w, ncopy: int):
 
 
 def run_train(P, I, dev, steps: int, peaks):
-    """Trainable-path workload (batch 2 x 9 frames, 12 heads, 3-frame chunks, sinks + top-16
-    + own chunk): forward (pbsa_attend) and backward (pbsa_attend_bwd), timed separately with
-    CUDA events, L2 flushed before each; inputs resident in HBM."""
+    """Trainable-path workload (batch 2 x 9 frames, 12 heads, 3-frame chunks; every query block
+    of a later chunk attends the 24 sinks + its top-16 earlier blocks by coarse score + its own
+    chunk): the masks (pbsa_blockify_train_select), the forward (pbsa_attend) and the backward
+    (pbsa_attend_bwd), each timed with CUDA events, L2 flushed before each; inputs resident in HBM."""
     w = I.TRAIN_FWD_BWD
     frames, batch = w.total_frames, w.batch
     qf = batch * frames
+    q4, k4, v4, do4 = I.train_inputs(w, device=dev)
     shape = (qf * w.tokens_per_frame, w.heads, w.head_dim)
-    gens = [torch.Generator(device=dev).manual_seed(I.stream_seed(w.seed, 20 + i)) for i in range(4)]
-    q, k, v, do = (torch.randn(shape, generator=g_, device=dev).to(torch.bfloat16) for g_ in gens)
-    lists = I.train_lists(w, I.stream_seed(w.seed, 30))
+    q, k, v, do = (t.reshape(shape) for t in (q4, k4, v4, do4))
     nq = qf * w.blocks_per_frame
-    ld = max(len(l) for row in lists for l in row)
-    kv = torch.zeros((w.heads, nq, ld), dtype=torch.int32)
-    cnt = torch.zeros((w.heads, nq), dtype=torch.int32)
-    for h in range(w.heads):
-        for r in range(nq):
-            kv[h, r, :len(lists[h][r])] = torch.tensor(lists[h][r], dtype=torch.int32)
-            cnt[h, r] = len(lists[h][r])
-    kv, cnt = kv.to(dev), cnt.to(dev)
     g = P.make_geom(w.heads, w.head_dim, w.frame_h, w.frame_w, w.tile_h, w.tile_w, w.scale, "bf16")
     slots = nq
+    ld = w.n_sink + w.topk + w.chunk_frames * w.blocks_per_frame
     kp = torch.empty((w.heads, slots, 64, w.head_dim), dtype=torch.bfloat16, device=dev)
     vp = torch.empty_like(kp)
-    reps = torch.empty((w.heads, slots, w.head_dim), device=dev)
+    k_reps = torch.empty((w.heads, slots, w.head_dim), device=dev)
+    q_reps = torch.empty((w.heads, nq, w.head_dim), device=dev)
+    kv = torch.empty((w.heads, nq, ld), dtype=torch.int32, device=dev)
+    cnt = torch.empty((w.heads, nq), dtype=torch.int32, device=dev)
     ws = torch.zeros(max(P.pbsa_workspace_bytes(g, 64, 64), P.pbsa_bwd_workspace_bytes(g, qf, slots, ld)),
                      dtype=torch.uint8, device=dev)
-    P.pbsa_blockify(g, k, qf, reps, slots, None, kp, slots, ws)
-    P.pbsa_blockify(g, v, qf, reps, slots, None, vp, slots, ws)
+    P.pbsa_blockify_kv(g, k, v, qf, k_reps, None, slots, None, kp, vp, slots, ws=ws)
     o = torch.empty_like(q)
     lse = torch.empty((w.heads, q.shape[0]), device=dev)
     dq = torch.empty_like(q)
     dk, dv = torch.empty_like(kp), torch.empty_like(vp)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    fwd_ms, bwd_ms = [], []
+    sel_ms, fwd_ms, bwd_ms = [], [], []
     for it in range(steps + 2):
-        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-        flush.fill_(1)
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+        flush.fill_(0)
         e[0].record()
-        P.pbsa_attend(g, q, qf, kp, vp, slots, kv, cnt, ld, o, lse, ws)
+        P.pbsa_blockify_train_select(g, q, qf, q_reps, k_reps, slots, frames, w.chunk_frames, 1, w.topk,
+                                     kv, cnt, ld, None, ws)
         e[1].record()
-        flush.fill_(2)
+        flush.fill_(1)
         e[2].record()
-        P.pbsa_attend_bwd(g, q, qf, kp, vp, slots, kv, cnt, ld, o, do, lse, dq, dk, dv, ws)
+        P.pbsa_attend(g, q, qf, kp, vp, slots, kv, cnt, ld, o, lse, ws)
         e[3].record()
+        flush.fill_(2)
+        e[4].record()
+        P.pbsa_attend_bwd(g, q, qf, kp, vp, slots, kv, cnt, ld, o, do, lse, dq, dk, dv, ws)
+        e[5].record()
         torch.cuda.synchronize(dev)
         if it >= 2:
-            fwd_ms.append(e[0].elapsed_time(e[1]))
-            bwd_ms.append(e[2].elapsed_time(e[3]))
+            sel_ms.append(e[0].elapsed_time(e[1]))
+            fwd_ms.append(e[2].elapsed_time(e[3]))
+            bwd_ms.append(e[4].elapsed_time(e[5]))
     _check_device(P, ws, "in the training workload")
     fwd_flops = 4.0 * 64 * 64 * w.head_dim * float(cnt.sum().item())
     bwd_flops = 2.5 * fwd_flops
-    fm, bm = statistics.mean(fwd_ms), statistics.mean(bwd_ms)
+    sm, fm, bm = statistics.mean(sel_ms), statistics.mean(fwd_ms), statistics.mean(bwd_ms)
+    sel_bytes = q.numel() * 2 + q_reps.numel() * 4 + k_reps.numel() * 4 + kv.numel() * 4
     return {"workload": w.name, "query_blocks": nq, "heads": w.heads, "steps": steps,
+            "masks": "24 sinks + top-16 by coarse score among the earlier non-sink blocks + own chunk "
+                     "(pbsa_blockify_train_select)",
+            "select_ms": sm, "select_algorithmic_bytes": sel_bytes,
+            "select_frac_hbm": sel_bytes / (sm * 1e-3) / 1e9 / peaks["hbm_gbs"],
             "fwd_ms": fm, "bwd_ms": bm, "fwd_flops": fwd_flops, "bwd_flops": bwd_flops,
             "fwd_tflops": fwd_flops / (fm * 1e-3) / 1e12, "bwd_tflops": bwd_flops / (bm * 1e-3) / 1e12,
+            "fwd_frac_of_bf16_peak": fwd_flops / (fm * 1e-3) / 1e12 / peaks["bf16"],
             "bwd_frac_of_bf16_peak": bwd_flops / (bm * 1e-3) / 1e12 / peaks["bf16"],
-            "launches_per_iteration": 6,
+            "launches_per_iteration": 1 + 1 + 5,
             "note": "bwd FLOPs counted as 2.5x the forward's (5 GEMM-sized contractions vs 2); "
                     "the deterministic kernels recompute S and dP in both the dQ and the dK/dV passes"}
 
@@ -311,7 +316,7 @@ def run_rollout(P, I, dev, w, max_chunks=None, k_schedule=None, label=None):
 
     stream = torch.cuda.current_stream(dev)
     per_chunk, flops_chunk, o = [], [], None
-    peak_alloc = 0
+    peak_alloc = peak_caches = 0
     for c, (f0, nf) in enumerate(chunks):
         if k_schedule is not None:
             for ca in caches:
@@ -321,6 +326,7 @@ def run_rollout(P, I, dev, w, max_chunks=None, k_schedule=None, label=None):
             o = torch.empty((nf * w.tokens_per_frame, H, d), dtype=torch.bfloat16, device=dev)
         torch.cuda.synchronize(dev)
         torch.cuda.reset_peak_memory_stats(dev)
+        harness = torch.cuda.memory_allocated(dev) - base_alloc - kv_alloc   # this chunk's inputs, o
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         cnt_layer0 = None
@@ -339,6 +345,7 @@ def run_rollout(P, I, dev, w, max_chunks=None, k_schedule=None, label=None):
         e1.synchronize()
         per_chunk.append(e0.elapsed_time(e1))
         peak_alloc = max(peak_alloc, torch.cuda.max_memory_allocated(dev) - base_alloc)
+        peak_caches = max(peak_caches, torch.cuda.max_memory_allocated(dev) - base_alloc - harness)
         blocks = int(cnt_layer0.sum().item()) if cnt_layer0 is not None else H * (nf * bpf) ** 2
         flops_chunk.append(4.0 * 64 * 64 * d * blocks * w.steps * w.layers)
         del inp
@@ -358,7 +365,9 @@ def run_rollout(P, I, dev, w, max_chunks=None, k_schedule=None, label=None):
         "selected_tflops_steady": tf_steady,
         "kv_cache_bytes": {"pbsa_all_layers": kv_bytes, "dense_all_frames_all_layers": dense,
                            "ratio": kv_bytes / dense, "allocated_by_caches": kv_alloc,
-                           "peak_allocated_during_chunks": peak_alloc},
+                           "peak_allocated_during_chunks": peak_alloc,
+                           "peak_during_chunks_minus_harness_inputs": peak_caches,
+                           "measured_ratio": peak_caches / dense},
         "timing": "CUDA events around each chunk's eager launches (all layers x steps; each layer commits "
                   "right after its last-step attention)",
         "inputs": "device-drawn N(0,1) + per-tile offsets" + (" (AR(1) drift)" if w.ar_rho > 0 else ""),
@@ -375,7 +384,11 @@ def run_variant(P, I, dev, w, steps: int, **cfg_changes):
     cfg = P.LayerConfig(w.heads, w.head_dim, w.frame_h, w.frame_w, w.tile_h, w.tile_w, w.capacity,
                         w.window_frames, w.chunk_frames, w.topk, w.gamma, w.dtype,
                         (w.hist_frames - w.window_frames) * bpf, **cfg_changes)
+    torch.cuda.synchronize(dev)
+    alloc0 = torch.cuda.memory_allocated(dev)
     cache = P.PBSALayerCache(cfg, dev)
+    cache_alloc = torch.cuda.memory_allocated(dev) - alloc0      # every device buffer the cache owns
+    cache_staging = 2 * cache.k_pool[:, cache.stage_base:].numel() * cache.k_pool.element_size()
     qd, kcd, vcd = q.to(dev), kc.to(dev), vc.to(dev)
     cache.prefill(k.to(dev), v.to(dev), w.hist_frames, cache.query_reps(qd))
     step = P.ChunkDecodeStep(cache)
@@ -532,7 +545,11 @@ def run_pbsa(args, w, rank, world, local_rank):
     cfg = P.LayerConfig(w.heads, w.head_dim, w.frame_h, w.frame_w, w.tile_h, w.tile_w, w.capacity,
                         w.window_frames, w.chunk_frames, w.topk, w.gamma, w.dtype,
                         (w.hist_frames - w.window_frames) * bpf)
+    torch.cuda.synchronize(dev)
+    alloc0 = torch.cuda.memory_allocated(dev)
     cache = P.PBSALayerCache(cfg, dev)
+    cache_alloc = torch.cuda.memory_allocated(dev) - alloc0      # every device buffer the cache owns
+    cache_staging = 2 * cache.k_pool[:, cache.stage_base:].numel() * cache.k_pool.element_size()
     qd, kcd, vcd = q.to(dev), kc.to(dev), vc.to(dev)
     cache.prefill(k.to(dev), v.to(dev), w.hist_frames, cache.query_reps(qd))
     step = P.ChunkDecodeStep(cache)
@@ -644,14 +661,19 @@ def run_pbsa(args, w, rank, world, local_rank):
                      "peak": peaks["bf16"], "unit": "TFLOP/s", "frac": att_tflops / peaks["bf16"],
                      "peak_source": f"{peaks['source']} burst bf16 (cuBLAS)",
                      "frac_of_sustained": att_tflops / peaks["bf16_sustained"],
-                     "traffic": profiled_traffic("attend_tc_decode_5s.md",
+                     "traffic": profiled_traffic("attend_tc_decode_5s.counters.json",
                                                  "block_sparse_attention_pbsa_b200/csrc/attend_tc.cu"),
                      "traffic_unit": "bytes per launch (ncu dram read + write)"},
         "step_frac_of_bf16_peak": value / world / peaks["bf16"],
         "kernels": kernels,
         "ms_per_step_groups_serialised": statistics.mean(parts_total),
         "kv_cache_bytes": {"pbsa_per_layer": cache.kv_bytes,
-                           "dense_21_frames_per_layer": 2 * w.heads * 21 * w.tokens_per_frame * w.head_dim * 2},
+                           "allocated_by_cache_measured": cache_alloc,
+                           "allocated_minus_prefill_staging": cache_alloc - cache_staging,
+                           "dense_21_frames_per_layer": 2 * w.heads * 21 * w.tokens_per_frame * w.head_dim * 2,
+                           "note": "measured = torch.cuda.memory_allocated() around the cache's construction: "
+                                   "K/V pools, key representatives, slot tables, lists, workspace; the staging "
+                                   "area only serves the one-time prefill of a mid-video history"},
         "e2e": {"value": world * flops / (e2e_ms_max * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "ms_per_step": e2e_ms_max, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": step.LAUNCHES * args.steps,

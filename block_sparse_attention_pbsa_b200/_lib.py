@@ -61,6 +61,8 @@ _SIGS = {
                                       _P, _P, _I, _P, _P, _I, _P, _P, _P]),
     "pbsa_blockify_select_ex": (_I, [ctypes.POINTER(Geom), _P, _I, _P, _P, _I, _P, _P, _I, _I, _I, _I,
                                      _P, _P, _I, _P, _I, _P, _P, _I, _P, _P, _P]),
+    "pbsa_blockify_train_select": (_I, [ctypes.POINTER(Geom), _P, _I, _P, _P, _I, _I, _I, _I, _I, _P, _P, _I,
+                                        _P, _P, _P]),
     "pbsa_attend": (_I, [ctypes.POINTER(Geom), _P, _I, _P, _P, _I, _P, _P, _I, _P, _P, _P, _P]),
     "pbsa_memory_update": (_I, [ctypes.POINTER(Geom), _P, _I, _P, _P, _P, _I, _P, _P, _I, _I, _P,
                                 _P, _I, ctypes.c_float, _P, _P, _P, _P]),
@@ -196,6 +198,15 @@ def pbsa_blockify_select_ex(g: Geom, q, q_frames, q_reps, k_reps, pool_slots, ca
         _ptr(cand_gid, torch.int32, "cand_gid"), ncand, k, top_frames, n_recent_frames,
         _ptr(prefix_slot, torch.int32, "prefix_slot"), _ptr(prefix_cnt, torch.int32, "prefix_cnt"),
         prefix_ld, _ptr(suffix_slot, torch.int32, "suffix_slot"), suffix_n,
+        _ptr(out_slot, torch.int32, "out_slot"), _ptr(out_cnt, torch.int32, "out_cnt"), out_ld,
+        _ptr(out_score, torch.float32, "out_score"), _ptr(ws, None, "ws"), _stream(stream)))
+
+
+def pbsa_blockify_train_select(g: Geom, q, q_frames, q_reps, k_reps, pool_slots, seq_frames, chunk_frames,
+                               sink_frames, k, out_slot, out_cnt, out_ld, out_score=None, ws=None, stream=None):
+    _check("pbsa_blockify_train_select", load().pbsa_blockify_train_select(
+        ctypes.byref(g), _ptr(q, _tok_dtype(g), "q"), q_frames, _ptr(q_reps, torch.float32, "q_reps"),
+        _ptr(k_reps, torch.float32, "k_reps"), pool_slots, seq_frames, chunk_frames, sink_frames, k,
         _ptr(out_slot, torch.int32, "out_slot"), _ptr(out_cnt, torch.int32, "out_cnt"), out_ld,
         _ptr(out_score, torch.float32, "out_score"), _ptr(ws, None, "ws"), _stream(stream)))
 

@@ -15,6 +15,7 @@ memory update scores and copies them.
 """
 from __future__ import annotations
 
+import collections
 import dataclasses
 
 import torch
@@ -111,21 +112,27 @@ class PBSALayerCache:
         return t.to(self.device, non_blocking=True)
 
     # Candidate lists depend only on the ring geometry and the frame schedule, which every
-    # layer of a model shares: they are built once per (device, heads, ring, list) and reused.
-    _LIST_MEMO: dict = {}
+    # layer of a model shares: they are built once per (device, heads, ring, list) and reused by
+    # the layers.  Their gids change with every chunk, so only the most recent lists are kept
+    # (the device memory they hold stays bounded over a rollout of any length).
+    _LIST_MEMO: "collections.OrderedDict" = collections.OrderedDict()
+    _LIST_MEMO_MAX = 8
 
     def _list_pair(self, pairs) -> tuple[torch.Tensor, torch.Tensor]:
         """Device tensors [H, n] of the slots and gids of ``pairs`` (a list of (slot, gid))."""
         H = self.cfg.heads
+        memo = PBSALayerCache._LIST_MEMO
         key = (str(self.device), H, self.ring_frames, self.cfg.bpf, self.ring_base, tuple(pairs))
-        hit = PBSALayerCache._LIST_MEMO.get(key)
+        hit = memo.get(key)
         if hit is None:
             n = len(pairs)
             hit = (self._ints([[s for s, _ in pairs]] * H).view(H, n),
                    self._ints([[g for _, g in pairs]] * H).view(H, n))
-            if len(PBSALayerCache._LIST_MEMO) > 4096:
-                PBSALayerCache._LIST_MEMO.clear()
-            PBSALayerCache._LIST_MEMO[key] = hit
+            memo[key] = hit
+            while len(memo) > PBSALayerCache._LIST_MEMO_MAX:
+                memo.popitem(last=False)
+        else:
+            memo.move_to_end(key)
         return hit
 
     def _frames_dst(self, first: int, n: int) -> torch.Tensor:
@@ -482,25 +489,49 @@ class ChunkDecodeStep:
         torch.cuda.current_stream(self.cache.device).wait_stream(side)
         return graph
 
-    def capture_pipeline(self, q, k, v, o, lse=None):
-        """Capture the step as three graphs for ``run_pipelined``: [blockify(Q) + selection +
-        attend], [memory update] and [commit blockify(K, V)].  The update reads neither K nor V
-        of the chunk (its candidates are blocks leaving the window, never the chunk's ring
-        positions), so it runs while they upload; only the commit waits for them.  (The
-        own-chunk variant, which needs K, V before the selection, is not split.)"""
+    def capture_pipeline(self, q, k, v, o, lse=None, parts=None):
+        """Capture the step for ``run_pipelined`` as ``parts`` front graphs (default: one per
+        frame of the chunk), each [blockify(Q) + selection + attend] of its frames, then
+        [memory update] and [commit blockify(K, V)].
+
+        Q arrives frame by frame in raster order, so the first frames' selection and attention
+        run while the later frames (and K, V) are still uploading, and their O rows download
+        while the later frames compute.  The memory update takes the representatives of the
+        whole chunk, which it recomputes from the resident Q (the same kernel and order as the
+        fused selection's, so the same bits); it reads neither K nor V of the chunk (its
+        candidates are blocks leaving the window, never the chunk's ring positions), so it runs
+        while they upload, and only the commit waits for them.  Every query block's selection and
+        attention are independent of the others', so the results equal ``run``'s bit for bit.
+        (The own-chunk variant, which needs K, V before the selection, is not split.)"""
         if self.cache.cfg.own_chunk:
             raise ValueError("the own-chunk variant writes K, V before the selection: use capture()")
-        dev = self.cache.device
-        front, mid, back = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        ca, c = self.cache, self.cache.cfg
+        parts = parts or self.q_frames
+        if self.q_frames % parts:
+            raise ValueError(f"{self.q_frames} frames do not split into {parts} equal parts")
+        fpp = self.q_frames // parts                 # frames per part
+        rows, nqp = fpp * c.tpf, fpp * c.bpf
+        dev = ca.device
+        g, ws, ps = ca.geom, ca.ws, ca.pool_slots
+        H = c.heads
         side = torch.cuda.Stream(device=dev)
         side.wait_stream(torch.cuda.current_stream(dev))
-        ca, c = self.cache, self.cache.cfg
-        g, ws, ps = ca.geom, ca.ws, ca.pool_slots
-        with torch.cuda.graph(front, stream=side):
-            ca._select_fused(q, self.q_frames, self.q_reps, self.kv_slot, self.kv_cnt, ca.kv_ld)
-            L.pbsa_attend(g, q, self.q_frames, ca.k_pool, ca.v_pool, ps, self.kv_slot, self.kv_cnt, ca.kv_ld,
-                          o, lse, ws=ws)
+        fronts, part_bufs = [], []
+        for p in range(parts):
+            qp, op = q[p * rows:(p + 1) * rows], o[p * rows:(p + 1) * rows]
+            lp = lse[:, p * rows:(p + 1) * rows].contiguous() if lse is not None else None
+            bufs = (torch.zeros((H, nqp, c.head_dim), dtype=torch.float32, device=dev),
+                    torch.zeros((H, nqp, ca.kv_ld), dtype=torch.int32, device=dev),
+                    torch.zeros((H, nqp), dtype=torch.int32, device=dev), lp)
+            part_bufs.append(bufs)
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=side):
+                ca._select_fused(qp, fpp, bufs[0], bufs[1], bufs[2], ca.kv_ld)
+                L.pbsa_attend(g, qp, fpp, ca.k_pool, ca.v_pool, ps, bufs[1], bufs[2], ca.kv_ld, op, lp, ws=ws)
+            fronts.append(gr)
+        mid, back = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
         with torch.cuda.graph(mid, stream=side):   # the kernels of run(): the same results, bit for bit
+            L.pbsa_blockify(g, q, self.q_frames, self.q_reps, self.nq, ws=ws)
             L.pbsa_memory_update_plan(g, self.q_reps, self.nq, ca.k_reps, ps, ca.slot_gid, ca.slot_ema, c.capacity,
                                       c.bpf, self.cs, self.cg, self.ncand, c.gamma, ca.p_list, ca.p_cnt, ws=ws)
             L.pbsa_memory_update_apply(g, ca.k_reps, ca.k_pool, ca.v_pool, ps, c.capacity, self.ncand, ws=ws)
@@ -508,38 +539,52 @@ class ChunkDecodeStep:
             L.pbsa_blockify_kv(g, k, v, self.q_frames, ca.k_reps, None, ps, self.dst, ca.k_pool, ca.v_pool, ps,
                                ws=ws)
         torch.cuda.current_stream(dev).wait_stream(side)
-        self._pipe = {"front": front, "mid": mid, "back": back, "bufs": (q, k, v, o),
+        self._pipe = {"fronts": fronts, "mid": mid, "back": back, "bufs": (q, k, v, o), "rows": rows,
+                      "part_bufs": part_bufs, "lse": lse,
                       "h2d": torch.cuda.Stream(device=dev), "d2h": torch.cuda.Stream(device=dev)}
+        # launches per pipelined step: per part the fused selection and attend; blockify(Q), plan,
+        # apply; the commit
+        self.PIPELINED_LAUNCHES = 2 * parts + 3 + 1
 
     def run_pipelined(self, qh, kh, vh, oh):
         """One step from pinned host buffers to a pinned host result, with the transfers
-        overlapped: Q is uploaded first and the front graph (selection + attention) starts as
-        soon as it lands, while K and V upload on a copy stream; O downloads on another stream
-        while the memory update runs, and the commit of K and V follows their upload.  All
-        work is ordered on the current stream's timeline when this returns (asynchronously)."""
+        overlapped: Q is uploaded part by part (frames in raster order) and each part's front
+        graph (selection + attention) starts as soon as its rows land, while the later parts and
+        then K and V upload on a copy stream; each part's O rows download on another stream as
+        soon as they are computed; the memory update runs while K and V upload, and the commit
+        of K and V follows their upload.  All work is ordered on the current stream's timeline
+        when this returns (asynchronously)."""
         p = self._pipe
         q, k, v, o = p["bufs"]
+        rows = p["rows"]
         main = torch.cuda.current_stream(self.cache.device)
         h2d, d2h = p["h2d"], p["d2h"]
         h2d.wait_stream(main)                       # previous step done with k, v, q
         d2h.wait_stream(main)
+        landed = []
         with torch.cuda.stream(h2d):
-            q.copy_(qh, non_blocking=True)
-            q_done = torch.cuda.Event()
-            q_done.record(h2d)
+            for i in range(len(p["fronts"])):
+                q[i * rows:(i + 1) * rows].copy_(qh[i * rows:(i + 1) * rows], non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(h2d)
+                landed.append(ev)
             k.copy_(kh, non_blocking=True)
             v.copy_(vh, non_blocking=True)
-        main.wait_event(q_done)
-        p["front"].replay()
-        front_done = torch.cuda.Event()
-        front_done.record(main)
-        with torch.cuda.stream(d2h):
-            d2h.wait_event(front_done)
-            oh.copy_(o, non_blocking=True)
+        for i, gr in enumerate(p["fronts"]):
+            main.wait_event(landed[i])
+            gr.replay()
+            done = torch.cuda.Event()
+            done.record(main)
+            with torch.cuda.stream(d2h):
+                d2h.wait_event(done)
+                oh[i * rows:(i + 1) * rows].copy_(o[i * rows:(i + 1) * rows], non_blocking=True)
         p["mid"].replay()                           # memory update (needs no K, V)
         main.wait_stream(h2d)                       # K, V uploaded
         p["back"].replay()
         main.wait_stream(d2h)                       # O downloaded
+        if p["lse"] is not None:
+            for i, b in enumerate(p["part_bufs"]):
+                p["lse"][:, i * rows:(i + 1) * rows].copy_(b[3])
         return oh
 
     def snapshot(self):

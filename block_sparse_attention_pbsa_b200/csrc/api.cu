@@ -204,6 +204,31 @@ pbsa_status pbsa_blockify_hsa_select(const pbsa_geom* gin, const void* q, int q_
                                  nullptr, 0, out_slot, out_cnt, out_ld, out_score, ws, stream);
 }
 
+pbsa_status pbsa_blockify_train_select(const pbsa_geom* gin, const void* q, int q_frames, float* q_reps,
+                                       const float* k_reps, int pool_slots, int seq_frames, int chunk_frames,
+                                       int sink_frames, int k, int* out_slot, int* out_cnt, int out_ld,
+                                       float* out_score, void* ws, void* stream) {
+  Geo g;
+  pbsa_status s = make_geo(gin, &g);
+  if (s != PBSA_OK) return s;
+  if (q == nullptr || q_reps == nullptr || k_reps == nullptr || out_slot == nullptr || out_cnt == nullptr)
+    return PBSA_ERR_INVALID_ARG;
+  if (q_frames <= 0 || seq_frames <= 0 || chunk_frames <= 0 || k < 0 || q_frames % seq_frames != 0)
+    return PBSA_ERR_INVALID_ARG;
+  if (sink_frames < 0 || sink_frames > chunk_frames || sink_frames > seq_frames) return PBSA_ERR_INVALID_ARG;
+  if ((int64_t)q_frames * g.bpf > 65535 * 64) return PBSA_ERR_INVALID_ARG;
+  if (pool_slots < q_frames * g.bpf) return PBSA_ERR_INVALID_ARG;
+  const int own = (chunk_frames < seq_frames ? chunk_frames : seq_frames) * g.bpf;
+  if ((int64_t)out_ld < (int64_t)sink_frames * g.bpf + k + own) return PBSA_ERR_INVALID_ARG;
+  const int n_chunks = (seq_frames + chunk_frames - 1) / chunk_frames;
+  if (n_chunks > 1 && (int64_t)((n_chunks - 1) * chunk_frames - sink_frames) * g.bpf > 1024)
+    return PBSA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(q_reps) || !aligned16(k_reps)) return PBSA_ERR_INVALID_ARG;
+  return from_cuda(launch_blockify_train_select(g, q, q_frames, q_reps, k_reps, pool_slots, seq_frames,
+                                                chunk_frames, sink_frames, k, out_slot, out_cnt, out_ld,
+                                                out_score, ws, static_cast<cudaStream_t>(stream)));
+}
+
 pbsa_status pbsa_attend(const pbsa_geom* gin, const void* q, int q_frames, const void* k_pool,
                         const void* v_pool, int pool_slots, const int* kv_slot, const int* kv_cnt,
                         int kv_ld, void* o, float* lse, void* ws, void* stream) {

@@ -25,6 +25,13 @@
 // of the frame's mean-pooled representative, by linearity), summed in block order; the
 // n_recent latest frames are always chosen, plus the top_frames best others (score
 // descending, the earlier frame on ties); blocks of the other frames leave the ranking.
+//
+// Chunk-causal variant (the trainable path: English 2.D "Training Strategy", the model is trained
+// with the same dynamic sparse cache): sequences are folded into the frame axis and the pool holds
+// their blocks in order (slot = global block id).  Query block r of sequence s, chunk c, attends
+// its own chunk; for c >= 1 also the sequence's sink blocks and the top-k blocks, by the same
+// coarse score, among the sequence's earlier non-sink blocks.  The lists come from r alone, so
+// no candidate list is read; the selection is the flat top-k above.
 #include <math.h>
 
 #include "common.cuh"
@@ -37,6 +44,35 @@ constexpr int BS_THREADS = 256;
 constexpr int BS_BATCH = 9;   // candidates per warp in flight (144 candidates: two rounds)
 constexpr int SORT_N = 256;   // candidate lists up to this long are ranked by a bitonic sort
 constexpr int HSA_MAX_FRAMES = 256;
+
+// Chunk-causal lists (seq_blocks = 0: the lists come from the call's arguments).
+struct Causal {
+  int seq_blocks;    // blocks per sequence
+  int chunk_blocks;  // blocks per chunk
+  int sink_blocks;   // leading blocks of a sequence that every later chunk attends
+  int n_chunks;      // chunks per sequence (the last may be shorter)
+  int groups;        // 8-query-block groups per chunk (the 8-block kernel's grid)
+};
+
+// Lists of query block r: candidates [cbase, cbase + ncand), prefix [pbase, pbase + pc),
+// suffix [sbase, sbase + sn) -- all slots = global block ids.
+struct CausalLists {
+  int cbase, ncand, pbase, pc, sbase, sn;
+};
+__device__ __forceinline__ CausalLists causal_lists(const Causal& cz, int r) {
+  const int sq0 = (r / cz.seq_blocks) * cz.seq_blocks;
+  const int c = (r - sq0) / cz.chunk_blocks;
+  const int cs = sq0 + c * cz.chunk_blocks;
+  const int ce = min(cs + cz.chunk_blocks, sq0 + cz.seq_blocks);
+  CausalLists l;
+  l.cbase = sq0 + cz.sink_blocks;
+  l.ncand = c == 0 ? 0 : cs - l.cbase;
+  l.pbase = sq0;
+  l.pc = c == 0 ? 0 : cz.sink_blocks;
+  l.sbase = cs;
+  l.sn = ce - cs;
+  return l;
+}
 
 template <typename T>
 __device__ __forceinline__ void add_chunk16(float* acc, const uint4& v);
@@ -66,14 +102,14 @@ __device__ __forceinline__ void vec_to(const float4& v, float* o) { o[0] = v.x; 
 __device__ __forceinline__ void vec_to(const float2& v, float* o) { o[0] = v.x; o[1] = v.y; }
 __device__ __forceinline__ void vec_to(const float& v, float* o) { o[0] = v; }
 
-template <typename T, int D, bool HSA>
+template <typename T, int D, bool HSA, bool CAUSAL>
 __global__ void __launch_bounds__(BS_THREADS) blockify_select_kernel(
     const T* __restrict__ x, Geo g, int nq, float* __restrict__ q_reps,
     const float* __restrict__ k_reps, int pool_slots, const int* __restrict__ cand_slot,
-    const int* __restrict__ cand_gid, int ncand, int k, const int* __restrict__ prefix_slot,
+    const int* __restrict__ cand_gid, int ncap, int k, const int* __restrict__ prefix_slot,
     const int* __restrict__ prefix_cnt, int prefix_ld, int* __restrict__ out_slot,
     int* __restrict__ out_cnt, int out_ld, float* __restrict__ out_score, int top_frames,
-    int n_recent, const int* __restrict__ suffix_slot, int suffix_n, void* ws) {
+    int n_recent, const int* __restrict__ suffix_slot, int suffix_n, Causal cz, void* ws) {
   constexpr int VEC = 16 / sizeof(T);   // token elements per 16-byte chunk
   constexpr int CPR = D / VEC;          // chunks per token row
   constexpr int RPP = BS_THREADS / CPR; // rows per pass
@@ -83,13 +119,16 @@ __global__ void __launch_bounds__(BS_THREADS) blockify_select_kernel(
   __shared__ float part[RPP][D];
   __shared__ float qb[D];
   extern __shared__ uint64_t dyn[];
-  uint64_t* key = dyn;                                          // [ncand]
-  float* sc = reinterpret_cast<float*>(key + ncand);            // [ncand]
-  int* gid = reinterpret_cast<int*>(sc + ncand);                // [ncand]
-  int* slot = gid + ncand;                                      // [ncand]
+  uint64_t* key = dyn;                                          // [ncap]
+  float* sc = reinterpret_cast<float*>(key + ncap);             // [ncap]
+  int* gid = reinterpret_cast<int*>(sc + ncap);                 // [ncap]
+  int* slot = gid + ncap;                                       // [ncap]
 
   const int r = blockIdx.x, h = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  CausalLists cl = {0, ncap, 0, 0, 0, suffix_n};
+  if (CAUSAL) cl = causal_lists(cz, r);
+  const int ncand = cl.ncand;
 
   // ---- 1. loads: the block's tokens and the candidate list
   const int f = r / g.bpf, rem = r - f * g.bpf;
@@ -104,8 +143,8 @@ __global__ void __launch_bounds__(BS_THREADS) blockify_select_kernel(
     v[p] = __ldg(reinterpret_cast<const uint4*>(x + (t * g.H + h) * D) + c);
   }
   for (int j = tid; j < ncand; j += BS_THREADS) {
-    gid[j] = cand_gid[(size_t)h * ncand + j];
-    slot[j] = cand_slot[(size_t)h * ncand + j];
+    gid[j] = CAUSAL ? cl.cbase + j : cand_gid[(size_t)h * ncap + j];
+    slot[j] = CAUSAL ? cl.cbase + j : cand_slot[(size_t)h * ncap + j];
   }
   // ---- 2. qbar (fixed-order sums, as in the blockify kernel)
   float acc[VEC];
@@ -169,13 +208,18 @@ __global__ void __launch_bounds__(BS_THREADS) blockify_select_kernel(
   }
 
   // ---- 4. prefix, count, ranks
-  int pc = prefix_cnt ? prefix_cnt[h] : 0;
-  if (pc < 0 || pc > prefix_ld) {
-    if (tid == 0 && r == 0) record_error(ws, PBSA_ERR_DEVICE_INDEX, pc, K_SCORE);
-    pc = pc < 0 ? 0 : prefix_ld;
+  int pc = cl.pc;
+  if (!CAUSAL) {
+    pc = prefix_cnt ? prefix_cnt[h] : 0;
+    if (pc < 0 || pc > prefix_ld) {
+      if (tid == 0 && r == 0) record_error(ws, PBSA_ERR_DEVICE_INDEX, pc, K_SCORE);
+      pc = pc < 0 ? 0 : prefix_ld;
+    }
   }
+  const int sn = cl.sn;
   const size_t o = (size_t)h * nq + r;
-  for (int j = tid; j < pc; j += BS_THREADS) out_slot[o * out_ld + j] = prefix_slot[(size_t)h * prefix_ld + j];
+  for (int j = tid; j < pc; j += BS_THREADS)
+    out_slot[o * out_ld + j] = CAUSAL ? cl.pbase + j : prefix_slot[(size_t)h * prefix_ld + j];
   int kk = min(k, ncand);
   __syncthreads();
   if (HSA) {
@@ -206,8 +250,9 @@ __global__ void __launch_bounds__(BS_THREADS) blockify_select_kernel(
     __syncthreads();
     kk = min(k, n_elig_s);
   }
-  if (tid == 0) out_cnt[o] = pc + kk + suffix_n;
-  for (int j = tid; j < suffix_n; j += BS_THREADS) out_slot[o * out_ld + pc + kk + j] = suffix_slot[j];
+  if (tid == 0) out_cnt[o] = pc + kk + sn;
+  for (int j = tid; j < sn; j += BS_THREADS)
+    out_slot[o * out_ld + pc + kk + j] = CAUSAL ? cl.sbase + j : suffix_slot[j];
   if (ncand <= SORT_N) {
     // bitonic sort, descending on (key, -position); padding sorts last
     __shared__ uint64_t skey[SORT_N];
@@ -286,14 +331,14 @@ struct S8Layout {
   }
 };
 
-template <typename T, int D>
+template <typename T, int D, bool CAUSAL>
 __global__ void __launch_bounds__(S8_THREADS) blockify_select8_kernel(
     const T* __restrict__ x, Geo g, int nq, float* __restrict__ q_reps,
     const float* __restrict__ k_reps, int pool_slots, const int* __restrict__ cand_slot,
-    const int* __restrict__ cand_gid, int ncand, int k, const int* __restrict__ prefix_slot,
+    const int* __restrict__ cand_gid, int ncap, int k, const int* __restrict__ prefix_slot,
     const int* __restrict__ prefix_cnt, int prefix_ld, int* __restrict__ out_slot,
     int* __restrict__ out_cnt, int out_ld, float* __restrict__ out_score,
-    const int* __restrict__ suffix_slot, int suffix_n, void* ws) {
+    const int* __restrict__ suffix_slot, int suffix_n, Causal cz, void* ws) {
   using L = S8Layout<T, D>;
   constexpr int VEC = L::VEC, CPR = L::CPR, RPP = L::RPP, KS = L::KS;
   constexpr int PASSES = BT / RPP;
@@ -301,15 +346,29 @@ __global__ void __launch_bounds__(S8_THREADS) blockify_select8_kernel(
   constexpr int CH = D / 4;   // 16-byte chunks of a representative row
   extern __shared__ __align__(16) float sm8[];
   float* part = sm8;                                        // [S8_R][RPP][D]
-  float* kb = part + L::part_bytes() / 4;                   // [ncand][KS]
-  float* qs = kb + (size_t)ncand * KS;                      // [16][KS]
+  float* kb = part + L::part_bytes() / 4;                   // [ncap][KS]
+  float* qs = kb + (size_t)ncap * KS;                       // [16][KS]
   float* ss = qs + 16 * KS;                                 // [S8_R][ncs]
-  const int ncs = L::ncs(ncand);
-  int* slot = reinterpret_cast<int*>(ss + S8_R * ncs);      // [ncand]
-  int* gid = slot + ncand;                                  // [ncand]
+  const int ncs = L::ncs(ncap);
+  int* slot = reinterpret_cast<int*>(ss + S8_R * ncs);      // [ncap]
+  int* gid = slot + ncap;                                   // [ncap]
 
-  const int h = blockIdx.y, r0 = blockIdx.x * S8_R;
-  const int nr = min(S8_R, nq - r0);
+  const int h = blockIdx.y;
+  int r0 = blockIdx.x * S8_R, nr = min(S8_R, nq - r0);
+  CausalLists cl = {0, ncap, 0, 0, 0, suffix_n};
+  if (CAUSAL) {
+    // CTA = (sequence, chunk, group of 8 query blocks inside the chunk): a group never spans
+    // two chunks, so its 8 rows share one candidate list
+    const int per_seq = cz.n_chunks * cz.groups;
+    const int seq = blockIdx.x / per_seq, rest = blockIdx.x - seq * per_seq;
+    const int c = rest / cz.groups;
+    const int cs = seq * cz.seq_blocks + c * cz.chunk_blocks;
+    r0 = cs + (rest - c * cz.groups) * S8_R;
+    cl = causal_lists(cz, cs);
+    nr = min(S8_R, cl.sbase + cl.sn - r0);
+    if (nr <= 0) return;   // a group past the end of a shorter last chunk (whole CTA, no barrier yet)
+  }
+  const int ncand = cl.ncand;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   // ---- 1. token loads: thread = (virtual blockify thread vt, block parity); blocks bp, bp+2, ..
@@ -331,8 +390,8 @@ __global__ void __launch_bounds__(S8_THREADS) blockify_select8_kernel(
     }
   }
   for (int j = tid; j < ncand; j += S8_THREADS) {
-    gid[j] = cand_gid[(size_t)h * ncand + j];
-    slot[j] = cand_slot[(size_t)h * ncand + j];
+    gid[j] = CAUSAL ? cl.cbase + j : cand_gid[(size_t)h * ncap + j];
+    slot[j] = CAUSAL ? cl.cbase + j : cand_slot[(size_t)h * ncap + j];
   }
   for (int i = tid; i < 8 * CH; i += S8_THREADS)   // query rows 8..15 of the MMA tile are zero
     reinterpret_cast<float4*>(qs + (8 + i / CH) * KS)[i % CH] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -396,18 +455,25 @@ __global__ void __launch_bounds__(S8_THREADS) blockify_select8_kernel(
       *reinterpret_cast<float2*>(ss + gq * ncs + nt * 8 + 2 * t4) = make_float2(r0v, r1v);
     }
   }
-  int pc = prefix_cnt ? prefix_cnt[h] : 0;
-  if (pc < 0 || pc > prefix_ld) {
-    if (tid == 0 && r0 == 0) record_error(ws, PBSA_ERR_DEVICE_INDEX, pc, K_SCORE);
-    pc = pc < 0 ? 0 : prefix_ld;
+  int pc = cl.pc;
+  if (!CAUSAL) {
+    pc = prefix_cnt ? prefix_cnt[h] : 0;
+    if (pc < 0 || pc > prefix_ld) {
+      if (tid == 0 && r0 == 0) record_error(ws, PBSA_ERR_DEVICE_INDEX, pc, K_SCORE);
+      pc = pc < 0 ? 0 : prefix_ld;
+    }
   }
+  const int sn = cl.sn;
   const int kk = min(k, ncand);
-  for (int i = tid; i < nr * (pc + suffix_n); i += S8_THREADS) {
-    const int b = i / (pc + suffix_n), j = i - b * (pc + suffix_n);
+  for (int i = tid; i < nr * (pc + sn); i += S8_THREADS) {
+    const int b = i / (pc + sn), j = i - b * (pc + sn);
     const size_t o = (size_t)h * nq + r0 + b;
-    out_slot[o * out_ld + (j < pc ? j : kk + j)] = j < pc ? prefix_slot[(size_t)h * prefix_ld + j] : suffix_slot[j - pc];
+    int val;
+    if (CAUSAL) val = j < pc ? cl.pbase + j : cl.sbase + (j - pc);
+    else val = j < pc ? prefix_slot[(size_t)h * prefix_ld + j] : suffix_slot[j - pc];
+    out_slot[o * out_ld + (j < pc ? j : kk + j)] = val;
   }
-  if (tid < nr) out_cnt[(size_t)h * nq + r0 + tid] = pc + kk + suffix_n;
+  if (tid < nr) out_cnt[(size_t)h * nq + r0 + tid] = pc + kk + sn;
   __syncthreads();
 
   // ---- 3. warp b selects query block b's k best: element e = j*32 + lane (j < 8)
@@ -543,32 +609,35 @@ __global__ void __launch_bounds__(S8_THREADS) blockify_select8_kernel(
   }
 }
 
-template <typename T, int D, bool HSA>
+// ncand: the candidate count (CAUSAL: the largest over the chunks, for the shared-memory layout).
+template <typename T, int D, bool HSA, bool CAUSAL>
 cudaError_t launch_t(const Geo& g, const void* x, int q_frames, float* q_reps, const float* k_reps,
                      int pool_slots, const int* cand_slot, const int* cand_gid, int ncand, int k,
                      const int* prefix_slot, const int* prefix_cnt, int prefix_ld, int* out_slot,
                      int* out_cnt, int out_ld, float* out_score, int top_frames, int n_recent,
-                     const int* suffix_slot, int suffix_n, void* ws, cudaStream_t st) {
+                     const int* suffix_slot, int suffix_n, Causal cz, void* ws, cudaStream_t st) {
   const int nq = q_frames * g.bpf;
   if (!HSA && ncand <= 256) {
     const size_t smem8 = S8Layout<T, D>::bytes(ncand);
-    auto kern8 = blockify_select8_kernel<T, D>;
+    auto kern8 = blockify_select8_kernel<T, D, CAUSAL>;
     cudaError_t e = set_smem_once((const void*)kern8, (int)smem8);
     if (e != cudaSuccess) return e;
-    kern8<<<dim3((nq + S8_R - 1) / S8_R, g.H), S8_THREADS, smem8, st>>>(
+    const int gx = CAUSAL ? (nq / cz.seq_blocks) * cz.n_chunks * cz.groups : (nq + S8_R - 1) / S8_R;
+    kern8<<<dim3(gx, g.H), S8_THREADS, smem8, st>>>(
         static_cast<const T*>(x), g, nq, q_reps, k_reps, pool_slots, cand_slot, cand_gid, ncand, k,
-        prefix_slot, prefix_cnt, prefix_ld, out_slot, out_cnt, out_ld, out_score, suffix_slot, suffix_n, ws);
+        prefix_slot, prefix_cnt, prefix_ld, out_slot, out_cnt, out_ld, out_score, suffix_slot, suffix_n,
+        cz, ws);
     return cudaGetLastError();
   }
   const size_t smem = (size_t)ncand * (8 + 4 + 4 + 4);
-  auto kern = blockify_select_kernel<T, D, HSA>;
+  auto kern = blockify_select_kernel<T, D, HSA, CAUSAL>;
   cudaError_t e = set_smem_once((const void*)kern, (int)(smem > 0 ? smem : 8));
   if (e != cudaSuccess) return e;
   kern<<<dim3(nq, g.H), BS_THREADS, smem, st>>>(static_cast<const T*>(x), g, nq, q_reps, k_reps,
                                                  pool_slots, cand_slot, cand_gid, ncand, k,
                                                  prefix_slot, prefix_cnt, prefix_ld, out_slot,
                                                  out_cnt, out_ld, out_score, top_frames, n_recent,
-                                                 suffix_slot, suffix_n, ws);
+                                                 suffix_slot, suffix_n, cz, ws);
   return cudaGetLastError();
 }
 
@@ -582,15 +651,16 @@ cudaError_t launch_blockify_select(const Geo& g, const void* x, int q_frames, fl
                                    int n_recent, const int* suffix_slot, int suffix_n, void* ws,
                                    cudaStream_t st) {
   const bool hsa = top_frames >= 0;
-#define PBSA_BS(TT, DD)                                                                          \
-  return hsa ? launch_t<TT, DD, true>(g, x, q_frames, q_reps, k_reps, pool_slots, cand_slot,     \
-                                      cand_gid, ncand, k, prefix_slot, prefix_cnt, prefix_ld,   \
-                                      out_slot, out_cnt, out_ld, out_score, top_frames,         \
-                                      n_recent, suffix_slot, suffix_n, ws, st)                  \
-             : launch_t<TT, DD, false>(g, x, q_frames, q_reps, k_reps, pool_slots, cand_slot,    \
-                                       cand_gid, ncand, k, prefix_slot, prefix_cnt, prefix_ld,  \
-                                       out_slot, out_cnt, out_ld, out_score, 0, 0, suffix_slot, \
-                                       suffix_n, ws, st);
+  const Causal off = {0, 0, 0, 0, 0};
+#define PBSA_BS(TT, DD)                                                                            \
+  return hsa ? launch_t<TT, DD, true, false>(g, x, q_frames, q_reps, k_reps, pool_slots, cand_slot, \
+                                             cand_gid, ncand, k, prefix_slot, prefix_cnt, prefix_ld, \
+                                             out_slot, out_cnt, out_ld, out_score, top_frames,     \
+                                             n_recent, suffix_slot, suffix_n, off, ws, st)         \
+             : launch_t<TT, DD, false, false>(g, x, q_frames, q_reps, k_reps, pool_slots,         \
+                                              cand_slot, cand_gid, ncand, k, prefix_slot,          \
+                                              prefix_cnt, prefix_ld, out_slot, out_cnt, out_ld,    \
+                                              out_score, 0, 0, suffix_slot, suffix_n, off, ws, st);
   if (g.dtype == PBSA_BF16) {
     if (g.d == 128) { PBSA_BS(__nv_bfloat16, 128) }
     if (g.d == 64) { PBSA_BS(__nv_bfloat16, 64) }
@@ -600,6 +670,36 @@ cudaError_t launch_blockify_select(const Geo& g, const void* x, int q_frames, fl
     if (g.d == 32) { PBSA_BS(float, 32) }
   }
 #undef PBSA_BS
+  return cudaErrorNotSupported;
+}
+
+cudaError_t launch_blockify_train_select(const Geo& g, const void* x, int q_frames, float* q_reps,
+                                         const float* k_reps, int pool_slots, int seq_frames,
+                                         int chunk_frames, int sink_frames, int k, int* out_slot,
+                                         int* out_cnt, int out_ld, float* out_score, void* ws,
+                                         cudaStream_t st) {
+  Causal cz;
+  cz.seq_blocks = seq_frames * g.bpf;
+  cz.chunk_blocks = chunk_frames * g.bpf;
+  cz.sink_blocks = sink_frames * g.bpf;
+  cz.n_chunks = (seq_frames + chunk_frames - 1) / chunk_frames;
+  cz.groups = (cz.chunk_blocks + S8_R - 1) / S8_R;
+  // the last chunk has the most candidates: every block of the earlier chunks but the sinks
+  const int ncap = cz.n_chunks > 1 ? (cz.n_chunks - 1) * cz.chunk_blocks - cz.sink_blocks : 0;
+  if (ncap > 1024) return cudaErrorNotSupported;
+#define PBSA_TS(TT, DD)                                                                           \
+  return launch_t<TT, DD, false, true>(g, x, q_frames, q_reps, k_reps, pool_slots, nullptr, nullptr, \
+                                       ncap, k, nullptr, nullptr, 0, out_slot, out_cnt, out_ld,    \
+                                       out_score, 0, 0, nullptr, 0, cz, ws, st);
+  if (g.dtype == PBSA_BF16) {
+    if (g.d == 128) { PBSA_TS(__nv_bfloat16, 128) }
+    if (g.d == 64) { PBSA_TS(__nv_bfloat16, 64) }
+  } else {
+    if (g.d == 128) { PBSA_TS(float, 128) }
+    if (g.d == 64) { PBSA_TS(float, 64) }
+    if (g.d == 32) { PBSA_TS(float, 32) }
+  }
+#undef PBSA_TS
   return cudaErrorNotSupported;
 }
 

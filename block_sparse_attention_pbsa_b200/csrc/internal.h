@@ -53,6 +53,13 @@ cudaError_t launch_blockify_select(const Geo& g, const void* x, int q_frames, fl
                                    int n_recent, const int* suffix_slot, int suffix_n, void* ws,
                                    cudaStream_t st);
 
+// The trainable path's lists (chunk-causal, sequences folded into the frame axis, slot = block id).
+cudaError_t launch_blockify_train_select(const Geo& g, const void* x, int q_frames, float* q_reps,
+                                         const float* k_reps, int pool_slots, int seq_frames,
+                                         int chunk_frames, int sink_frames, int k, int* out_slot,
+                                         int* out_cnt, int out_ld, float* out_score, void* ws,
+                                         cudaStream_t st);
+
 cudaError_t launch_attend_f32(const Geo& g, const float* q, int q_frames, const float* k_pool,
                               const float* v_pool, int pool_slots, const int* kv_slot,
                               const int* kv_cnt, int kv_ld, float* o, float* lse, void* ws,

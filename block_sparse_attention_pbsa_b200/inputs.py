@@ -209,9 +209,10 @@ def train_lists(w: Workload, seed: int, n_frames: int | None = None, batch: int 
     Query block r of batch b (global block id b*F*bpf + r, F = frames per sequence) attends:
     its own chunk's blocks; and, for chunks after the first, the sink blocks (frame 0 of its
     sequence) plus ``topk`` blocks drawn uniformly (seeded) from the earlier non-sink blocks
-    of its sequence -- a fixed mask with the structure the trainable path uses, standing in
-    for a learned selection.  Pool slot = global block id.  Returns a list over heads of
-    lists over query blocks of slot lists.
+    of its sequence -- masks with the structure of the trainable path but random contents,
+    for structural tests of the attention kernels (the method's own masks are computed by
+    the library from the coarse scores).  Pool slot = global block id.  Returns a list over
+    heads of lists over query blocks of slot lists.
     """
     F = n_frames or w.total_frames
     B = batch or w.batch

@@ -190,6 +190,33 @@ PBSA_API pbsa_status pbsa_blockify_select_ex(const pbsa_geom* g, const void* q, 
                                     int suffix_n, int* out_slot, int* out_cnt, int out_ld,
                                     float* out_score, void* ws, void* stream);
 
+/* a1 + a2 fused, the trainable path's lists -- the masks of chunk-wise training with the dynamic
+ * sparse cache (English 2.D "Training Strategy": the model is trained with the same sparse cache
+ * it uses at inference).  Sequences of seq_frames frames are folded into the frame axis
+ * (q_frames = n_seq * seq_frames) and cut into chunks of chunk_frames frames (the last chunk of a
+ * sequence may be shorter).  The pool holds every sequence's blocks in order: the slot of a block
+ * is its global block id (pbsa_blockify / pbsa_blockify_kv with dst_slot = NULL), so k_reps are
+ * the keys' representatives.  For query block r of sequence s (blocks [s0, s0 + seq_frames*bpf)),
+ * chunk c (blocks [cs, ce)):
+ *   c == 0:  out_slot[h][r] = cs .. ce-1                                (its own chunk)
+ *   c >= 1:  out_slot[h][r] = s0 .. s0+S-1                              (the sinks, S = sink_frames*bpf)
+ *                           + the k best of s0+S .. cs-1 by scale * <q_reps[h][r], k_reps[h][slot]>
+ *                             (score descending, ties to the lower slot), best first
+ *                           + cs .. ce-1                                (its own chunk)
+ *   out_cnt[h][r] = the row's length; out_score[h][r][i] (nullable) = the i-th selected score.
+ * q_reps[h][r] = mean of query block r's 64 tokens (bit-identical to pbsa_blockify).
+ *  q       [q_frames*frame_h*frame_w][H][d] raster, geometry dtype (16-byte aligned).
+ *  q_reps  out [H][q_frames*bpf][d] fp32;  k_reps [H][pool_slots][d] fp32, pool_slots >= q_frames*bpf.
+ *  out_slot out [H][q_frames*bpf][out_ld], out_ld >= S + k + min(chunk_frames, seq_frames)*bpf;
+ *  out_cnt  out [H][q_frames*bpf];  out_score nullable out [H][q_frames*bpf][k].
+ *  0 <= sink_frames <= chunk_frames (the sinks lie in chunk 0); q_frames a multiple of seq_frames.
+ *  At most 1024 candidates in a sequence's last chunk, else PBSA_ERR_UNSUPPORTED. */
+PBSA_API pbsa_status pbsa_blockify_train_select(const pbsa_geom* g, const void* q, int q_frames,
+                                       float* q_reps, const float* k_reps, int pool_slots,
+                                       int seq_frames, int chunk_frames, int sink_frames, int k,
+                                       int* out_slot, int* out_cnt, int out_ld, float* out_score,
+                                       void* ws, void* stream);
+
 /* a3 -- fine attention over the selected blocks (the hybrid mask of the Chinese
  * explainer 2.2 "掩码机制"; English 2.C "Global Access" + "Local Sparsity"):
  * for every token i of query block r of head h,
@@ -296,8 +323,6 @@ PBSA_API pbsa_status pbsa_memory_update_noalloc(const pbsa_geom* g, const float*
                                                 const int* cand_gid, int ncand, float gamma,
                                                 int* p_list, int* p_cnt, void* stream);
 
-/* Synchronises `stream`, reads and clears the workspace's device error word, and returns
- * it (PBSA_OK when clean). */
 /* Self-test of the bounded waits (the paper has no counterpart).  Every kernel that waits on an
  * mbarrier gives up after a time limit, records PBSA_ERR_TIMEOUT in the workspace's error word
  * and returns instead of hanging.  This launches one thread that waits, with that same code, on
@@ -306,6 +331,8 @@ PBSA_API pbsa_status pbsa_memory_update_noalloc(const pbsa_geom* g, const float*
  *  ws: a workspace whose first 256 bytes are the error word. */
 PBSA_API pbsa_status pbsa_selftest_wait_timeout(void* ws, unsigned int limit_us, void* stream);
 
+/* Synchronises `stream`, reads and clears the workspace's device error word, and returns
+ * it (PBSA_OK when clean). */
 PBSA_API pbsa_status pbsa_get_device_error(void* ws, void* stream);
 
 /* Static description of a status code. */

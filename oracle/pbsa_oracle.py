@@ -352,6 +352,7 @@ class RolloutOracle:
         self.P = [dict() for _ in range(heads)]
         self.kreps = {}            # gid -> [H, d]
         self.last_gap = []
+        self.last_pool_ema = []    # per head: {gid: EMA} of every pool entry of the last update
 
     def local(self) -> list[int]:
         return frame_blocks(window_frames(self.hist, self.W), self.bpf)
@@ -388,6 +389,7 @@ class RolloutOracle:
         evicted = frame_blocks((old_win | entering) - new_win, self.bpf)
         new_sinks = frame_blocks([0], self.bpf) if first_frame == 0 else []
         self.last_gap = []
+        self.last_pool_ema = []
         for h in range(self.H):
             pool = sorted(self.P[h]) + new_sinks + evicted
             prev = [self.P[h].get(g, np.nan) for g in pool]
@@ -397,6 +399,7 @@ class RolloutOracle:
                                          self.geom["scale"], self.gamma, self.C)
             self.P[h] = {g: float(e) for g, e, kp in zip(pool, ema, keep) if kp}
             self.last_gap.append(ema_boundary_gap(ema, pool, sink, self.C))
+            self.last_pool_ema.append({g: float(e) for g, e in zip(pool, ema)})
         self.hist = new_hist
         return evicted
 

@@ -157,6 +157,19 @@ def test_every_entry_point_checks_its_arguments_on_the_host(lib):
     assert L.pbsa_blockify_hsa_select(gp, f, 3, f, f, 400, f, f, 144, -1, 1, 32, f, f, 96, f, f, 128, None, f,
                                       None) == 1
 
+    # trainable-path lists: gp, q, q_frames, q_reps, k_reps, pool, seq_frames, chunk_frames, sink_frames,
+    # k, out_slot, out_cnt, out_ld, out_score, ws, stream (18 frames = 2 sequences of 9, 432 blocks)
+    def ts(qf=18, pool=432, seq=9, chunk=3, sink=1, k=16, out_ld=112, q=f):
+        return L.pbsa_blockify_train_select(gp, q, qf, f, f, pool, seq, chunk, sink, k, f, f, out_ld, None, f, None)
+    assert ts(qf=17) == 1                     # not a whole number of sequences
+    assert ts(pool=431) == 1                  # slot = block id needs every block in the pool
+    assert ts(sink=4) == 1                    # sinks beyond the first chunk
+    assert ts(sink=-1) == 1
+    assert ts(out_ld=111) == 1                # 24 sinks + 16 + 72 own
+    assert ts(k=-1) == 1
+    assert ts(q=m) == 1
+    assert ts(qf=48, seq=48, pool=1152) == 2  # last chunk: 44 earlier non-sink frames = 1056 candidates
+
     # attention: gp, q, q_frames, k_pool, v_pool, pool, kv_slot, kv_cnt, kv_ld, o, lse, ws, stream
     def at(geom=gp, qf=3, pool=400, ld=128, o=f):
         return L.pbsa_attend(geom, f, qf, f, f, pool, f, f, ld, o, None, f, None)

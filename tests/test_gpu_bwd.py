@@ -1,5 +1,7 @@
 """GPU parity of the backward pass (pbsa_attend_bwd) against the oracle's textbook
-gradients, under fixed seeded block lists with the structure of the trainable path."""
+gradients, under fixed seeded block lists with the structure of the trainable path (random
+selections: structural cases such as odd query-block pairs and unattended slots).  The
+trainable-path workload under the method's own masks is in test_gpu_train.py."""
 import dataclasses
 
 import numpy as np
@@ -98,32 +100,3 @@ def test_bwd_small(fh, fw, frames, batch, topk, extra):
         _rel_close(f64(dv[h]), want_dv, f"dv h{h}")
         if extra:
             assert (dk[h, nq:] == 0).all() and (dv[h, nq:] == 0).all()
-
-
-@pytest.mark.slow
-def test_bwd_train_workload_sampled():
-    """The trainable-path shapes (batch 2 x 9 frames x 1536 tokens, 12 heads): dQ on sampled
-    query blocks, dK/dV on sampled slots (every query block that attends them)."""
-    w = I.TRAIN_FWD_BWD
-    frames, batch = w.total_frames, w.batch
-    q, k, v, do, lists, kv, cnt, ld, slots = _setup(w, frames, batch, 0, seed=4)
-    q_frames = batch * frames
-    dq, dk, dv = _gpu(w, q, k, v, do, kv, cnt, ld, slots, q_frames)
-    q64, k64, v64, do64 = (f64(t) for t in (q, k, v, do))
-    bpf, nq = w.blocks_per_frame, q_frames * w.blocks_per_frame
-    rng = np.random.default_rng(0)
-    for h in (0, 7):
-        for r in rng.choice(nq, 4, replace=False).tolist() + [0, nq - 1]:
-            rows, gq, _, _ = _oracle_unit(w, q64, k64, v64, do64, h, r, lists[h][r])
-            _rel_close(f64(dq[rows, h]), gq, f"dq h{h} r{r}")
-        for s in (5 * bpf + 3, frames * bpf + 2):   # an own-chunk block of chunk 1, a sink of batch 1
-            want_dk = np.zeros((64, w.head_dim))
-            want_dv = np.zeros((64, w.head_dim))
-            for r in range(nq):
-                if s in lists[h][r]:
-                    _, _, gk, gv = _oracle_unit(w, q64, k64, v64, do64, h, r, lists[h][r])
-                    i = lists[h][r].index(s)
-                    want_dk += gk[i * 64:(i + 1) * 64]
-                    want_dv += gv[i * 64:(i + 1) * 64]
-            _rel_close(f64(dk[h, s]), want_dk, f"dk h{h} s{s}")
-            _rel_close(f64(dv[h, s]), want_dv, f"dv h{h} s{s}")
