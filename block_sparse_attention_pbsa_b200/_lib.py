@@ -71,6 +71,7 @@ _SIGS = {
     "pbsa_memory_update_apply": (_I, [ctypes.POINTER(Geom), _P, _P, _P, _I, _I, _I, _P, _P]),
     "pbsa_memory_update_noalloc": (_I, [ctypes.POINTER(Geom), _P, _I, _P, _P, _P, _I, _P, _P, _I, _I,
                                         _P, _P, _I, ctypes.c_float, _P, _P, _P]),
+    "pbsa_memory_update_noalloc_error": (_I, [_P]),
     "pbsa_get_device_error": (_I, [_P, _P]),
     "pbsa_selftest_wait_timeout": (_I, [_P, ctypes.c_uint, _P]),
     "pbsa_status_string": (ctypes.c_char_p, [_I]),
@@ -263,6 +264,11 @@ def pbsa_memory_update_noalloc(g: Geom, q_reps, nq, k_reps, k_pool, v_pool, pool
         n_sink_gid, _ptr(cand_slot, torch.int32, "cand_slot"), _ptr(cand_gid, torch.int32, "cand_gid"),
         ncand, float(gamma), _ptr(p_list, torch.int32, "p_list"), _ptr(p_cnt, torch.int32, "p_cnt"),
         _stream(stream)))
+
+
+def pbsa_memory_update_noalloc_error(stream=None) -> int:
+    """Read and clear the error word of pbsa_memory_update_noalloc's built-in scratch."""
+    return int(load().pbsa_memory_update_noalloc_error(_stream(stream)))
 
 
 def pbsa_bwd_workspace_bytes(g: Geom, q_frames: int, pool_slots: int, kv_ld: int) -> int:

@@ -19,7 +19,8 @@
 // scratch byte they read.  Two calls whose work overlaps on
 // the GPU (different streams, or the same stream from two threads without ordering)
 // race on the array.  Device-side index errors found by this variant are recorded in
-// the scratch and not reported to the caller.
+// the scratch's error word; pbsa_memory_update_noalloc_error reads and clears it (the
+// next call of the update clears it too, so read it in between).
 #include <mutex>
 
 #include "common.cuh"
@@ -72,4 +73,10 @@ extern "C" pbsa_status pbsa_memory_update_noalloc(const pbsa_geom* g, const floa
   return pbsa_memory_update(g, q_reps, nq, k_reps, k_pool, v_pool, pool_slots, slot_gid, slot_ema,
                             capacity, n_sink_gid, cand_slot, cand_gid, ncand, gamma, p_list, p_cnt,
                             ws, stream);
+}
+
+extern "C" pbsa_status pbsa_memory_update_noalloc_error(void* stream) {
+  void* ws = nullptr;
+  if (pbsa::noalloc_scratch(&ws) != cudaSuccess) return PBSA_ERR_CUDA;
+  return pbsa_get_device_error(ws, stream);
 }

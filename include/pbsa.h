@@ -314,7 +314,8 @@ PBSA_API pbsa_status pbsa_memory_update_apply(const pbsa_geom* g, float* k_reps,
  *    (cudaGetSymbolAddress); make that first call before any stream capture.
  *  - Sharing: every call uses the same scratch, which keeps the last call's contents;
  *    calls whose work overlaps on the GPU race.  Device-side index errors are recorded in
- *    the scratch and not reported.
+ *    the scratch's error word, which each call clears when it starts: read it with
+ *    pbsa_memory_update_noalloc_error before the next call.
  *  - Allocates nothing (no cudaMalloc or allocating library call). */
 PBSA_API pbsa_status pbsa_memory_update_noalloc(const pbsa_geom* g, const float* q_reps, int nq,
                                                 float* k_reps, void* k_pool, void* v_pool,
@@ -330,6 +331,15 @@ PBSA_API pbsa_status pbsa_memory_update_noalloc(const pbsa_geom* g, const float*
  * pbsa_get_device_error(ws) reports PBSA_ERR_TIMEOUT and the context remains usable.
  *  ws: a workspace whose first 256 bytes are the error word. */
 PBSA_API pbsa_status pbsa_selftest_wait_timeout(void* ws, unsigned int limit_us, void* stream);
+
+/* The device error word of pbsa_memory_update_noalloc's built-in scratch, for its callers,
+ * who hold no workspace to pass to pbsa_get_device_error (the paper has no counterpart).
+ * Synchronises `stream`, reads and clears the word and returns it (PBSA_OK when clean):
+ * PBSA_ERR_DEVICE_INDEX when the last update on this device met a candidate slot outside the
+ * pool (that candidate was left out), PBSA_ERR_TIMEOUT when a bounded wait expired.  Runs on
+ * the current device; the first use on a device looks up the scratch's address, like the
+ * update's own first call. */
+PBSA_API pbsa_status pbsa_memory_update_noalloc_error(void* stream);
 
 /* Synchronises `stream`, reads and clears the workspace's device error word, and returns
  * it (PBSA_OK when clean). */

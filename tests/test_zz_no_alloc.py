@@ -65,6 +65,7 @@ def test_noalloc_matches_workspace_update_twice(ncand):
                                      lists["b"][0], lists["b"][1])
         torch.cuda.synchronize()
         assert P.pbsa_get_device_error(ws) == 0
+        assert P.pbsa_memory_update_noalloc_error() == 0
         assert torch.equal(a[3], b[3]), f"call {call}: persistent sets differ"
         assert (a[3] >= 0).sum() > S, "the update promoted nothing; the check would be vacuous"
         torch.testing.assert_close(a[4], b[4], rtol=2e-5, atol=1e-9)
@@ -91,3 +92,31 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
         P.pbsa_memory_update_noalloc(g, qr, nq, kr, kp, kp, C + ncand, sgid, sema, C, 24, cs, cs,
                                      ncand, 0.9)
     assert e.value.code == 2
+
+
+def test_noalloc_reports_a_bad_candidate_slot_through_its_error_query():
+    """Callers of the scratch-free update hold no workspace, so its device error word is read
+    with pbsa_memory_update_noalloc_error: a candidate whose slot lies outside the pool is
+    reported (PBSA_ERR_DEVICE_INDEX) and left out, like the workspace update does, and reading
+    the word clears it.  The result equals the workspace update's on the same inputs."""
+    H, d, nq, C, S, ncand = 2, 128, 24, 16, 4, 12
+    w = dataclasses.replace(I.DECODE_5S, heads=H)
+    g = P.make_geom(H, d, w.frame_h, w.frame_w, w.tile_h, w.tile_w, w.scale, "bf16")
+    pool = C + ncand + 4
+    a = _state(7, H, C, S, pool, d)
+    b = [t.clone() for t in a]
+    cs = (torch.arange(ncand, dtype=torch.int32) + C).repeat(H, 1)
+    cs[1, 5] = pool + 9                               # out of range: checked and skipped on the device
+    cg = (torch.arange(ncand, dtype=torch.int32) + 500).repeat(H, 1)
+    cs, cg = cs.to(DEV), cg.to(DEV)
+    qr = (torch.randn((H, nq, d), generator=torch.Generator().manual_seed(8)) * 0.3).to(DEV)
+    ws = torch.zeros(P.pbsa_workspace_bytes(g, nq, C + ncand), dtype=torch.uint8, device=DEV)
+    kr, kp, vp, sgid, sema = a
+    P.pbsa_memory_update(g, qr, nq, kr, kp, vp, pool, sgid, sema, C, S, cs, cg, ncand, 0.9, ws=ws)
+    kr, kp, vp, sgid, sema = b
+    P.pbsa_memory_update_noalloc(g, qr, nq, kr, kp, vp, pool, sgid, sema, C, S, cs, cg, ncand, 0.9)
+    assert P.pbsa_get_device_error(ws) == 5
+    assert P.pbsa_memory_update_noalloc_error() == 5
+    assert P.pbsa_memory_update_noalloc_error() == 0       # read once, cleared
+    assert torch.equal(a[3], b[3]) and 505 not in b[3][1].tolist()
+    torch.testing.assert_close(a[4], b[4], rtol=2e-5, atol=1e-9)
