@@ -522,6 +522,14 @@ def max_over_ranks(x: float, device, world: int) -> float:
     return float(t.item())
 
 
+def sum_over_ranks(x: float, device, world: int) -> float:
+    """The whole job's total of a per-rank quantity (e.g. the FLOPs of one step)."""
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item())
+
+
 def _check_device(P, ws, when: str):
     """Raise with the workspace's device error word (code, info, kernel id) if one is set."""
     torch.cuda.synchronize()
@@ -537,7 +545,10 @@ def run_pbsa(args, w, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     peaks = load_peaks()
-    wr = rank_workload(w, rank)
+    heads_split = args.shard == "heads" and world > 1
+    # weak scaling: every rank its own independent layer; head split (strong scaling): the one
+    # layer's heads partitioned over the ranks, each rank its heads' cache and inputs
+    wr = w if heads_split else rank_workload(w, rank)
     q, k, v = I.single_step(wr)
     kc = I.tokens(wr, wr.chunk_frames, I.stream_seed(wr.seed, 4))
     vc = I.tokens(wr, wr.chunk_frames, I.stream_seed(wr.seed, 5))
@@ -545,6 +556,10 @@ def run_pbsa(args, w, rank, world, local_rank):
     cfg = P.LayerConfig(w.heads, w.head_dim, w.frame_h, w.frame_w, w.tile_h, w.tile_w, w.capacity,
                         w.window_frames, w.chunk_frames, w.topk, w.gamma, w.dtype,
                         (w.hist_frames - w.window_frames) * bpf)
+    if heads_split:
+        from block_sparse_attention_pbsa_b200 import shard
+        q, k, v, kc, vc = (shard.head_slice(t, w.heads, world, rank) for t in (q, k, v, kc, vc))
+        cfg = shard.local_config(cfg, world, rank)
     torch.cuda.synchronize(dev)
     alloc0 = torch.cuda.memory_allocated(dev)
     cache = P.PBSALayerCache(cfg, dev)
@@ -623,7 +638,7 @@ def run_pbsa(args, w, rank, world, local_rank):
     qh, kh, vh = (t.pin_memory() for t in (q, kc, vc))
     oh = torch.empty(q.shape, dtype=q.dtype).pin_memory()
     step.restore(snap)
-    step.capture_pipeline(qd, kcd, vcd, o)
+    step.capture_pipeline(qd, kcd, vcd, o, qh, kh, vh, oh)
     e2e_ms = []
     for s in range(max(1, args.steps // 2) + 1):
         step.restore(snap)
@@ -638,6 +653,7 @@ def run_pbsa(args, w, rank, world, local_rank):
     if not torch.equal(oh, o.cpu()):
         raise RuntimeError("the pipelined end-to-end step returned a different O")
     e2e_ms_max = max_over_ranks(statistics.mean(e2e_ms), dev, world)
+    job_flops = sum_over_ranks(flops, dev, world)    # every rank's layer, or the shared layer's heads
 
     if rank != 0:
         return
@@ -648,15 +664,17 @@ def run_pbsa(args, w, rank, world, local_rank):
                            "frac_hbm": b / (per[g] * 1e-3) / 1e9 / peaks["hbm_gbs"]})
     att_tflops = flops / (per["attend"] * 1e-3) / 1e12
     kernels["attend"].update({"flops": flops, "achieved_tflops": att_tflops})
-    value = world * flops / (step_ms_max * 1e-3) / 1e12
+    value = job_flops / (step_ms_max * 1e-3) / 1e12
     h2d = sum(t.numel() * t.element_size() for t in (q, kc, vc))
     d2h = o.numel() * o.element_size()
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": max(args.warmup, 3), "ms_per_step": step_ms_max, "ms_per_chunk_decode": step_ms_max,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic", "config": {**workload_config(w),
-                                        "parallelism": f"{world} independent layer decodes (one per GPU)"},
+        "higher_is_better": True, "scaling": "strong" if heads_split else "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {**workload_config(w),
+                   "parallelism": (f"the layer's {w.heads} heads split over {world} GPUs (no exchange in the step)"
+                                   if heads_split else f"{world} independent layer decodes (one per GPU)")},
         "roofline": {"bound": "tensor", "kernel": "pbsa_attend (attend_tc_kernel)", "achieved": att_tflops,
                      "peak": peaks["bf16"], "unit": "TFLOP/s", "frac": att_tflops / peaks["bf16"],
                      "peak_source": f"{peaks['source']} burst bf16 (cuBLAS)",
@@ -674,7 +692,7 @@ def run_pbsa(args, w, rank, world, local_rank):
                            "note": "measured = torch.cuda.memory_allocated() around the cache's construction: "
                                    "K/V pools, key representatives, slot tables, lists, workspace; the staging "
                                    "area only serves the one-time prefill of a mid-video history"},
-        "e2e": {"value": world * flops / (e2e_ms_max * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "e2e": {"value": job_flops / (e2e_ms_max * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "ms_per_step": e2e_ms_max, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": step.LAUNCHES * args.steps,
         "clocks": clk.summary(),
@@ -709,6 +727,9 @@ def main():
     ap.add_argument("--no-train", action="store_true", help="skip the forward+backward training workload")
     ap.add_argument("--train-only", action="store_true", help="only the training workload (for profiling)")
     ap.add_argument("--no-rollout", action="store_true", help="skip the 30-layer 5 s and 1-minute rollouts")
+    ap.add_argument("--shard", choices=["layers", "heads"], default="layers",
+                    help="N > 1: every rank its own layer (weak scaling, the default) or one layer's heads "
+                         "split over the ranks (strong scaling)")
     args = ap.parse_args()
     from block_sparse_attention_pbsa_b200 import inputs as I
     w = I.DECODE_5S

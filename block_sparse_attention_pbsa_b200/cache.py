@@ -489,24 +489,30 @@ class ChunkDecodeStep:
         torch.cuda.current_stream(self.cache.device).wait_stream(side)
         return graph
 
-    def capture_pipeline(self, q, k, v, o, lse=None, parts=None):
-        """Capture the step for ``run_pipelined`` as ``parts`` front graphs (default: one per
-        frame of the chunk), each [blockify(Q) + selection + attend] of its frames, then
-        [memory update] and [commit blockify(K, V)].
+    def capture_pipeline(self, q, k, v, o, qh, kh, vh, oh, parts=None):
+        """Capture one end-to-end step, transfers included, as one CUDA graph for
+        ``run_pipelined``: pinned host Q, K, V (``qh``, ``kh``, ``vh``) -> the device buffers
+        ``q``, ``k``, ``v`` -> the step -> O (``o``) -> pinned host ``oh``.
 
-        Q arrives frame by frame in raster order, so the first frames' selection and attention
-        run while the later frames (and K, V) are still uploading, and their O rows download
-        while the later frames compute.  The memory update takes the representatives of the
-        whole chunk, which it recomputes from the resident Q (the same kernel and order as the
-        fused selection's, so the same bits); it reads neither K nor V of the chunk (its
-        candidates are blocks leaving the window, never the chunk's ring positions), so it runs
-        while they upload, and only the commit waits for them.  Every query block's selection and
-        attention are independent of the others', so the results equal ``run``'s bit for bit.
-        (The own-chunk variant, which needs K, V before the selection, is not split.)"""
+        Q goes up first, then K and V, on one copy stream; [blockify(Q) + selection + attend]
+        starts as soon as Q has landed, and O goes down on a second copy stream as soon as it is
+        computed.  The memory update reads neither K nor V of the chunk (its candidates are
+        blocks leaving the window, never the chunk's ring positions), so it runs while they
+        upload, and only the commit waits for them.  With ``parts`` > 1, Q goes up in that many
+        slices of whole frames, each followed by the selection and attention of its frames, and
+        the memory update recomputes the chunk's representatives from the resident Q (the same
+        kernel and order as the fused selection's, so the same bits).  Every query block's
+        selection and attention are independent of the others', so the results equal ``run``'s
+        bit for bit.  The graph holds the host buffers' addresses: ``run_pipelined`` takes the
+        same four buffers.  (The own-chunk variant, which needs K, V before the selection, is
+        not split.)"""
         if self.cache.cfg.own_chunk:
             raise ValueError("the own-chunk variant writes K, V before the selection: use capture()")
+        for t in (qh, kh, vh, oh):
+            if t.is_cuda or not t.is_pinned():
+                raise ValueError("the host buffers must be pinned CPU tensors")
         ca, c = self.cache, self.cache.cfg
-        parts = parts or self.q_frames
+        parts = parts or 1
         if self.q_frames % parts:
             raise ValueError(f"{self.q_frames} frames do not split into {parts} equal parts")
         fpp = self.q_frames // parts                 # frames per part
@@ -514,77 +520,61 @@ class ChunkDecodeStep:
         dev = ca.device
         g, ws, ps = ca.geom, ca.ws, ca.pool_slots
         H = c.heads
-        side = torch.cuda.Stream(device=dev)
-        side.wait_stream(torch.cuda.current_stream(dev))
-        fronts, part_bufs = [], []
-        for p in range(parts):
-            qp, op = q[p * rows:(p + 1) * rows], o[p * rows:(p + 1) * rows]
-            lp = lse[:, p * rows:(p + 1) * rows].contiguous() if lse is not None else None
-            bufs = (torch.zeros((H, nqp, c.head_dim), dtype=torch.float32, device=dev),
-                    torch.zeros((H, nqp, ca.kv_ld), dtype=torch.int32, device=dev),
-                    torch.zeros((H, nqp), dtype=torch.int32, device=dev), lp)
-            part_bufs.append(bufs)
-            gr = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(gr, stream=side):
-                ca._select_fused(qp, fpp, bufs[0], bufs[1], bufs[2], ca.kv_ld)
-                L.pbsa_attend(g, qp, fpp, ca.k_pool, ca.v_pool, ps, bufs[1], bufs[2], ca.kv_ld, op, lp, ws=ws)
-            fronts.append(gr)
-        mid, back = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-        with torch.cuda.graph(mid, stream=side):   # the kernels of run(): the same results, bit for bit
-            L.pbsa_blockify(g, q, self.q_frames, self.q_reps, self.nq, ws=ws)
+        if parts == 1:   # the step's own buffers: the same kernels as run()
+            part_bufs = [(self.q_reps, self.kv_slot, self.kv_cnt)]
+        else:
+            part_bufs = [(torch.zeros((H, nqp, c.head_dim), dtype=torch.float32, device=dev),
+                          torch.zeros((H, nqp, ca.kv_ld), dtype=torch.int32, device=dev),
+                          torch.zeros((H, nqp), dtype=torch.int32, device=dev)) for _ in range(parts)]
+        main, h2d, d2h = (torch.cuda.Stream(device=dev) for _ in range(3))
+        main.wait_stream(torch.cuda.current_stream(dev))
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=main):
+            h2d.wait_stream(main)
+            d2h.wait_stream(main)
+            landed = []
+            with torch.cuda.stream(h2d):
+                for i in range(parts):
+                    q[i * rows:(i + 1) * rows].copy_(qh[i * rows:(i + 1) * rows], non_blocking=True)
+                    ev = torch.cuda.Event()
+                    ev.record(h2d)
+                    landed.append(ev)
+                k.copy_(kh, non_blocking=True)
+                v.copy_(vh, non_blocking=True)
+            for i, (qr, kv, cnt) in enumerate(part_bufs):
+                main.wait_event(landed[i])
+                qp, op = q[i * rows:(i + 1) * rows], o[i * rows:(i + 1) * rows]
+                ca._select_fused(qp, fpp, qr, kv, cnt, ca.kv_ld)
+                L.pbsa_attend(g, qp, fpp, ca.k_pool, ca.v_pool, ps, kv, cnt, ca.kv_ld, op, None, ws=ws)
+                done = torch.cuda.Event()
+                done.record(main)
+                d2h.wait_event(done)
+                with torch.cuda.stream(d2h):
+                    oh[i * rows:(i + 1) * rows].copy_(op, non_blocking=True)
+            # the memory update: the same kernels as run(), the same results bit for bit
+            if parts > 1:
+                L.pbsa_blockify(g, q, self.q_frames, self.q_reps, self.nq, ws=ws)
             L.pbsa_memory_update_plan(g, self.q_reps, self.nq, ca.k_reps, ps, ca.slot_gid, ca.slot_ema, c.capacity,
                                       c.bpf, self.cs, self.cg, self.ncand, c.gamma, ca.p_list, ca.p_cnt, ws=ws)
             L.pbsa_memory_update_apply(g, ca.k_reps, ca.k_pool, ca.v_pool, ps, c.capacity, self.ncand, ws=ws)
-        with torch.cuda.graph(back, stream=side):
+            main.wait_stream(h2d)                   # K, V uploaded
             L.pbsa_blockify_kv(g, k, v, self.q_frames, ca.k_reps, None, ps, self.dst, ca.k_pool, ca.v_pool, ps,
                                ws=ws)
-        torch.cuda.current_stream(dev).wait_stream(side)
-        self._pipe = {"fronts": fronts, "mid": mid, "back": back, "bufs": (q, k, v, o), "rows": rows,
-                      "part_bufs": part_bufs, "lse": lse,
-                      "h2d": torch.cuda.Stream(device=dev), "d2h": torch.cuda.Stream(device=dev)}
-        # launches per pipelined step: per part the fused selection and attend; blockify(Q), plan,
+            main.wait_stream(d2h)                   # O downloaded
+        torch.cuda.current_stream(dev).wait_stream(main)
+        self._pipe = {"graph": graph, "host": (qh, kh, vh, oh), "bufs": part_bufs}
+        # launches per pipelined step: per part the fused selection and attend; [blockify(Q)], plan,
         # apply; the commit
-        self.PIPELINED_LAUNCHES = 2 * parts + 3 + 1
+        self.PIPELINED_LAUNCHES = 2 * parts + (3 if parts > 1 else 2) + 1
 
     def run_pipelined(self, qh, kh, vh, oh):
-        """One step from pinned host buffers to a pinned host result, with the transfers
-        overlapped: Q is uploaded part by part (frames in raster order) and each part's front
-        graph (selection + attention) starts as soon as its rows land, while the later parts and
-        then K and V upload on a copy stream; each part's O rows download on another stream as
-        soon as they are computed; the memory update runs while K and V upload, and the commit
-        of K and V follows their upload.  All work is ordered on the current stream's timeline
-        when this returns (asynchronously)."""
+        """One step from the pinned host buffers given to ``capture_pipeline`` to the pinned
+        host result, with the transfers overlapped with the kernels: one graph launch on the
+        current stream (asynchronous; ``oh`` holds O once the stream reaches this point)."""
         p = self._pipe
-        q, k, v, o = p["bufs"]
-        rows = p["rows"]
-        main = torch.cuda.current_stream(self.cache.device)
-        h2d, d2h = p["h2d"], p["d2h"]
-        h2d.wait_stream(main)                       # previous step done with k, v, q
-        d2h.wait_stream(main)
-        landed = []
-        with torch.cuda.stream(h2d):
-            for i in range(len(p["fronts"])):
-                q[i * rows:(i + 1) * rows].copy_(qh[i * rows:(i + 1) * rows], non_blocking=True)
-                ev = torch.cuda.Event()
-                ev.record(h2d)
-                landed.append(ev)
-            k.copy_(kh, non_blocking=True)
-            v.copy_(vh, non_blocking=True)
-        for i, gr in enumerate(p["fronts"]):
-            main.wait_event(landed[i])
-            gr.replay()
-            done = torch.cuda.Event()
-            done.record(main)
-            with torch.cuda.stream(d2h):
-                d2h.wait_event(done)
-                oh[i * rows:(i + 1) * rows].copy_(o[i * rows:(i + 1) * rows], non_blocking=True)
-        p["mid"].replay()                           # memory update (needs no K, V)
-        main.wait_stream(h2d)                       # K, V uploaded
-        p["back"].replay()
-        main.wait_stream(d2h)                       # O downloaded
-        if p["lse"] is not None:
-            for i, b in enumerate(p["part_bufs"]):
-                p["lse"][:, i * rows:(i + 1) * rows].copy_(b[3])
+        if any(a.data_ptr() != b.data_ptr() for a, b in zip((qh, kh, vh, oh), p["host"])):
+            raise ValueError("run_pipelined takes the host buffers the step was captured with")
+        p["graph"].replay()
         return oh
 
     def snapshot(self):

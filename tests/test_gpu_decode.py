@@ -334,9 +334,10 @@ def test_chunk_decode_step_needs_a_history():
 
 
 def test_pipelined_host_step_matches_the_graph_step():
-    """ChunkDecodeStep.run_pipelined (transfers overlapped with the kernels, the memory update
-    ahead of the commit of K and V) gives the same O and the same cache, bit for bit, as the
-    single-graph step on the same inputs."""
+    """ChunkDecodeStep.run_pipelined (one graph with the transfers: the selection and attention
+    behind the upload of Q, as a whole or frame by frame, O downloaded behind them, the memory
+    update ahead of the commit of K and V) gives the same O and the same cache, bit for bit,
+    as the single-graph step on the same inputs."""
     w = I.DECODE_5S
     q, k, v = I.single_step(w)
     kc = I.tokens(w, w.chunk_frames, I.stream_seed(w.seed, 4))
@@ -354,14 +355,47 @@ def test_pipelined_host_step_matches_the_graph_step():
     want = [getattr(cache, n).cpu() for n in names]
     step.restore(snap)
     qb, kb, vb, ob = (torch.empty_like(t) for t in (qd, kcd, vcd, o))
-    step.capture_pipeline(qb, kb, vb, ob)
     qh, kh, vh = (t.pin_memory() for t in (q, kc, vc))
     oh = torch.empty(q.shape, dtype=q.dtype).pin_memory()
-    for _ in range(2):
+    for parts in (1, 3):
         step.restore(snap)
-        step.run_pipelined(qh, kh, vh, oh)
-        torch.cuda.synchronize()
-        assert torch.equal(oh, want_o)
-        for n, t in zip(names, want):
-            assert torch.equal(getattr(cache, n).cpu(), t), n
+        step.capture_pipeline(qb, kb, vb, ob, qh, kh, vh, oh, parts=parts)
+        for _ in range(2):
+            step.restore(snap)
+            oh.zero_()
+            step.run_pipelined(qh, kh, vh, oh)
+            torch.cuda.synchronize()
+            assert torch.equal(oh, want_o), parts
+            for n, t in zip(names, want):
+                assert torch.equal(getattr(cache, n).cpu(), t), (parts, n)
     assert P.pbsa_get_device_error(cache.ws) == 0
+
+
+@pytest.mark.parametrize("world", [3, 5])
+def test_head_sharded_caches_match_the_whole_layer(world):
+    """The layer split by heads over ``world`` ranks (each rank its heads' cache, inputs and
+    kernels; here the ranks run one after another on one GPU, with no waits between them):
+    over five chunks of the 5 s rollout the ranks' outputs and caches equal the whole layer's
+    heads, bit for bit."""
+    from block_sparse_attention_pbsa_b200 import shard
+    w = I.ROLLOUT_5S
+    full = P.PBSALayerCache(layer_cfg(w))
+    parts = [P.PBSALayerCache(shard.local_config(layer_cfg(w), world, r)) for r in range(world)]
+    for c, (f0, nf) in enumerate(I.rollout_chunks(w)[:5]):
+        wc = dataclasses.replace(w, chunk_frames=nf)
+        for s in range(2):
+            q, k, v = (I.tokens(wc, nf, I.stream_seed(w.seed, c, s, t)).to(DEV) for t in range(3))
+            o = full.decode_step(q, k, v)
+            for r, ca in enumerate(parts):
+                h0, h1 = shard.head_range(w.heads, world, r)
+                qs, ks, vs = (shard.head_slice(t, w.heads, world, r) for t in (q, k, v))
+                assert torch.equal(ca.decode_step(qs, ks, vs), o[:, h0:h1]), (c, s, r)
+                if s == 1:
+                    ca.commit(ks, vs)
+            if s == 1:
+                full.commit(k, v)
+        for r, ca in enumerate(parts):
+            h0, h1 = shard.head_range(w.heads, world, r)
+            for name in ("slot_gid", "slot_ema", "k_pool", "v_pool", "k_reps", "p_list", "p_cnt"):
+                assert torch.equal(getattr(ca, name), getattr(full, name)[h0:h1]), (c, r, name)
+            assert P.pbsa_get_device_error(ca.ws) == 0
