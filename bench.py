@@ -254,11 +254,13 @@ def run_train(P, I, dev, steps: int, peaks):
     bwd_flops = 2.5 * fwd_flops
     sm, fm, bm = statistics.mean(sel_ms), statistics.mean(fwd_ms), statistics.mean(bwd_ms)
     sel_bytes = q.numel() * 2 + q_reps.numel() * 4 + k_reps.numel() * 4 + kv.numel() * 4
+    sel_floor = same_bytes_copy_ms(dev, sel_bytes, flush)
     return {"workload": w.name, "query_blocks": nq, "heads": w.heads, "steps": steps,
             "masks": "24 sinks + top-16 by coarse score among the earlier non-sink blocks + own chunk "
                      "(pbsa_blockify_train_select)",
             "select_ms": sm, "select_algorithmic_bytes": sel_bytes,
             "select_frac_hbm": sel_bytes / (sm * 1e-3) / 1e9 / peaks["hbm_gbs"],
+            "select_same_bytes_copy_ms": sel_floor, "select_frac_of_same_bytes_copy": sel_floor / sm,
             "fwd_ms": fm, "bwd_ms": bm, "fwd_flops": fwd_flops, "bwd_flops": bwd_flops,
             "fwd_tflops": fwd_flops / (fm * 1e-3) / 1e12, "bwd_tflops": bwd_flops / (bm * 1e-3) / 1e12,
             "fwd_frac_of_bf16_peak": fwd_flops / (fm * 1e-3) / 1e12 / peaks["bf16"],
@@ -522,6 +524,26 @@ def max_over_ranks(x: float, device, world: int) -> float:
     return float(t.item())
 
 
+def same_bytes_copy_ms(dev, nbytes: int, flush, reps: int = 10) -> float:
+    """Device time of a plain device-to-device copy that moves ``nbytes`` (half read, half
+    written), L2 flushed before each: the floor, at this size, that launch and first-byte
+    latency leave for any kernel moving the same bytes.  Median of ``reps``."""
+    half = max(16, (nbytes // 2) // 16 * 16)
+    src = torch.empty(half, dtype=torch.uint8, device=dev)
+    dst = torch.empty_like(src)
+    ts = []
+    for i in range(reps + 2):
+        flush.fill_(i & 255)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        dst.copy_(src)
+        e1.record()
+        e1.synchronize()
+        if i >= 2:
+            ts.append(e0.elapsed_time(e1))
+    return statistics.median(ts)
+
+
 def sum_over_ranks(x: float, device, world: int) -> float:
     """The whole job's total of a per-rank quantity (e.g. the FLOPs of one step)."""
     t = torch.tensor([x], dtype=torch.float64, device=device)
@@ -660,8 +682,10 @@ def run_pbsa(args, w, rank, world, local_rank):
     ab = algorithmic_bytes(w, ncopy)
     kernels = {g: {"ms": per[g]} for g in groups}
     for g, b in ab.items():
+        floor = same_bytes_copy_ms(dev, b, flush)
         kernels[g].update({"algorithmic_bytes": b, "achieved_gbs": b / (per[g] * 1e-3) / 1e9,
-                           "frac_hbm": b / (per[g] * 1e-3) / 1e9 / peaks["hbm_gbs"]})
+                           "frac_hbm": b / (per[g] * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                           "same_bytes_copy_ms": floor, "frac_of_same_bytes_copy": floor / per[g]})
     att_tflops = flops / (per["attend"] * 1e-3) / 1e12
     kernels["attend"].update({"flops": flops, "achieved_tflops": att_tflops})
     value = job_flops / (step_ms_max * 1e-3) / 1e12
