@@ -104,6 +104,11 @@ CASES = {
     "bf16_k_above_candidates": (dict(heads=2, frame_h=16, frame_w=32), 1, 6, 20, 1),
     # 264 candidates in the last chunk: past the 8-block kernel's 256
     "bf16_long_sequence": (dict(heads=1), 1, 15, 16, 1),
+    # three sequences of two frames each: every sequence is a single, shorter-than-a-chunk chunk
+    "f32_sequences_shorter_than_a_chunk": (dict(heads=2, head_dim=64, frame_h=16, frame_w=16, dtype="f32"),
+                                           3, 2, 4, 1),
+    # 5 blocks per frame (an odd count: groups of 8 query blocks end inside a frame)
+    "bf16_odd_blocks_per_frame": (dict(heads=1, frame_h=8, frame_w=40), 2, 7, 6, 1),
 }
 
 
