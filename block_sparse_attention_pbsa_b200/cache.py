@@ -345,6 +345,32 @@ class PBSALayerCache:
         self.hist = hist_frames
         self._refresh_window()
 
+    # ------------------------------------------------------------------ checkpoint / resume
+    _STATE = ("k_pool", "v_pool", "k_reps", "slot_gid", "slot_ema", "p_list", "p_cnt")
+
+    def state_dict(self, device="cpu") -> dict:
+        """Everything a rollout needs to continue from here: the pools, key representatives and
+        slot tables (copied to ``device``), the number of committed frames and the local top-k.
+        The ring holds the window, so a copy taken after a commit resumes the rollout exactly."""
+        st = {name: getattr(self, name).to(device, copy=True) for name in self._STATE}
+        st["hist"] = self.hist
+        st["topk"] = self.topk
+        st["config"] = dataclasses.asdict(self.cfg)
+        return st
+
+    def load_state_dict(self, st: dict):
+        """Restore a ``state_dict`` taken from a cache of the same configuration."""
+        if st.get("config") != dataclasses.asdict(self.cfg):
+            raise ValueError("the state was taken from a cache of another configuration")
+        for name in self._STATE:
+            dst = getattr(self, name)
+            if tuple(st[name].shape) != tuple(dst.shape) or st[name].dtype != dst.dtype:
+                raise ValueError(f"{name}: shape or dtype does not match the cache")
+            dst.copy_(st[name])
+        self.hist = int(st["hist"])
+        self.topk = int(st["topk"])
+        self._refresh_window()
+
     # ------------------------------------------------------------------ inspection
     def persistent_gids(self) -> list[set[int]]:
         g = self.slot_gid.cpu()

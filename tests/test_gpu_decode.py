@@ -399,3 +399,41 @@ def test_head_sharded_caches_match_the_whole_layer(world):
             for name in ("slot_gid", "slot_ema", "k_pool", "v_pool", "k_reps", "p_list", "p_cnt"):
                 assert torch.equal(getattr(ca, name), getattr(full, name)[h0:h1]), (c, r, name)
             assert P.pbsa_get_device_error(ca.ws) == 0
+
+
+def test_rollout_resumes_from_a_checkpoint():
+    """A 5 s rollout checkpointed after its fourth chunk (state copied to the host) and resumed in
+    a fresh cache gives the same outputs and the same cache, bit for bit, over the remaining
+    chunks as the uninterrupted rollout."""
+    w = I.ROLLOUT_5S
+    chunks = I.rollout_chunks(w)
+    inputs = {}
+
+    def step(ca, c, s):
+        f0, nf = chunks[c]
+        wc = dataclasses.replace(w, chunk_frames=nf)
+        if (c, s) not in inputs:
+            inputs[c, s] = [I.tokens(wc, nf, I.stream_seed(w.seed, c, s, t)).to(DEV) for t in range(3)]
+        q, k, v = inputs[c, s]
+        o = ca.decode_step(q, k, v)
+        if s == 1:
+            ca.commit(k, v)
+        return o
+
+    full = P.PBSALayerCache(layer_cfg(w))
+    for c in range(4):
+        for s in range(2):
+            step(full, c, s)
+    ckpt = full.state_dict()
+    assert all(t.device.type == "cpu" for t in ckpt.values() if isinstance(t, torch.Tensor))
+    resumed = P.PBSALayerCache(layer_cfg(w))
+    resumed.load_state_dict(ckpt)
+    for c in range(4, len(chunks)):
+        for s in range(2):
+            assert torch.equal(step(full, c, s), step(resumed, c, s)), (c, s)
+    for name in P.PBSALayerCache._STATE:
+        assert torch.equal(getattr(full, name), getattr(resumed, name)), name
+    assert resumed.hist == full.hist
+    with pytest.raises(ValueError):
+        P.PBSALayerCache(dataclasses.replace(layer_cfg(w), capacity=48)).load_state_dict(ckpt)
+    assert P.pbsa_get_device_error(full.ws) == 0 and P.pbsa_get_device_error(resumed.ws) == 0
