@@ -20,6 +20,7 @@ same workload instead.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -199,12 +200,13 @@ def algorithmic_bytes(w, ncopy: int):
     }
 
 
-def run_train(P, I, dev, steps: int, peaks):
+def run_train(P, I, dev, steps: int, peaks, batch: int | None = None):
     """Trainable-path workload (batch 2 x 9 frames, 12 heads, 3-frame chunks; every query block
     of a later chunk attends the 24 sinks + its top-16 earlier blocks by coarse score + its own
     chunk): the masks (pbsa_blockify_train_select), the forward (pbsa_attend) and the backward
-    (pbsa_attend_bwd), each timed with CUDA events, L2 flushed before each; inputs resident in HBM."""
-    w = I.TRAIN_FWD_BWD
+    (pbsa_attend_bwd), each timed with CUDA events, L2 flushed before each; inputs resident in HBM.
+    ``batch`` overrides the workload's batch (a smaller case for profiler captures)."""
+    w = I.TRAIN_FWD_BWD if batch is None else dataclasses.replace(I.TRAIN_FWD_BWD, batch=batch)
     frames, batch = w.total_frames, w.batch
     qf = batch * frames
     q4, k4, v4, do4 = I.train_inputs(w, device=dev)
@@ -255,7 +257,7 @@ def run_train(P, I, dev, steps: int, peaks):
     sm, fm, bm = statistics.mean(sel_ms), statistics.mean(fwd_ms), statistics.mean(bwd_ms)
     sel_bytes = q.numel() * 2 + q_reps.numel() * 4 + k_reps.numel() * 4 + kv.numel() * 4
     sel_floor = same_bytes_copy_ms(dev, sel_bytes, flush)
-    return {"workload": w.name, "query_blocks": nq, "heads": w.heads, "steps": steps,
+    return {"workload": w.name, "batch": w.batch, "query_blocks": nq, "heads": w.heads, "steps": steps,
             "masks": "24 sinks + top-16 by coarse score among the earlier non-sink blocks + own chunk "
                      "(pbsa_blockify_train_select)",
             "select_ms": sm, "select_algorithmic_bytes": sel_bytes,
@@ -267,7 +269,8 @@ def run_train(P, I, dev, steps: int, peaks):
             "bwd_frac_of_bf16_peak": bwd_flops / (bm * 1e-3) / 1e12 / peaks["bf16"],
             "launches_per_iteration": 1 + 1 + 5,
             "note": "bwd FLOPs counted as 2.5x the forward's (5 GEMM-sized contractions vs 2); "
-                    "the deterministic kernels recompute S and dP in both the dQ and the dK/dV passes"}
+                    "the dK/dV pass computes S and dP once per pair and stores the dS tiles "
+                    "(bf16, 8 KB per pair) that the dQ pass reads back"}
 
 
 def run_rollout(P, I, dev, w, max_chunks=None, k_schedule=None, label=None):
@@ -675,6 +678,20 @@ def run_pbsa(args, w, rank, world, local_rank):
     if not torch.equal(oh, o.cpu()):
         raise RuntimeError("the pipelined end-to-end step returned a different O")
     e2e_ms_max = max_over_ranks(statistics.mean(e2e_ms), dev, world)
+    # the transfers alone (the same pinned buffers and bytes, upload then download on one
+    # stream, no kernels): the floor the end-to-end step approaches once its kernels hide
+    # behind the upload
+    xfer_ms = []
+    for s in range(4):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for dst, src in ((qd, qh), (kcd, kh), (vcd, vh), (oh, o)):
+            dst.copy_(src, non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        if s > 0:
+            xfer_ms.append(e0.elapsed_time(e1))
+    xfer_ms_max = max_over_ranks(statistics.mean(xfer_ms), dev, world)
     job_flops = sum_over_ranks(flops, dev, world)    # every rank's layer, or the shared layer's heads
 
     if rank != 0:
@@ -717,7 +734,8 @@ def run_pbsa(args, w, rank, world, local_rank):
                                    "K/V pools, key representatives, slot tables, lists, workspace; the staging "
                                    "area only serves the one-time prefill of a mid-video history"},
         "e2e": {"value": job_flops / (e2e_ms_max * 1e-3) / 1e12, "unit": "TFLOP/s",
-                "ms_per_step": e2e_ms_max, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "ms_per_step": e2e_ms_max, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "transfers_alone_ms": xfer_ms_max, "frac_of_transfers_alone": xfer_ms_max / e2e_ms_max},
         "gpu_launches": step.LAUNCHES * args.steps,
         "clocks": clk.summary(),
     }
@@ -750,6 +768,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-train", action="store_true", help="skip the forward+backward training workload")
     ap.add_argument("--train-only", action="store_true", help="only the training workload (for profiling)")
+    ap.add_argument("--train-batch", type=int, default=None,
+                    help="with --train-only: sequences in the training batch (default: the workload's 2)")
     ap.add_argument("--no-rollout", action="store_true", help="skip the 30-layer 5 s and 1-minute rollouts")
     ap.add_argument("--shard", choices=["layers", "heads"], default="layers",
                     help="N > 1: every rank its own layer (weak scaling, the default) or one layer's heads "
@@ -767,7 +787,7 @@ def main():
         import block_sparse_attention_pbsa_b200 as P
         dev = torch.device("cuda", local_rank)
         torch.cuda.set_device(dev)
-        print(json.dumps(run_train(P, I, dev, args.steps, load_peaks())), flush=True)
+        print(json.dumps(run_train(P, I, dev, args.steps, load_peaks(), args.train_batch)), flush=True)
         return
     if world > 1:
         import datetime

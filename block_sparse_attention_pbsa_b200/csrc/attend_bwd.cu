@@ -6,16 +6,22 @@
 //   P = exp(scale*Q K^T - LSE),  D_i = dO_i . O_i,  dP = dO V^T,  dS = P * (dP - D),
 //   dV = P^T dO,  dQ = scale * dS K,  dK = scale * dS^T Q.
 //
-// Deterministic design (no floating-point atomics), five launches:
+// Deterministic design (no floating-point atomics), five launches; S and dP are computed
+// once per (query block, KV block) pair, so the passes issue the five contractions S, dP, dV,
+// dK, dQ:
 //   1. bwd_prep_kernel  -- per query block: D and log2-domain LSE in block order, and the
 //      number of query blocks attending each KV slot (integer atomics);
 //   2. bwd_scan_kernel  -- per head: exclusive scan of those counts;
-//   3. bwd_fill_kernel  -- per query block: the inverse lists (KV slot -> query blocks);
-//   4. bwd_dq_kernel    -- one CTA per (head, pair of query blocks), like the forward:
-//      S = Q K^T and dP = dO V^T on tcgen05, dS into TMEM, dQ += dS K with A from TMEM;
-//   5. bwd_dkdv_kernel  -- one CTA per (head, pair of KV slots) over the query blocks that
+//   3. bwd_fill_kernel  -- per query block: the inverse lists (KV slot -> query block and the
+//      slot's position in that block's list);
+//   4. bwd_dkdv_kernel  -- one CTA per (head, pair of KV slots) over the query blocks that
 //      attend them (sorted, merged with a per-half mask): S^T = K Q^T, dP^T = V dO^T,
-//      dV += P^T dO and dK += dS^T Q with P^T, dS^T read from TMEM.
+//      dV += P^T dO and dK += dS^T Q with P^T, dS^T read from TMEM; each 64 x 64 dS^T tile
+//      also goes to the workspace (one tile per list entry, 8 KB);
+//   5. bwd_dqs_kernel   -- one CTA per (head, pair of query blocks): dQ += dS K over the
+//      merged list, A = the stored dS^T tiles read query-contiguous (MN-major).
+// The dS^T round trip through HBM (2 x 8 KB per pair) replaces the recomputation of S and dP
+// that a dQ pass needs otherwise.
 #include <math.h>
 
 #include "common.cuh"
@@ -30,7 +36,7 @@ constexpr float LOG2E = 1.4426950408889634f;
 __host__ __device__ inline size_t a256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct BwdLayout {
-  size_t dvec, lvec, cnt, off, cur, inv, end;
+  size_t dvec, lvec, cnt, off, cur, inv, zero, ds, end;
 };
 __host__ __device__ inline BwdLayout bwd_layout(int H, int nq, int ps, int kv_ld) {
   BwdLayout L;
@@ -40,7 +46,9 @@ __host__ __device__ inline BwdLayout bwd_layout(int H, int nq, int ps, int kv_ld
   L.off = L.cnt + a256((size_t)H * ps * 4);
   L.cur = L.off + a256((size_t)H * ps * 4);
   L.inv = L.cur + a256((size_t)H * ps * 4);
-  L.end = L.inv + a256((size_t)H * nq * kv_ld * 4);
+  L.zero = L.inv + a256((size_t)H * nq * kv_ld * 4);
+  L.ds = L.zero + BT * BT * 2;
+  L.end = L.ds + (size_t)H * nq * kv_ld * BT * BT * 2;   // one 64 x 64 bf16 dS^T tile per list entry
   return L;
 }
 
@@ -151,7 +159,7 @@ __global__ void __launch_bounds__(64) bwd_fill_kernel(BwdGeo g, const int* __res
     if (s < 0 || s >= g.pool_slots) continue;
     const size_t hs = (size_t)h * g.pool_slots + s;
     const int pos = off[hs] + atomicAdd(cur + hs, 1);
-    inv[(size_t)h * g.nq * g.kv_ld + pos] = r;
+    inv[(size_t)h * g.nq * g.kv_ld + pos] = r * g.kv_ld + e;   // query block and list position
   }
 }
 
@@ -168,23 +176,29 @@ __device__ __forceinline__ void wait_or_abort(uint64_t* bar, uint32_t parity, vo
 // ---------------------------------------------------------------------------- shared pieces
 constexpr int NT = 384;                                 // 12 warps
 constexpr uint32_t REG_CTRL = 56, REG_WORK = 224;       // 128*56 + 256*224 = 384*168
-constexpr uint32_t IDESC_KMAJ = idesc_bf16_f32(128, 128, 0, 0);   // A, B K-major
 constexpr uint32_t IDESC_BMN = idesc_bf16_f32(128, 128, 0, 1);    // B MN-major
 
-// Merge two lists (la[0..cA), lb[0..cB)) into mslot/mflag: A's entries (bit 0, plus bit 1
-// when also in B), then the B-only entries (bit 1), in order.  Returns the merged count.
-// All threads of the CTA call it; it ends with __syncthreads().
-__device__ int merge_pair(const int* la, int cA, const int* lb, int cB, int* mslot, uint8_t* mflag,
-                          uint8_t* onlyb, int* n_out) {
+// Merge two lists of keys (la[0..cA), lb[0..cB)): A's entries (mflag bit 0, plus bit 1 when
+// also in B), then the B-only entries (bit 1), in order; mkey receives the keys.  pos_a /
+// pos_b give each entry's position in its query block's list (nullptr: its index); mpa / mpb
+// receive them per merged key (-1 where the key is absent from that list).  All NTH threads
+// of the CTA call it; it ends with __syncthreads() and returns the merged count.
+template <int NTH>
+__device__ int merge_pair_pos(const int* la, const short* pos_a, int cA, const int* lb, const short* pos_b,
+                              int cB, int* mkey, short* mpa, short* mpb, uint8_t* mflag, uint8_t* onlyb,
+                              int* n_out) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  for (int i = tid; i < cA; i += NT) {
+  for (int i = tid; i < cA; i += NTH) {
     const int s = la[i];
-    uint8_t f = 1;
-    for (int j = 0; j < cB; ++j) f |= (lb[j] == s) ? 2 : 0;
-    mslot[i] = s;
-    mflag[i] = f;
+    int pb = -1;
+    for (int j = 0; j < cB; ++j)
+      if (lb[j] == s) pb = pos_b ? pos_b[j] : j;
+    mkey[i] = s;
+    mpa[i] = (short)(pos_a ? pos_a[i] : i);
+    mpb[i] = (short)pb;
+    mflag[i] = pb >= 0 ? 3 : 1;
   }
-  for (int j = tid; j < cB; j += NT) {
+  for (int j = tid; j < cB; j += NTH) {
     const int s = lb[j];
     bool in_a = false;
     for (int i = 0; i < cA; ++i) in_a |= (la[i] == s);
@@ -199,7 +213,9 @@ __device__ int merge_pair(const int* la, int cA, const int* lb, int cB, int* msl
       const unsigned bal = __ballot_sync(0xffffffffu, take);
       if (take) {
         const int at = pos + __popc(bal & ((1u << lane) - 1u));
-        mslot[at] = lb[j];
+        mkey[at] = lb[j];
+        mpa[at] = -1;
+        mpb[at] = (short)(pos_b ? pos_b[j] : j);
         mflag[at] = 2;
       }
       pos += __popc(bal);
@@ -210,302 +226,11 @@ __device__ int merge_pair(const int* la, int cA, const int* lb, int cB, int* msl
   return *n_out;
 }
 
-// ---------------------------------------------------------------------------- 4. dQ
-// smem: Q | dO (2 panels x [128 rows][128 B] each) | K ring (3) | V (1) | barriers | lists.
-// K(i) is read by S(i) and again by dQ(i) (the B operand), so its ring is the deeper one;
-// V(i) is free as soon as dP(i) is done.
-constexpr int QK_STAGES = 3;
-constexpr uint32_t Q_SM_Q = 0, Q_SM_DO = 32768, Q_SM_K = 65536, Q_SM_V = Q_SM_K + QK_STAGES * 32768;
-constexpr uint32_t Q_SM_BAR = Q_SM_V + 32768;
-constexpr uint32_t Q_SM_MISC = Q_SM_BAR + 256;
-constexpr uint32_t Q_SM_SLOT = Q_SM_MISC + 64;
-constexpr uint32_t Q_SM_FLAG = Q_SM_SLOT + 4 * 1024;
-constexpr uint32_t Q_SM_LA = Q_SM_FLAG + 1024;
-constexpr uint32_t Q_SM_LB = Q_SM_LA + 4 * 512;
-constexpr uint32_t Q_SM_ONLYB = Q_SM_LB + 4 * 512;
-constexpr uint32_t Q_SMEM_BYTES = Q_SM_ONLYB + 512 + 1024;
-enum { QB_QFULL = 0, QB_KFULL = 1, QB_KEMPTY = QB_KFULL + QK_STAGES, QB_VFULL = QB_KEMPTY + QK_STAGES,
-       QB_VEMPTY = QB_VFULL + 1, QB_SFULL = QB_VEMPTY + 1 /* [i&1] */,
-       QB_PFULL = QB_SFULL + 2 /* [w][i&1], 128 arrivals */, QB_DPFREE = QB_PFULL + 4 /* 256 arrivals */,
-       QB_SBFREE = QB_DPFREE + 1 /* [i&1]: dQ(i) has read dS(i) */, QB_MMADONE = QB_SBFREE + 2 /* 2 arrivals */,
-       QB_NUM = QB_MMADONE + 1 };
-
-struct DqParams {
-  BwdGeo g;
-  int kv_rows;
-  float scale, scale_log2;
-  const int* kv_slot;
-  const int* kv_cnt;
-  const float* dvec;
-  const float* lvec;
-  __nv_bfloat16* dq;
-  void* ws;
-};
-
-__global__ void __launch_bounds__(NT, 1)
-    bwd_dq_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap domap,
-                  const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
-                  const DqParams prm) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Q_SM_BAR);
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + Q_SM_MISC);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + Q_SM_MISC + 4);
-  int* n_merged_s = reinterpret_cast<int*>(sm + Q_SM_MISC + 8);
-  int* mslot = reinterpret_cast<int*>(sm + Q_SM_SLOT);
-  uint8_t* mflag = sm + Q_SM_FLAG;
-  int* la = reinterpret_cast<int*>(sm + Q_SM_LA);
-  int* lb = reinterpret_cast<int*>(sm + Q_SM_LB);
-  const BwdGeo& g = prm.g;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int h = blockIdx.y, rA = 2 * blockIdx.x, rB = rA + 1;
-  const bool hasB = rB < g.nq;
-
-  if (tid == 0) {
-    for (int i = 0; i < QB_NUM; ++i) mbar_init(&bars[i], 1);
-    for (int i = 0; i < 4; ++i) mbar_init(&bars[QB_PFULL + i], 128);
-    mbar_init(&bars[QB_DPFREE], 256);
-    mbar_init(&bars[QB_MMADONE], 2);
-    *abort_flag = 0;
-    fence_barrier_init();
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_holder, 512);
-    tmem_relinquish();
-  }
-  int cA = prm.kv_cnt[(size_t)h * g.nq + rA];
-  int cB = hasB ? prm.kv_cnt[(size_t)h * g.nq + rB] : 0;
-  cA = min(max(cA, 0), g.kv_ld);
-  cB = min(max(cB, 0), g.kv_ld);
-  const int* listA = prm.kv_slot + ((size_t)h * g.nq + rA) * g.kv_ld;
-  const int* listB = prm.kv_slot + ((size_t)h * g.nq + (hasB ? rB : rA)) * g.kv_ld;
-  for (int i = tid; i < cA; i += NT) la[i] = listA[i];
-  for (int i = tid; i < cB; i += NT) lb[i] = listB[i];
-  __syncthreads();
-  const int n = merge_pair(la, cA, lb, cB, mslot, mflag, sm + Q_SM_ONLYB, n_merged_s);
-  for (int i = tid; i < n; i += NT) {
-    const int s = mslot[i];
-    if (s < 0 || s >= g.pool_slots) {
-      record_error(prm.ws, PBSA_ERR_DEVICE_INDEX, s, K_BWD_Q);
-      mslot[i] = -1;
-      mflag[i] = 0;
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_holder;
-  const int nsteps = (n + 1) >> 1;
-
-  if (warp < 4) {
-    setmaxnreg_dec<REG_CTRL>();
-    auto load_pair = [&](const CUtensorMap* map, uint8_t* dst, uint64_t* bar, int i) {
-      for (int b = 0; b < 2; ++b) {
-        const int e = 2 * i + b;
-        const int slot = e < n ? mslot[e] : -1;
-        const int row0 = slot >= 0 ? (h * g.pool_slots + slot) * 64 : prm.kv_rows;
-        for (int p = 0; p < 2; ++p) tma_load_2d(dst + p * 16384 + b * 8192, map, bar, p * 64, row0);
-      }
-    };
-    if (warp == 0 && lane == 0 && nsteps > 0) {
-      // ---- producer: Q and dO once, then the K ring
-      tma_prefetch_desc(&qmap);
-      tma_prefetch_desc(&domap);
-      tma_prefetch_desc(&kmap);
-      mbar_arrive_expect_tx(&bars[QB_QFULL], 65536);
-      for (int half = 0; half < 2; ++half) {
-        const int r = (half == 1 && hasB) ? rB : rA;
-        const int f = r / g.bpf, rem = r - f * g.bpf;
-        const int ty = rem / g.tpr, tx = rem - ty * g.tpr;
-        for (int p = 0; p < 2; ++p) {
-          tma_load_5d(sm + Q_SM_Q + p * 16384 + half * 8192, &qmap, &bars[QB_QFULL], p * 64, h, tx * g.tw, ty * g.th, f);
-          tma_load_5d(sm + Q_SM_DO + p * 16384 + half * 8192, &domap, &bars[QB_QFULL], p * 64, h, tx * g.tw, ty * g.th, f);
-        }
-      }
-      int kiss = 0;
-      for (int i = 0; i < nsteps; ++i) {
-        const int s = i % QK_STAGES;
-        wait_or_abort(&bars[QB_KEMPTY + s], ((i / QK_STAGES) & 1) ^ 1, abort_flag, prm.ws, 1, K_BWD_Q);
-        if (*abort_flag) break;
-        mbar_arrive_expect_tx(&bars[QB_KFULL + s], 32768);
-        load_pair(&kmap, sm + Q_SM_K + s * 32768, &bars[QB_KFULL + s], i);
-        kiss = i + 1;
-      }
-      if (*abort_flag) {
-        mbar_wait(&bars[QB_QFULL], 0, kWaitLimitNs);
-        for (int i = (kiss > QK_STAGES ? kiss - QK_STAGES : 0); i < kiss; ++i)
-          mbar_wait(&bars[QB_KFULL + i % QK_STAGES], (i / QK_STAGES) & 1, kWaitLimitNs);
-      }
-    }
-    if (warp == 2 && lane == 0 && nsteps > 0) {
-      // ---- producer: V of each step (one stage)
-      tma_prefetch_desc(&vmap);
-      int viss = 0;
-      for (int i = 0; i < nsteps; ++i) {
-        wait_or_abort(&bars[QB_VEMPTY], (i & 1) ^ 1, abort_flag, prm.ws, 2, K_BWD_Q);
-        if (*abort_flag) break;
-        mbar_arrive_expect_tx(&bars[QB_VFULL], 32768);
-        load_pair(&vmap, sm + Q_SM_V, &bars[QB_VFULL], i);
-        viss = i + 1;
-      }
-      if (*abort_flag && viss > 0) mbar_wait(&bars[QB_VFULL], (viss - 1) & 1, kWaitLimitNs);
-    }
-    // ---- MMA issuers.  TMEM: S[i&1] at 128*(i&1), dP at 256, dQ at 384.
-    // Warp 1 issues S(i) (once dQ(i-2) has read the dS over S[i&1]) and dP(i) (once the
-    // warpgroups hold dP(i-1) in registers), so the tensor pipe computes S(i+1) and dP(i+1)
-    // while the warpgroups form dS(i).  Warp 3 issues dQ += dS(i) K(i) for every step in
-    // order, one thread, so dQ accumulates in a fixed order.
-    if (warp == 1 && lane == 0 && nsteps > 0) {
-      const uint64_t dq_ = sw128_desc(smem_u32(sm + Q_SM_Q), 16, 1024);
-      const uint64_t ddo = sw128_desc(smem_u32(sm + Q_SM_DO), 16, 1024);
-      const uint64_t dk = sw128_desc(smem_u32(sm + Q_SM_K), 16, 1024);
-      const uint64_t dv = sw128_desc(smem_u32(sm + Q_SM_V), 16, 1024);
-      wait_or_abort(&bars[QB_QFULL], 0, abort_flag, prm.ws, 4, K_BWD_Q);
-      for (int i = 0; i < nsteps && !*abort_flag; ++i) {
-        const int sk = i % QK_STAGES;
-        // S(i) = Q K(i)^T into S[i&1]
-        if (i >= 2) wait_or_abort(&bars[QB_SBFREE + (i & 1)], ((i - 2) >> 1) & 1, abort_flag, prm.ws, 10, K_BWD_Q);
-        wait_or_abort(&bars[QB_KFULL + sk], (i / QK_STAGES) & 1, abort_flag, prm.ws, 5, K_BWD_Q);
-        if (*abort_flag) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
-          mma_bf16_ss(tmem + (i & 1) * 128, dq_ + off, dk + ((sk * 32768) >> 4) + off, IDESC_KMAJ,
-                      kk > 0 ? 1u : 0u);
-        }
-        // dP(i) = dO V(i)^T, then V's stage is free
-        if (i >= 1) wait_or_abort(&bars[QB_DPFREE], (i - 1) & 1, abort_flag, prm.ws, 9, K_BWD_Q);
-        wait_or_abort(&bars[QB_VFULL], i & 1, abort_flag, prm.ws, 6, K_BWD_Q);
-        if (*abort_flag) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
-          mma_bf16_ss(tmem + 256, ddo + off, dv + off, IDESC_KMAJ, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(&bars[QB_VEMPTY]);
-        mma_commit(&bars[QB_SFULL + (i & 1)]);
-      }
-      mma_commit(&bars[QB_MMADONE]);
-      mbar_wait(&bars[QB_MMADONE], 0, kWaitLimitNs);
-    }
-    if (warp == 3 && lane == 0 && nsteps > 0) {
-      const uint64_t dk_mn = sw128_desc(smem_u32(sm + Q_SM_K), 16384, 1024);
-      for (int i = 0; i < nsteps && !*abort_flag; ++i) {
-        const int s = i & 1, sk = i % QK_STAGES;
-        // dQ += dS(i) K(i): dS(i) (bf16 pairs) sits over S[s], warpgroup w's 64 keys in its
-        // half; K(i) is the B operand (keys x d, d contiguous).  S(i) completed before dS(i)
-        // was formed, so the commits below cover every MMA that read K(i) and S[s].
-        for (int w = 0; w < 2; ++w) {
-          wait_or_abort(&bars[QB_PFULL + 2 * w + s], (i >> 1) & 1, abort_flag, prm.ws, 3, K_BWD_Q);
-          if (*abort_flag) break;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_ts(tmem + 384, tmem + s * 128 + w * 64 + kk * 8,
-                        dk_mn + ((sk * 32768 + w * 8192 + kk * 2048) >> 4), IDESC_BMN,
-                        (i > 0 || w > 0 || kk > 0) ? 1u : 0u);
-        }
-        mma_commit(&bars[QB_KEMPTY + sk]);
-        mma_commit(&bars[QB_SBFREE + s]);
-      }
-      mma_commit(&bars[QB_MMADONE]);
-      mbar_wait(&bars[QB_MMADONE], 0, kWaitLimitNs);
-    }
-    __syncwarp();
-  } else {
-    setmaxnreg_inc<REG_WORK>();
-    // ---- dS = P * (dP - D) for the block of the step this warpgroup owns
-    const int wg = (warp - 4) >> 2, wq = warp & 3;
-    const int row = wq * 32 + lane, half = row >> 6;
-    const bool row_valid = half == 0 || hasB;
-    const int r = half ? rB : rA;
-    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-    const size_t bi = ((size_t)h * g.nq + (row_valid ? r : rA)) * BT + (row & 63);
-    const float lse2 = prm.lvec[bi], dd = prm.dvec[bi];
-    const float c = prm.scale_log2;
-    for (int i = 0; i < nsteps; ++i) {
-      const int e = 2 * i + wg;
-      const bool v = row_valid && e < n && ((mflag[e] >> half) & 1);
-      const uint32_t tS = tmem + lane_off + (i & 1) * 128 + wg * 64;
-      const uint32_t tP = tmem + lane_off + 256 + wg * 64;
-      wait_or_abort(&bars[QB_SFULL + (i & 1)], (i >> 1) & 1, abort_flag, prm.ws, 7, K_BWD_Q);
-      if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
-      tc_fence_after();
-      // every column holds a finite value (a block that does not exist was loaded as
-      // zeros), so all are read and masking is arithmetic
-      uint32_t xs[2][32], xp[2][32];
-      tmem_ld32(tS, xs[0]);
-      tmem_ld32(tS + 32, xs[1]);
-      tmem_ld32(tP, xp[0]);
-      tmem_ld32(tP + 32, xp[1]);
-      tmem_wait_ld();
-      // dP(i) is in registers: the issuer may overwrite its TMEM with dP(i+1)
-      tc_fence_before();
-      mbar_arrive(&bars[QB_DPFREE]);
-      // dS = P * (dP - D), P = 2^(s*c - lse2); a masked block uses the factor 0 and the offset
-      // -inf, so P (and dS) are exact zeros without a branch
-      const float cs = v ? c : 0.f, ms = v ? -lse2 : -INFINITY;
-      uint32_t pk[32];
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
-#pragma unroll
-        for (int e2 = 0; e2 < 16; ++e2) {
-          float a0, a1, t0, t1, d0, d1;
-          ffma2(__uint_as_float(xs[q][2 * e2]), __uint_as_float(xs[q][2 * e2 + 1]), cs, ms, a0, a1);
-          ffma2(__uint_as_float(xp[q][2 * e2]), __uint_as_float(xp[q][2 * e2 + 1]), 1.f, -dd, t0, t1);
-          fmul2(ex2_approx(a0), ex2_approx(a1), t0, t1, d0, d1);
-          pk[q * 16 + e2] = pack_bf16(d0, d1);
-        }
-      }
-      tmem_st32(tS, pk);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&bars[QB_PFULL + 2 * wg + (i & 1)]);
-    }
-    // ---- epilogue: dQ = scale * (dS K) -> bf16 raster rows; warpgroup w writes columns [64w, +64)
-    if (nsteps > 0) wait_or_abort(&bars[QB_MMADONE], 0, abort_flag, prm.ws, 8, K_BWD_Q);
-    if (row_valid && !__any_sync(0xffffffffu, *abort_flag != 0)) {
-      const size_t t = token_of(g, r, row & 63);
-      uint4* dst = reinterpret_cast<uint4*>(prm.dq + (t * g.H + h) * D) + wg * 8;
-      tc_fence_after();
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        uint32_t ov[32];
-        if (nsteps > 0) {
-          tmem_ld32(tmem + lane_off + 384 + wg * 64 + q * 32, ov);
-          tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int e2 = 0; e2 < 32; ++e2) ov[e2] = 0u;
-        }
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          uint32_t wv[4];
-#pragma unroll
-          for (int e2 = 0; e2 < 4; ++e2)
-            wv[e2] = pack_bf16(__uint_as_float(ov[cc * 8 + 2 * e2]) * prm.scale,
-                               __uint_as_float(ov[cc * 8 + 2 * e2 + 1]) * prm.scale);
-          dst[q * 4 + cc] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-        }
-      }
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, 512);
-  }
-}
-
-
-// ---------------------------------------------------------------------------- 5. dK, dV
+// ---------------------------------------------------------------------------- 4. dK, dV
 // smem: K pair | V pair (2 panels x [128 keys][128 B] each) | KV_QST stages x (Q, dO tiles of one
 // query block: 2 panels x [64 rows][128 B] each) | KV_QST x [log2-LSE | D] x 64 f32 | barriers |
-// lists
-constexpr int KV_QST = 4;                                            // query-block stages
+// lists | per formation warp, a 4 KB buffer of dS^T rows on their way to the workspace
+constexpr int KV_QST = 3;                                            // query-block stages
 constexpr uint32_t KV_SM_K = 0, KV_SM_V = 32768, KV_SM_Q = 65536;    // Q stage s at +KV_STAGE*s
 constexpr uint32_t KV_STAGE = 32768;                                 // Q (16 KB) + dO (16 KB)
 constexpr uint32_t KV_SM_VEC = KV_SM_Q + KV_QST * KV_STAGE;          // [stage][lse2 | D][64] f32
@@ -517,7 +242,13 @@ constexpr uint32_t KV_SM_LA = KV_SM_FLAG + 1024;
 constexpr uint32_t KV_SM_LB = KV_SM_LA + 4 * 512;
 constexpr uint32_t KV_SM_ONLYB = KV_SM_LB + 4 * 512;
 constexpr uint32_t KV_SM_TMP = KV_SM_ONLYB + 512;                    // int[512] sort scratch
-constexpr uint32_t KV_SMEM_BYTES = KV_SM_TMP + 4 * 512 + 1024;
+constexpr uint32_t KV_SM_MPA = KV_SM_TMP + 4 * 512;                  // short[1024] positions in the
+constexpr uint32_t KV_SM_MPB = KV_SM_MPA + 2 * 1024;                 //   query blocks' lists
+constexpr uint32_t KV_SM_PLA = KV_SM_MPB + 2 * 1024;                 // short[512] each
+constexpr uint32_t KV_SM_PLB = KV_SM_PLA + 2 * 512;
+constexpr uint32_t KV_SM_STG = (KV_SM_PLB + 2 * 512 + 1023) & ~1023u;  // [8 warps][32 rows][128 B] dS^T
+constexpr uint32_t KV_SMEM_BYTES = KV_SM_STG + 8 * 4096 + 1024;
+static_assert(KV_SMEM_BYTES <= 227 * 1024, "shared memory of one CTA");
 enum { KB_KVFULL = 0, KB_QFULL = 1, KB_QEMPTY = KB_QFULL + KV_QST, KB_SFULL = KB_QEMPTY + KV_QST /* [b] */,
        KB_PFULL = KB_SFULL + 2 /* [b], 128 arrivals */, KB_BFREE = KB_PFULL + 2 /* [b] */,
        KB_MMADONE = KB_BFREE + 2 /* 2 arrivals */, KB_NUM = KB_MMADONE + 1 };
@@ -535,6 +266,7 @@ struct DkvParams {
   const float* lvec;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
+  __nv_bfloat16* ds;   // dS^T tiles, one per (head, query block, list position)
   void* ws;
 };
 
@@ -602,7 +334,24 @@ __global__ void __launch_bounds__(NT, 1)
   __syncthreads();
   sort_small(tmp, cB, lb);
   __syncthreads();
-  const int n = merge_pair(la, cA, lb, cB, mslot, mflag, sm + KV_SM_ONLYB, n_merged_s);
+  // split each entry into its query block and the slot's position in that block's list
+  short* pla = reinterpret_cast<short*>(sm + KV_SM_PLA);
+  short* plb = reinterpret_cast<short*>(sm + KV_SM_PLB);
+  short* mpa = reinterpret_cast<short*>(sm + KV_SM_MPA);
+  short* mpb = reinterpret_cast<short*>(sm + KV_SM_MPB);
+  for (int i = tid; i < cA; i += NT) {
+    const int v = la[i];
+    la[i] = v / g.kv_ld;
+    pla[i] = (short)(v - (v / g.kv_ld) * g.kv_ld);
+  }
+  for (int i = tid; i < cB; i += NT) {
+    const int v = lb[i];
+    lb[i] = v / g.kv_ld;
+    plb[i] = (short)(v - (v / g.kv_ld) * g.kv_ld);
+  }
+  __syncthreads();
+  const int n = merge_pair_pos<NT>(la, pla, cA, lb, plb, cB, mslot, mpa, mpb, mflag, sm + KV_SM_ONLYB,
+                                   n_merged_s);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -752,7 +501,30 @@ __global__ void __launch_bounds__(NT, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars[KB_PFULL + wg]);
+      // dS^T rows for the dQ pass, off the chain (this step's dV/dK MMAs run meanwhile): tile
+      // (query block, position of this slot in its list), row = key, 64 query columns (128 B),
+      // 16-byte chunk c of row k at ((c ^ (k & 7)) << 4) (the 128-byte swizzle, so that a plain
+      // copy into aligned shared memory is an MMA operand).  The warp's 32 rows are staged in
+      // shared memory and leave as one 4 KB bulk copy.  v is warp-uniform.
+      if (v) {
+        uint8_t* stg = sm + KV_SM_STG + (warp - 4) * 4096;
+        if (lane == 0) bulk_wait_read<0>();   // this warp's previous copy has left the buffer
+        __syncwarp();
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc)
+          *reinterpret_cast<uint4*>(stg + lane * 128 + ((cc ^ (lane & 7)) << 4)) =
+              make_uint4(pd[4 * cc], pd[4 * cc + 1], pd[4 * cc + 2], pd[4 * cc + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          const int pos = kh ? mpb[j] : mpa[j];
+          bulk_store(prm.ds + ((((size_t)h * g.nq + mslot[j]) * g.kv_ld + pos) * BT + (wq & 1) * 32) * BT, stg, 4096);
+          bulk_commit();
+        }
+      }
     }
+    if (lane == 0) bulk_wait_all();   // every dS^T copy of this warp has been written
+    __syncwarp();
     // ---- epilogue: dV and dK = scale * (dS^T Q) rows of the pair's slots, warpgroup w
     // writes columns [64w, +64) of both
     if (nsteps > 0) wait_or_abort(&bars[KB_MMADONE], 0, abort_flag, prm.ws, 6, K_BWD_KV);
@@ -795,6 +567,177 @@ __global__ void __launch_bounds__(NT, 1)
   }
 }
 
+// ---------------------------------------------------------------------------- 5. dQ from dS
+// dQ = scale * dS K with the dS^T tiles the dK/dV pass stored: one CTA per (head, pair of
+// query blocks), 128 threads.  The two lists are merged; merged entry e brings the K block of
+// its slot and the dS^T tiles of the two query blocks (a block that does not attend the slot
+// gets a tile loaded out of bounds, i.e. zeros) into one stage; four MMAs (K = 16 keys each)
+// accumulate dQ (128 query rows x 128 d) in TMEM, in the merged order (deterministic).
+//   A = dS (M = the pair's 128 queries, K = keys): the two tiles, query-contiguous (MN-major),
+//   B = K  (K = keys, N = d): d-contiguous (MN-major).
+constexpr int DQ_NT = 128;
+constexpr int DS_STAGES = 3;
+constexpr uint32_t DS_STAGE = 32768;                            // K block (16 KB) + two dS^T tiles
+constexpr uint32_t DS_SM_BAR = DS_STAGES * DS_STAGE;
+constexpr uint32_t DS_SM_MISC = DS_SM_BAR + 128;
+constexpr uint32_t DS_SM_SLOT = DS_SM_MISC + 64;                // int[1024] merged slots
+constexpr uint32_t DS_SM_MPA = DS_SM_SLOT + 4 * 1024;           // short[1024] positions in list A
+constexpr uint32_t DS_SM_MPB = DS_SM_MPA + 2 * 1024;            // short[1024] positions in list B
+constexpr uint32_t DS_SM_FLAG = DS_SM_MPB + 2 * 1024;           // uint8[1024]
+constexpr uint32_t DS_SM_LA = DS_SM_FLAG + 1024;                // int[512]
+constexpr uint32_t DS_SM_LB = DS_SM_LA + 4 * 512;               // int[512]
+constexpr uint32_t DS_SM_ONLYB = DS_SM_LB + 4 * 512;            // uint8[512]
+constexpr uint32_t DS_SMEM_BYTES = DS_SM_ONLYB + 512 + 1024;
+static_assert(2 * DS_SMEM_BYTES <= 228 * 1024, "two CTAs per SM");
+enum { DB_FULL = 0, DB_EMPTY = DB_FULL + DS_STAGES, DB_DONE = DB_EMPTY + DS_STAGES, DB_NUM = DB_DONE + 1 };
+static_assert(DB_NUM * 8 <= 128, "barrier area");
+constexpr uint32_t IDESC_AMN_BMN = idesc_bf16_f32(128, 128, 1, 1);
+
+struct DqsParams {
+  BwdGeo g;
+  int kv_rows;   // first out-of-bounds row of the K pool map
+  float scale;
+  const __nv_bfloat16* ds;     // dS^T tiles (128-byte swizzled rows)
+  const __nv_bfloat16* zero;   // one all-zero tile, for a query block that does not attend
+  const int* kv_slot;
+  const int* kv_cnt;
+  __nv_bfloat16* dq;
+  void* ws;
+};
+
+__global__ void __launch_bounds__(DQ_NT, 2)
+    bwd_dqs_kernel(const __grid_constant__ CUtensorMap kmap, const DqsParams prm) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + DS_SM_BAR);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + DS_SM_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + DS_SM_MISC + 4);
+  int* n_merged_s = reinterpret_cast<int*>(sm + DS_SM_MISC + 8);
+  int* mslot = reinterpret_cast<int*>(sm + DS_SM_SLOT);
+  short* mpa = reinterpret_cast<short*>(sm + DS_SM_MPA);
+  short* mpb = reinterpret_cast<short*>(sm + DS_SM_MPB);
+  int* la = reinterpret_cast<int*>(sm + DS_SM_LA);
+  int* lb = reinterpret_cast<int*>(sm + DS_SM_LB);
+  const BwdGeo& g = prm.g;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int h = blockIdx.y, rA = 2 * blockIdx.x, rB = rA + 1;
+  const bool hasB = rB < g.nq;
+
+  if (tid == 0) {
+    for (int i = 0; i < DB_NUM; ++i) mbar_init(&bars[i], 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, 128);
+    tmem_relinquish();
+  }
+  int cA = prm.kv_cnt[(size_t)h * g.nq + rA];
+  int cB = hasB ? prm.kv_cnt[(size_t)h * g.nq + rB] : 0;
+  cA = min(max(cA, 0), min(g.kv_ld, 512));
+  cB = min(max(cB, 0), min(g.kv_ld, 512));
+  const int* listA = prm.kv_slot + ((size_t)h * g.nq + rA) * g.kv_ld;
+  const int* listB = prm.kv_slot + ((size_t)h * g.nq + (hasB ? rB : rA)) * g.kv_ld;
+  for (int i = tid; i < cA; i += DQ_NT) la[i] = listA[i];
+  for (int i = tid; i < cB; i += DQ_NT) lb[i] = listB[i];
+  __syncthreads();
+  const int n = merge_pair_pos<DQ_NT>(la, nullptr, cA, lb, nullptr, cB, mslot, mpa, mpb, sm + DS_SM_FLAG,
+                                      sm + DS_SM_ONLYB, n_merged_s);
+  for (int i = tid; i < n; i += DQ_NT) {
+    const int s = mslot[i];
+    if (s < 0 || s >= g.pool_slots) {   // no dS was stored for it: zeros on both halves
+      record_error(prm.ws, PBSA_ERR_DEVICE_INDEX, s, K_BWD_Q);
+      mslot[i] = -1;
+      mpa[i] = -1;
+      mpb[i] = -1;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0 && lane == 0 && n > 0) {
+    // ---- producer: per merged entry, K block + the two dS^T tiles into one stage
+    tma_prefetch_desc(&kmap);
+    int iss = 0;
+    for (int e = 0; e < n; ++e) {
+      const int st = e % DS_STAGES;
+      wait_or_abort(&bars[DB_EMPTY + st], ((e / DS_STAGES) & 1) ^ 1, abort_flag, prm.ws, 1, K_BWD_Q);
+      if (*abort_flag) break;
+      mbar_arrive_expect_tx(&bars[DB_FULL + st], DS_STAGE);
+      uint8_t* dst = sm + st * DS_STAGE;
+      const int slot = mslot[e];
+      const int krow = slot >= 0 ? (h * g.pool_slots + slot) * BT : prm.kv_rows;
+      tma_load_2d(dst, &kmap, &bars[DB_FULL + st], 0, krow);
+      tma_load_2d(dst + 8192, &kmap, &bars[DB_FULL + st], 64, krow);
+      const int pa = mpa[e], pb = mpb[e];
+      const __nv_bfloat16* ta = pa >= 0 ? prm.ds + (((size_t)h * g.nq + rA) * g.kv_ld + pa) * BT * BT : prm.zero;
+      const __nv_bfloat16* tb = (pb >= 0 && hasB) ? prm.ds + (((size_t)h * g.nq + rB) * g.kv_ld + pb) * BT * BT : prm.zero;
+      bulk_load(dst + 16384, ta, 8192, &bars[DB_FULL + st]);
+      bulk_load(dst + 24576, tb, 8192, &bars[DB_FULL + st]);
+      iss = e + 1;
+    }
+    if (*abort_flag)
+      for (int e = (iss > DS_STAGES ? iss - DS_STAGES : 0); e < iss; ++e)
+        mbar_wait(&bars[DB_FULL + e % DS_STAGES], (e / DS_STAGES) & 1, kWaitLimitNs);
+  }
+  if (warp == 1 && lane == 0 && n > 0) {
+    // ---- MMA issuer: dQ += dS_e K_e, in merged order
+    for (int e = 0; e < n && !*abort_flag; ++e) {
+      const int st = e % DS_STAGES;
+      wait_or_abort(&bars[DB_FULL + st], (e / DS_STAGES) & 1, abort_flag, prm.ws, 2, K_BWD_Q);
+      if (*abort_flag) break;
+      tc_fence_after();
+      const uint32_t base = smem_u32(sm + st * DS_STAGE);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_bf16_ss(tmem, sw128_desc(base + 16384 + kk * 2048, 8192, 1024),
+                    sw128_desc(base + kk * 2048, 8192, 1024), IDESC_AMN_BMN, (e > 0 || kk > 0) ? 1u : 0u);
+      mma_commit(&bars[DB_EMPTY + st]);
+    }
+    mma_commit(&bars[DB_DONE]);
+  }
+  __syncwarp();
+  // ---- epilogue: every warp, its 32 TMEM lanes = query rows
+  const int row = warp * 32 + lane, half = row >> 6;
+  const bool row_valid = half == 0 || hasB;
+  if (n > 0) wait_or_abort(&bars[DB_DONE], 0, abort_flag, prm.ws, 3, K_BWD_Q);
+  tc_fence_after();
+  if (row_valid && !__any_sync(0xffffffffu, *abort_flag != 0)) {
+    const int r = half ? rB : rA;
+    const size_t t = token_of(g, r, row & 63);
+    uint4* dst = reinterpret_cast<uint4*>(prm.dq + (t * g.H + h) * D);
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint32_t ov[32];
+      if (n > 0) {
+        tmem_ld32(tmem + lane_off + q * 32, ov);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int e2 = 0; e2 < 32; ++e2) ov[e2] = 0u;
+      }
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t wv[4];
+#pragma unroll
+        for (int e2 = 0; e2 < 4; ++e2)
+          wv[e2] = pack_bf16(__uint_as_float(ov[cc * 8 + 2 * e2]) * prm.scale,
+                             __uint_as_float(ov[cc * 8 + 2 * e2 + 1]) * prm.scale);
+        dst[q * 4 + cc] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
 }  // namespace
 
 size_t attend_bwd_ws_bytes(const Geo& g, int q_frames, int pool_slots, int kv_ld) {
@@ -826,7 +769,11 @@ cudaError_t launch_attend_bwd(const Geo& gg, const void* q, int q_frames, const 
   int* off = reinterpret_cast<int*>(base + L.off);
   int* cur = reinterpret_cast<int*>(base + L.cur);
   int* inv = reinterpret_cast<int*>(base + L.inv);
+  __nv_bfloat16* ds = reinterpret_cast<__nv_bfloat16*>(base + L.ds);
+  __nv_bfloat16* dzero = reinterpret_cast<__nv_bfloat16*>(base + L.zero);
+  if (kv_ld > 32767) return cudaErrorNotSupported;
   cudaError_t e;
+  if ((e = cudaMemsetAsync(dzero, 0, BT * BT * 2, st)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(cnt, 0, (size_t)g.H * pool_slots * 4, st)) != cudaSuccess) return e;
 
   CUtensorMap qmap, domap, kmap, vmap;
@@ -856,21 +803,6 @@ cudaError_t launch_attend_bwd(const Geo& gg, const void* q, int q_frames, const 
   bwd_fill_kernel<<<dim3(g.nq, g.H), 64, 0, st>>>(g, kv_slot, kv_cnt, off, cur, inv);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
-  DqParams dp;
-  dp.g = g;
-  dp.kv_rows = g.H * pool_slots * BT;
-  dp.scale = scale;
-  dp.scale_log2 = scale * LOG2E;
-  dp.kv_slot = kv_slot;
-  dp.kv_cnt = kv_cnt;
-  dp.dvec = dvec;
-  dp.lvec = lvec;
-  dp.dq = static_cast<__nv_bfloat16*>(dq);
-  dp.ws = ws;
-  if ((e = set_smem_once((const void*)bwd_dq_kernel, (int)Q_SMEM_BYTES)) != cudaSuccess) return e;
-  bwd_dq_kernel<<<dim3((g.nq + 1) / 2, g.H), NT, Q_SMEM_BYTES, st>>>(qmap, domap, kmap, vmap, dp);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-
   DkvParams kp;
   kp.g = g;
   kp.kv_rows = g.H * pool_slots * BT;
@@ -884,9 +816,24 @@ cudaError_t launch_attend_bwd(const Geo& gg, const void* q, int q_frames, const 
   kp.lvec = lvec;
   kp.dk = static_cast<__nv_bfloat16*>(dk_pool);
   kp.dv = static_cast<__nv_bfloat16*>(dv_pool);
+  kp.ds = ds;
   kp.ws = ws;
   if ((e = set_smem_once((const void*)bwd_dkdv_kernel, (int)KV_SMEM_BYTES)) != cudaSuccess) return e;
   bwd_dkdv_kernel<<<dim3((pool_slots + 1) / 2, g.H), NT, KV_SMEM_BYTES, st>>>(qmap, domap, kmap, vmap, kp);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+  DqsParams dp;
+  dp.g = g;
+  dp.kv_rows = g.H * pool_slots * BT;
+  dp.ds = ds;
+  dp.zero = dzero;
+  dp.scale = scale;
+  dp.kv_slot = kv_slot;
+  dp.kv_cnt = kv_cnt;
+  dp.dq = static_cast<__nv_bfloat16*>(dq);
+  dp.ws = ws;
+  if ((e = set_smem_once((const void*)bwd_dqs_kernel, (int)DS_SMEM_BYTES)) != cudaSuccess) return e;
+  bwd_dqs_kernel<<<dim3((g.nq + 1) / 2, g.H), DQ_NT, DS_SMEM_BYTES, st>>>(kmap, dp);
   return cudaGetLastError();
 }
 

@@ -245,9 +245,13 @@ PBSA_API pbsa_status pbsa_attend(const pbsa_geom* g, const void* q, int q_frames
  *  dk_pool, dv_pool out [H][pool_slots][64][d] bf16: every slot is written (slots that no
  *          query block attends get zeros).
  *  bf16, d = 128, kv_ld <= 512, q_frames*bpf <= 512 query blocks.  Deterministic (no
- *  floating-point atomics).
+ *  floating-point atomics).  S and dP are computed once per (query block, listed block) pair:
+ *  the dK/dV pass stores each 64 x 64 dS tile (bf16) in the workspace and the dQ pass reads
+ *  it back.
  *  ws: pbsa_bwd_workspace_bytes(g, q_frames, pool_slots, kv_ld) bytes of device memory whose
- *  first 256 bytes (the error word) are zero before first use. */
+ *  first 256 bytes (the error word) are zero before first use.  It holds one 8 KB dS tile per
+ *  (head, query block, list entry): H * q_frames*bpf * kv_ld * 8192 bytes, plus a few bytes
+ *  per query row and per slot. */
 PBSA_API size_t pbsa_bwd_workspace_bytes(const pbsa_geom* g, int q_frames, int pool_slots, int kv_ld);
 PBSA_API pbsa_status pbsa_attend_bwd(const pbsa_geom* g, const void* q, int q_frames,
                                      const void* k_pool, const void* v_pool, int pool_slots,

@@ -132,6 +132,10 @@ def test_every_entry_point_checks_its_arguments_on_the_host(lib):
         assert L.pbsa_workspace_bytes(ctypes.byref(geom), 8, 8) == 0, what
         assert L.pbsa_bwd_workspace_bytes(ctypes.byref(geom), 1, 8, 8) == 0, what
     assert L.pbsa_bwd_workspace_bytes(gp, 0, 8, 8) == 0
+    # the backward keeps one 8 KB bf16 dS tile per (head, query block, list entry): 12 heads,
+    # 24 blocks per frame, 8 more entries per row
+    ws8, ws16 = L.pbsa_bwd_workspace_bytes(gp, 1, 8, 8), L.pbsa_bwd_workspace_bytes(gp, 1, 8, 16)
+    assert ws16 - ws8 >= 12 * 24 * 8 * 8192
 
     # score + top-k: gp, q_reps, nq, k_reps, pool, cand_slot, cand_gid, ncand, k, prefix_slot,
     # prefix_cnt, prefix_ld, out_slot, out_cnt, out_ld, out_score, ws, stream
