@@ -15,17 +15,24 @@
 //    the V blocks, with TMA (128-byte swizzle) into a 3-stage K ring and a 2-stage V ring;
 //    a block that does not exist (odd count) is loaded out of bounds, i.e. zero-filled.
 //    Q is loaded first, before the lists are read.
-//  * Two softmax warpgroups take alternate steps; each has its own TMEM S/P buffer and O
-//    accumulator (TMEM = S0 | S1 | O0 | O1 = 512 columns) and its own MMA issuer warp
-//    (warps 1 and 3, one thread each), so the two chains S -> softmax -> P -> PV -> next S
-//    run independently.  One TMEM lane = one query row per thread; the online softmax
-//    works in the exp2 domain with packed f32x2 arithmetic, writes P (bf16) back over the
-//    S columns it consumed, and the issuer accumulates O_w += P V with the A operand read
-//    from TMEM, then issues the next S = Q K^T of that warpgroup right behind it.
+//  * TMEM holds three S/P buffers and one O accumulator (S0 | S1 | S2 | O = 512 columns);
+//    step i uses S buffer i mod 3.  Two softmax warpgroups take alternate steps; one TMEM
+//    lane = one query row per thread.  The online softmax works in the exp2 domain with
+//    packed f32x2 arithmetic and writes P (bf16) back over the S columns it consumed.
+//  * Warps 1 and 3 issue the MMAs of the even and the odd steps (one thread each; two
+//    issuing threads keep the tensor pipe fuller than one).  Once P(i) is handed over, the
+//    issuer of step i accumulates O += P(i) V(i) with the A operand read from TMEM, then
+//    issues S(i+3) = Q K^T into the buffer P(i) occupied.  S(i+1) and S(i+2) already exist
+//    by then, so a warpgroup never waits for its own PV before its next S: the loop is paced
+//    by the exponentials and the tensor pipe, not by the chain S -> P -> PV -> next S.
+//    PV(i) is issued once PV(i-1) has completed, so O accumulates in step order.
 //  * The warpgroups take turns on the exponentials (the MUFU pipe is as busy as the tensor
-//    pipe), so one warpgroup's exponentials overlap the other's MMAs.
-//  * O_w is rescaled only when its running max grows by more than 2^8; the epilogue
-//    merges the two streams exactly.
+//    pipe), so one warpgroup's exponentials overlap the other's MMAs.  That hand-off also
+//    carries the row's reference maximum (shared memory): O has one reference per row, and
+//    each warpgroup keeps its share of the row sum against the reference it last used.
+//  * O is rescaled (in place, after PV(i-1) has completed) only when the reference grows by
+//    more than 2^8; the epilogue adds the two warpgroups' row sums against the final
+//    reference.
 //  * Register split: the producer/issuer warpgroup runs on 64 registers, the softmax
 //    warpgroups on 216 (setmaxnreg), so the softmax holds its row in registers.
 //  * Each CTA signals programmatic dependents at its start (griddepcontrol.launch_dependents).
@@ -60,16 +67,20 @@ constexpr uint32_t SM_LA = SM_FLAG + MAXL;            // int[512]
 constexpr uint32_t SM_LB = SM_LA + 4 * 512;           // int[512]
 constexpr uint32_t SM_ONLYB = SM_LB + 4 * 512;        // uint8[512]
 constexpr uint32_t SM_STAT = SM_ONLYB + 512;          // float2[2][128] epilogue (m, l) exchange
-constexpr uint32_t SM_BITS = SM_STAT + 2 * 128 * 8;   // uint32[2][BITMAP_SLOTS / 32] list membership
+constexpr uint32_t SM_MREF = SM_STAT + 2 * 128 * 8;   // float[128] running reference max per row
+constexpr uint32_t SM_BITS = SM_MREF + 128 * 4;       // uint32[2][BITMAP_SLOTS / 32] list membership
 constexpr int BITMAP_SLOTS = 8192;                    // pools up to this many slots merge in O(n)
 constexpr uint32_t SM_TOTAL = SM_BITS + 2 * BITMAP_SLOTS / 8;
 constexpr uint32_t SMEM_BYTES = SM_TOTAL + 1024;      // + alignment slack
 
+constexpr int NSBUF = 3;             // S/P buffers in TMEM (O takes the fourth 128 columns)
 enum { B_QFULL = 0, B_KFULL = 1, B_KEMPTY = B_KFULL + KSTAGES, B_VFULL = B_KEMPTY + KSTAGES,
-       B_VEMPTY = B_VFULL + VSTAGES, B_SFULL = B_VEMPTY + VSTAGES,
-       B_PFULL = B_SFULL + 2,      // [warpgroup], 128 arrivals (one per row)
-       B_MMADONE = B_PFULL + 2,
-       B_XDONE = B_MMADONE + 1,    // [warpgroup], 128 arrivals: its exponentials of a step are done
+       B_VEMPTY = B_VFULL + VSTAGES,
+       B_SFULL = B_VEMPTY + VSTAGES,   // [S buffer]
+       B_PFULL = B_SFULL + NSBUF,      // [S buffer], 128 arrivals (one per row)
+       B_PVDONE = B_PFULL + NSBUF,     // [step parity]: PV of that step has completed
+       B_MMADONE = B_PVDONE + 2,
+       B_XDONE = B_MMADONE + 1,        // [warpgroup], 128 arrivals: its exponentials of a step are done
        NUM_BARS = B_XDONE + 2 };
 static_assert(NUM_BARS * 8 <= 256, "barrier area");
 
@@ -120,7 +131,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   // ---------------------------------------------------------------- setup
   if (tid == 0) {
     for (int i = 0; i < NUM_BARS; ++i) mbar_init(&bars[i], 1);
-    for (int i = 0; i < 2; ++i) mbar_init(&bars[B_PFULL + i], 128);
+    for (int i = 0; i < NSBUF; ++i) mbar_init(&bars[B_PFULL + i], 128);
     for (int i = 0; i < 2; ++i) mbar_init(&bars[B_XDONE + i], 128);
     mbar_init(&bars[B_MMADONE], 2);
     *abort_flag = 0;
@@ -153,6 +164,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const bool use_bits = prm.pool_slots <= BITMAP_SLOTS;
   if (use_bits)
     for (int i = tid; i < 2 * BITMAP_SLOTS / 32; i += NTHREADS) bitsA[i] = 0u;
+  float* mref = reinterpret_cast<float*>(sm + SM_MREF);
+  if (tid < 128) mref[tid] = -INFINITY;
   const int* listA = prm.kv_slot + ((size_t)h * prm.nq + rA) * prm.kv_ld;
   const int* listB = prm.kv_slot + ((size_t)h * prm.nq + (hasB ? rB : rA)) * prm.kv_ld;
   int cA = prm.kv_cnt[(size_t)h * prm.nq + rA];
@@ -289,57 +302,63 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
 
   // ---------------------------------------------------------------- MMA issuers
-  // Warp 1 issues the tensor-core work of softmax warpgroup 0 (steps 0, 2, 4, ...), warp 3
-  // that of warpgroup 1 (steps 1, 3, ...), each from one thread, so the two chains
-  // S -> softmax -> P -> PV -> next S never wait on each other's issue.  Warpgroup w owns
-  // TMEM columns [128 w, +128) for S and P and [256 + 128 w, +128) for its O accumulator.
-  // QK(i) into S_w is issued after PV(i-2), which read P(i-2) from the same columns, by
-  // the same thread, so the tensor pipe orders them; and the commit that signals S(i)
-  // also covers PV(i-2), so O_w is never rescaled under a running MMA.
+  // Step i uses S buffer i % 3 (TMEM columns [128 b, +128)); O is one accumulator in columns
+  // [384, 512).  Warp 1 issues the tensor-core work of the even steps, warp 3 that of the
+  // odd ones (one thread each: two issuing threads keep the tensor pipe fuller than one).
+  // Once P(i) is handed over, the issuer of step i issues O += P(i) V(i) and then QK(i+3)
+  // into the buffer P(i) occupied (same thread, so the tensor pipe runs them in that order);
+  // S(i+1) and S(i+2) are computed by then, so no warpgroup's next S waits for its own PV.
+  // PV(i) is issued only once PV(i-1) has completed, so O accumulates in step order (and
+  // every earlier PV has completed when a softmax warpgroup rescales O).
   if (warp == 1 || warp == 3) {
-    const int wg = warp >> 1;
+    const int w = warp >> 1;
     if (lane == 0 && nsteps > 0) {
-      const uint32_t tS = tmem + wg * 128, tO = tmem + 256 + wg * 128;
+      const uint32_t tO = tmem + 384;
       // descriptors of the first 16-element K slice of each operand; a slice further on is
       // the same descriptor plus its byte offset / 16 (the start-address field)
       const uint64_t dq = sw128_desc(smem_u32(sm + SM_Q), 16, 1024);
       const uint64_t dk = sw128_desc(smem_u32(sm + SM_K), 16, 1024);
       const uint64_t dv = sw128_desc(smem_u32(sm + SM_V), 16384, 1024);
-      auto issue_qk = [&](int i) {   // S_w = Q K_i^T, then free the K stage
-        const int sk = i % KSTAGES;
+      auto issue_qk = [&](int i) {   // S_(i mod 3) = Q K_i^T, then free the K stage
+        const int sk = i % KSTAGES, b = i % NSBUF;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
-          mma_bf16_ss(tS, dq + off, dk + ((sk * 32768) >> 4) + off, IDESC_QK, kk > 0 ? 1u : 0u);
+          mma_bf16_ss(tmem + b * 128, dq + off, dk + ((sk * 32768) >> 4) + off, IDESC_QK, kk > 0 ? 1u : 0u);
         }
-        mma_commit(&bars[B_SFULL + wg]);
+        mma_commit(&bars[B_SFULL + b]);
         mma_commit(&bars[B_KEMPTY + sk]);
       };
       wait_or_abort(&bars[B_QFULL], 0, abort_flag, prm.ws, 5);
-      if (wg < nsteps) {
-        wait_or_abort(&bars[B_KFULL + wg % KSTAGES], (wg / KSTAGES) & 1, abort_flag, prm.ws, 6);
-        if (!*abort_flag) {
-          tc_fence_after();
-          issue_qk(wg);
-        }
-      }
-      // Steady state: everything but P(i) is awaited first, so PV(i) and QK(i+2) go to the
-      // tensor pipe back to back once the warpgroup hands over P(i).
-      for (int i = wg; i < nsteps && !*abort_flag; i += 2) {
-        const int sv = i % VSTAGES;
-        const bool more = i + 2 < nsteps;
-        wait_or_abort(&bars[B_VFULL + sv], (i / VSTAGES) & 1, abort_flag, prm.ws, 4);
-        if (more) wait_or_abort(&bars[B_KFULL + (i + 2) % KSTAGES], ((i + 2) / KSTAGES) & 1, abort_flag, prm.ws, 6);
-        wait_or_abort(&bars[B_PFULL + wg], (i >> 1) & 1, abort_flag, prm.ws, 3);
+      // the first three S: steps 0 and 2 from warp 1, step 1 from warp 3
+      for (int j = w; j < NSBUF && j < nsteps; j += 2) {
+        wait_or_abort(&bars[B_KFULL + j % KSTAGES], (j / KSTAGES) & 1, abort_flag, prm.ws, 6);
         if (*abort_flag) break;
         tc_fence_after();
-        // O_w += P_i V_i: P_i (128 rows x 128 keys, bf16 pairs) sits over S_w in TMEM
+        issue_qk(j);
+      }
+      for (int i = w; i < nsteps && !*abort_flag; i += 2) {
+        const int sv = i % VSTAGES, b = i % NSBUF;
+        // PV(i-1) complete first: it also orders the P-ready wait below after P(i-3)'s
+        if (i >= 1) wait_or_abort(&bars[B_PVDONE + ((i - 1) & 1)], ((i - 1) >> 1) & 1, abort_flag, prm.ws, 12);
+        wait_or_abort(&bars[B_VFULL + sv], (i / VSTAGES) & 1, abort_flag, prm.ws, 4);
+        wait_or_abort(&bars[B_PFULL + b], (i / NSBUF) & 1, abort_flag, prm.ws, 3);
+        if (*abort_flag) break;
+        tc_fence_after();
+        // O += P_i V_i: P_i (128 rows x 128 keys, bf16 pairs) sits over S_b in TMEM
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ts(tO, tS + kk * 8, dv + ((sv * 32768 + kk * 2048) >> 4), IDESC_PV,
-                      (i > wg || kk > 0) ? 1u : 0u);
+          mma_bf16_ts(tO, tmem + b * 128 + kk * 8, dv + ((sv * 32768 + kk * 2048) >> 4), IDESC_PV,
+                      (i > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&bars[B_VEMPTY + sv]);
-        if (more) issue_qk(i + 2);
+        mma_commit(&bars[B_PVDONE + (i & 1)]);
+        if (i + NSBUF < nsteps) {
+          wait_or_abort(&bars[B_KFULL + (i + NSBUF) % KSTAGES], ((i + NSBUF) / KSTAGES) & 1, abort_flag,
+                        prm.ws, 6);
+          if (*abort_flag) break;
+          tc_fence_after();
+          issue_qk(i + NSBUF);
+        }
       }
       // every MMA of both issuers has completed once this barrier (count 2) flips
       mma_commit(&bars[B_MMADONE]);
@@ -358,14 +377,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int half = row >> 6;
     const bool row_valid = half == 0 || hasB;
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-    const uint32_t tS = tmem + lane_off + wg * 128;          // S_i / P_i of this warpgroup's steps
-    const uint32_t tO = tmem + lane_off + 256 + wg * 128;
+    const uint32_t tO = tmem + lane_off + 384;
     const float c = prm.scale_log2;
+    // O has one reference maximum per row, mref[row], shared by both warpgroups: step i
+    // reads it after the other warpgroup's step i-1 has published it.  l is this
+    // warpgroup's share of the row sum, expressed against the reference m it last used.
     float m = -INFINITY, l = 0.f;
     for (int i = wg; i < nsteps; i += 2) {
+      const int b = i % NSBUF;
+      const uint32_t tS = tmem + lane_off + b * 128;
       const bool va = row_valid && ((mflag[2 * i] >> half) & 1);
       const bool vb = row_valid && 2 * i + 1 < n && ((mflag[2 * i + 1] >> half) & 1);
-      wait_or_abort(&bars[B_SFULL + wg], (i >> 1) & 1, abort_flag, prm.ws, 7);
+      wait_or_abort(&bars[B_SFULL + b], (i / NSBUF) & 1, abort_flag, prm.ws, 7);
       if (__any_sync(0xffffffffu, *abort_flag != 0)) break;  // warp-uniform exit
       tc_fence_after();
       uint32_t x[4][32];
@@ -392,18 +415,25 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const float mba = va ? fmaxf(mx[0][0], mx[0][1]) : -INFINITY;
       const float mbb = vb ? fmaxf(mx[1][0], mx[1][1]) : -INFINITY;
       const float mb = fmaxf(mba, mbb) * c;
-      float alpha = 1.f;
-      bool rescale_o = false;
-      if (mb > m + 8.0f) {  // also true on the first valid block (m = -inf)
-        rescale_o = (m != -INFINITY) && i > wg;
-        alpha = ex2_approx(m - mb);
-        l *= alpha;
-        m = mb;
-      }
       // The two warpgroups take turns on the exponentials (the MUFU pipe is the scarce unit):
       // step i waits until the other warpgroup has finished those of step i-1, so one
       // warpgroup's exponentials overlap the other's MMAs instead of competing with them.
+      // That wait also makes the reference maximum of step i-1 visible here.
       if (i >= 1) wait_or_abort(&bars[B_XDONE + (wg ^ 1)], ((i - 1) >> 1) & 1, abort_flag, prm.ws, 10);
+      float alpha = 1.f;       // O's rescale factor for this row
+      {
+        const float mcur = mref[row];
+        float mn = mcur;
+        if (mb > mcur + 8.0f) {  // also true on the first valid block (mcur = -inf)
+          if (mcur != -INFINITY) alpha = ex2_approx(mcur - mb);   // O holds earlier steps against mcur
+          mn = mb;
+        }
+        mref[row] = mn;
+        if (mn != m) {         // l in the new reference (l = 0 while m = -inf)
+          l *= ex2_approx(m - mn);
+          m = mn;
+        }
+      }
       // p = 2^(s*c - m) as bf16 pairs over the consumed S columns (32 keys per store).  A
       // masked block uses the factor 0 and the offset -inf, so it gives exact zeros without a
       // branch (x is finite).
@@ -427,10 +457,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
       if (i + 1 < nsteps) mbar_arrive(&bars[B_XDONE + wg]);
-      // PV(i-2), the last MMA into O_w, completed before S(i) was signalled.  tcgen05.ld/st
-      // are warp-collective, so the warp rescales if any of its rows must.
-      if (__any_sync(0xffffffffu, rescale_o)) {
-        if (!rescale_o) alpha = 1.f;
+      // O holds PV(0..i-1) against the reference before this step.  Once PV(i-1) has
+      // completed (PV(i) waits for this warpgroup's P), rows whose reference grew by more
+      // than 2^8 are rescaled in place (alpha = 2^(old - new)).
+      // tcgen05.ld/st are warp-collective, so the warp rescales if any of its rows must.
+      if (__any_sync(0xffffffffu, alpha != 1.f)) {
+        wait_or_abort(&bars[B_PVDONE + ((i - 1) & 1)], ((i - 1) >> 1) & 1, abort_flag, prm.ws, 11);
+        tc_fence_after();
 #pragma unroll 1
         for (int q = 0; q < 4; ++q) {
           uint32_t ov[32];
@@ -443,16 +476,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bars[B_PFULL + wg]);
+      mbar_arrive(&bars[B_PFULL + b]);
     }
-    // epilogue: combine the two streams, O = (O_0 2^(m0-M) + O_1 2^(m1-M)) / L.  The
-    // all-MMAs-done barrier has a single phase, so this wait cannot alias.
+    // epilogue: O is against the final reference M = mref[row]; L = l_0 2^(m_0-M) + l_1 2^(m_1-M).
+    // The all-MMAs-done barrier has a single phase, so this wait cannot alias.
     if (nsteps > 0) wait_or_abort(&bars[B_MMADONE], 0, abort_flag, prm.ws, 9);
     float2* stat = reinterpret_cast<float2*>(sm + SM_STAT);
     stat[wg * 128 + row] = make_float2(m, l);
     asm volatile("bar.sync 1, 256;" ::: "memory");   // both softmax warpgroups, every path
     const float2 st0 = stat[row], st1 = stat[128 + row];
-    const float M = fmaxf(st0.x, st1.x);
+    const float M = mref[row];
     const float f0 = st0.x == -INFINITY ? 0.f : ex2_approx(st0.x - M);
     const float f1 = st1.x == -INFINITY ? 0.f : ex2_approx(st1.x - M);
     const float Lsum = st0.y * f0 + st1.y * f1;
@@ -464,15 +497,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const size_t t = (size_t)f * prm.tpf + (size_t)(ty * prm.th + ly) * prm.fw + tx * prm.tw + lx;
       uint4* dst = reinterpret_cast<uint4*>(prm.o + (t * prm.H + h) * D) + wg * 8;
       const float inv = Lsum > 0.f ? 1.0f / Lsum : 0.f;
-      const float g0 = f0 * inv, g1 = f1 * inv;
       tc_fence_after();
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
-        uint32_t oa[32], ob[32];
+        uint32_t oa[32];
 #pragma unroll
-        for (int e2 = 0; e2 < 32; ++e2) oa[e2] = ob[e2] = 0u;
-        if (nsteps > 0) tmem_ld32(tmem + lane_off + 256 + wg * 64 + q * 32, oa);
-        if (nsteps > 1) tmem_ld32(tmem + lane_off + 384 + wg * 64 + q * 32, ob);   // O_1 is written from step 1 on
+        for (int e2 = 0; e2 < 32; ++e2) oa[e2] = 0u;
+        if (nsteps > 0) tmem_ld32(tO + wg * 64 + q * 32, oa);
         tmem_wait_ld();
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
@@ -480,8 +511,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
           for (int e2 = 0; e2 < 4; ++e2) {
             const int k0 = cc * 8 + 2 * e2;
-            wv[e2] = pack_bf16(__uint_as_float(oa[k0]) * g0 + __uint_as_float(ob[k0]) * g1,
-                               __uint_as_float(oa[k0 + 1]) * g0 + __uint_as_float(ob[k0 + 1]) * g1);
+            wv[e2] = pack_bf16(__uint_as_float(oa[k0]) * inv, __uint_as_float(oa[k0 + 1]) * inv);
           }
           dst[q * 4 + cc] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
         }
