@@ -437,6 +437,37 @@ def test_attend_bf16_running_max_grows():
     assert jumps > 100
 
 
+def test_attend_bf16_short_lists():
+    """Merged lists of 0 to 5 steps (128 keys each): fewer steps than the kernel's three S
+    buffers, exactly three, and more, so the first S of each buffer, the last PV and the
+    hand-offs between the two softmax streams are exercised at each count.  The two query
+    blocks of a pair attend disjoint blocks (one sometimes nothing), so the merged list, its
+    masks and the odd last step differ from either list."""
+    w = dataclasses.replace(I.DECODE_5S, heads=2, frame_h=8, frame_w=64)   # 8 query blocks, 4 pairs
+    nq, slots = w.blocks_per_frame, 40
+    rng = np.random.default_rng(23)
+    # (|A|, |B|) per pair, disjoint lists: merged lengths 0, 1, 2, 3, 5, 6, 7, 9 -> 0 to 5 steps
+    sizes = [(0, 0), (1, 0), (1, 1), (2, 1), (3, 2), (0, 6), (4, 3), (5, 4)]
+    lists = []
+    for h in range(w.heads):
+        rows = []
+        for p in range(nq // 2):
+            na, nb = sizes[h * (nq // 2) + p]
+            perm = rng.permutation(slots).tolist()
+            rows += [perm[:na], perm[na:na + nb]]
+        lists.append(rows)
+    q, kp, vp, kv, cnt, ld = _attend_case(w, 1, slots, lists, 29)
+    o, lse = _run_attend(w, q, 1, kp, vp, kv, cnt, ld)
+    for h in range(w.heads):
+        for r in range(nq):
+            rows, (want, wlse) = _oracle_unit(w, q, kp, vp, h, r, lists[h][r])
+            assert_bf16_close(f64(o[rows, h]), want, f"h{h} r{r}")
+            if lists[h][r]:
+                np.testing.assert_allclose(f64(lse[h, rows]), wlse, rtol=0, atol=2e-3)
+            else:
+                assert np.isneginf(f64(lse[h, rows])).all()
+
+
 @pytest.mark.parametrize("case", ["pool_above_bitmap", "merged_list_at_capacity"])
 def test_attend_bf16_list_merge_limits(case):
     """The pair's list merge at its limits: a pool of more slots than the membership bitmaps
