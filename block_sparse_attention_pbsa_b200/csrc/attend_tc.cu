@@ -127,6 +127,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int h = blockIdx.y;
   const int rA = 2 * blockIdx.x, rB = rA + 1;
   const bool hasB = rB < prm.nq;
+  // The two lists are read first (at most 512 entries each: two per thread), before any set-up,
+  // so their global loads are in flight while the barriers, Q's copy and TMEM are set up.
+  static_assert(2 * NTHREADS >= 512, "two list entries per thread");
+  const int* listA = prm.kv_slot + ((size_t)h * prm.nq + rA) * prm.kv_ld;
+  const int* listB = prm.kv_slot + ((size_t)h * prm.nq + (hasB ? rB : rA)) * prm.kv_ld;
+  int cA = prm.kv_cnt[(size_t)h * prm.nq + rA];
+  int cB = hasB ? prm.kv_cnt[(size_t)h * prm.nq + rB] : 0;
+  int la0 = 0, lb0 = 0, la1 = 0, lb1 = 0;
+  if (tid < prm.kv_ld) { la0 = listA[tid]; lb0 = listB[tid]; }
+  if (tid + NTHREADS < prm.kv_ld) { la1 = listA[tid + NTHREADS]; lb1 = listB[tid + NTHREADS]; }
 
   // ---------------------------------------------------------------- setup
   if (tid == 0) {
@@ -166,14 +176,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     for (int i = tid; i < 2 * BITMAP_SLOTS / 32; i += NTHREADS) bitsA[i] = 0u;
   float* mref = reinterpret_cast<float*>(sm + SM_MREF);
   if (tid < 128) mref[tid] = -INFINITY;
-  const int* listA = prm.kv_slot + ((size_t)h * prm.nq + rA) * prm.kv_ld;
-  const int* listB = prm.kv_slot + ((size_t)h * prm.nq + (hasB ? rB : rA)) * prm.kv_ld;
-  int cA = prm.kv_cnt[(size_t)h * prm.nq + rA];
-  int cB = hasB ? prm.kv_cnt[(size_t)h * prm.nq + rB] : 0;
-  for (int i = tid; i < prm.kv_ld; i += NTHREADS) {
-    la[i] = listA[i];
-    lb[i] = listB[i];
-  }
+  if (tid < prm.kv_ld) { la[tid] = la0; lb[tid] = lb0; }
+  if (tid + NTHREADS < prm.kv_ld) { la[tid + NTHREADS] = la1; lb[tid + NTHREADS] = lb1; }
   if (cA < 0 || cA > prm.kv_ld || cB < 0 || cB > prm.kv_ld) {
     if (tid == 0) record_error(prm.ws, PBSA_ERR_DEVICE_INDEX, cA < 0 || cA > prm.kv_ld ? cA : cB, K_ATTEND_TC);
     cA = min(max(cA, 0), prm.kv_ld);
