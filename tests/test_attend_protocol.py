@@ -16,26 +16,9 @@ import random
 
 import pytest
 
+from tests._protocol import Bar, run_actors, wait_for, wait_released
+
 KSTAGES, VSTAGES, NSBUF = 3, 2, 3
-
-
-class Bar:
-    """An mbarrier: `count` arrivals complete a phase; `done` = completed phases."""
-
-    def __init__(self, name, count):
-        self.name, self.count, self.arrived, self.done = name, count, 0, 0
-
-    def arrive(self, n=1):
-        self.arrived += n
-        assert self.arrived <= self.count, f"{self.name}: too many arrivals in one phase"
-        if self.arrived == self.count:
-            self.arrived = 0
-            self.done += 1
-
-    def passes(self, parity):
-        # try_wait.parity passes once the phase of that parity has completed: the current
-        # (incomplete) phase has the other parity
-        return (self.done & 1) != parity
 
 
 class Sim:
@@ -67,20 +50,11 @@ class Sim:
         self.completed = {0: 0, 1: 0}      # batches completed per issuer
         self.loads = []                    # in-flight TMA loads: (barrier, kind, stage, step)
 
-    # -- waits: a generator yields a predicate; the check runs when it passes
     def wait(self, bar, n):
-        """Wait for completion n (0-based) of `bar`, as the kernel does with parity n & 1;
-        assert that exactly completions 0..n have happened when the wait passes."""
-        b = self.B[bar]
-        yield lambda: b.passes(n & 1)
-        assert b.done == n + 1, f"{bar}: wait for completion {n} passed with {b.done} completions"
+        yield from wait_for(self.B[bar], n)
 
     def wait_free(self, bar, n):
-        """Producer-side wait for completion n-1 of an 'empty' barrier (n = use index; the first
-        use of a stage passes at once on the fresh barrier's previous-phase parity)."""
-        b = self.B[bar]
-        yield lambda: b.passes((n & 1) ^ 1)
-        assert b.done == n, f"{bar}: use {n} started after {b.done} releases"
+        yield from wait_released(self.B[bar], n)
 
     def issue(self, who, kind, step):
         self.pipe[who].append((kind, step))
@@ -162,10 +136,10 @@ class Sim:
 
     # -- the tensor pipe (each issuing thread's MMAs in its issue order; no order between the
     # two threads) and the copy engine, stepped by the scheduler
-    def pipe_step(self):
+    def pipe_step(self, probe=False):
         busy = [w for w in (0, 1) if self.pipe[w]]
-        if not busy:
-            return False
+        if probe or not busy:
+            return bool(busy)
         who = self.rng.choice(busy)
         kind, i = self.pipe[who].pop(0)
         b = i % NSBUF
@@ -190,9 +164,9 @@ class Sim:
         self.pending_commits = keep
         return True
 
-    def load_step(self):
-        if not self.loads:
-            return False
+    def load_step(self, probe=False):
+        if probe or not self.loads:
+            return bool(self.loads)
         bar, kind, s, i = self.loads.pop(self.rng.randrange(len(self.loads)))
         (self.kst if kind == "k" else self.vst)[s] = i
         self.B[bar].arrive()
@@ -208,30 +182,10 @@ class Sim:
                 keep.append(c)
         self.pending_commits = keep
 
-    def run(self, max_events=2_000_000):
+    def run(self):
         actors = [self.k_producer(), self.v_producer(), self.issuer(0), self.issuer(1)]
         actors += [self.warp(wg, wq) for wg in (0, 1) for wq in range(4)]
-        waiting = {k: None for k in range(len(actors))}
-        live = set(range(len(actors)))
-        for _ in range(max_events):
-            self.commits_without_mmas()
-            ready = [k for k in live if waiting[k] is None or waiting[k]()]
-            choices = ready + (["pipe"] if self.pipe[0] or self.pipe[1] else []) + (["load"] if self.loads else [])
-            if not choices:
-                assert not live, f"deadlock: {len(live)} actors blocked"
-                return
-            c = self.rng.choice(choices)
-            if c == "pipe":
-                self.pipe_step()
-            elif c == "load":
-                self.load_step()
-            else:
-                try:
-                    waiting[c] = next(actors[c])
-                except StopIteration:
-                    live.discard(c)
-                    waiting[c] = None
-        raise AssertionError("no progress bound reached")
+        run_actors(actors, [self.pipe_step, self.load_step], self.rng, before_step=self.commits_without_mmas)
 
 
 @pytest.mark.parametrize("nsteps", [0, 1, 2, 3, 4, 5, 7, 12, 40])
